@@ -1,0 +1,289 @@
+"""Python binding of liblgattn.so -- the LongGen sparse-attention hot path on B200.
+
+Argument marshalling only: every function below checks tensor dtypes, shapes
+and devices, converts them to raw pointers and calls the C entry point of the
+same name (include/lg_attn.h). All computation happens in the CUDA kernels of
+the library; there is no fallback. Importing works without a GPU; any call
+into the library raises if ``liblgattn.so`` has not been built.
+
+Method: "A Little Goes a Long Way: Efficient Long Context Training and
+Inference with Partial Contexts" (LongGen, arXiv 2410.01485) -- sparse layers
+with attention-sink / window / strided-block static patterns, full-attention
+middle layers, decode over the reduced KV cache.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import NamedTuple, Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "liblgattn.so")
+INT32_MAX = 2**31 - 1
+
+__all__ = [
+    "LgError", "Pattern", "lib", "lg_strerror", "lg_version",
+    "lg_pattern_expand", "lg_pattern_expand_t", "lg_pattern_pairs", "lg_pattern_iterate_device",
+    "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd",
+    "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd",
+    "lg_sparse_decode_splits", "lg_sparse_decode_workspace", "lg_sparse_decode",
+    "lg_device_status", "EXPORTED_SYMBOLS",
+]
+
+EXPORTED_SYMBOLS = (
+    "lg_strerror", "lg_version", "lg_pattern_expand", "lg_pattern_expand_t", "lg_pattern_pairs",
+    "lg_pattern_iterate_device", "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd",
+    "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd", "lg_sparse_decode_splits",
+    "lg_sparse_decode_workspace", "lg_sparse_decode", "lg_device_status",
+)
+
+
+class Pattern(NamedTuple):
+    """{block_size, sink_blocks, local_blocks, stride}; stride 0 = no strided term."""
+
+    block_size: int
+    sink_blocks: int
+    local_blocks: int
+    stride: int = 0
+
+    @staticmethod
+    def full(block_size: int = 64) -> "Pattern":
+        return Pattern(block_size, 0, INT32_MAX, 0)
+
+
+class _lg_pattern_t(ctypes.Structure):
+    _fields_ = [("block_size", ctypes.c_int32), ("sink_blocks", ctypes.c_int32),
+                ("local_blocks", ctypes.c_int32), ("stride", ctypes.c_int32)]
+
+
+class LgError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lg_strerror(status)} (status {status})")
+
+
+_c_i32, _c_i64, _c_sz, _c_vp, _c_f = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
+_P = ctypes.POINTER
+_SIGS = {
+    "lg_strerror": (ctypes.c_char_p, [_c_i32]),
+    "lg_version": (_c_i32, []),
+    "lg_pattern_expand": (_c_i32, [_P(_lg_pattern_t), _c_i32, _P(_c_i32), _P(_c_i32), _c_i64, _P(_c_i64)]),
+    "lg_pattern_expand_t": (_c_i32, [_P(_lg_pattern_t), _c_i32, _P(_c_i32), _P(_c_i32), _c_i64, _P(_c_i64)]),
+    "lg_pattern_pairs": (_c_i32, [_P(_lg_pattern_t), _c_i32, _P(_c_i64)]),
+    "lg_pattern_iterate_device": (_c_i32, [_P(_lg_pattern_t), _c_i32, _c_i32, _c_i32, _c_vp, _c_i32, _c_vp]),
+    "lg_sparse_attn_fwd_workspace": (_c_i32, [_P(_lg_pattern_t)] + [_c_i32] * 5 + [_P(_c_sz)]),
+    "lg_sparse_attn_fwd": (_c_i32, [_P(_lg_pattern_t), _c_vp, _c_vp, _c_vp, _c_vp, _c_vp] + [_c_i32] * 5
+                           + [_c_f, _c_vp, _c_sz, _c_vp]),
+    "lg_sparse_attn_bwd_workspace": (_c_i32, [_P(_lg_pattern_t)] + [_c_i32] * 5 + [_P(_c_sz)]),
+    "lg_sparse_attn_bwd": (_c_i32, [_P(_lg_pattern_t)] + [_c_vp] * 9 + [_c_i32] * 5 + [_c_f, _c_vp, _c_sz, _c_vp]),
+    "lg_sparse_decode_splits": (_c_i32, [_c_i32] * 6 + [_P(_c_i32)]),
+    "lg_sparse_decode_workspace": (_c_i32, [_c_i32] * 6 + [_P(_c_sz)]),
+    "lg_sparse_decode": (_c_i32, [_c_vp] * 6 + [_c_i32] * 6 + [_c_f, _c_vp, _c_sz, _c_vp]),
+    "lg_device_status": (_c_i32, [_c_i32, _P(ctypes.c_uint32)]),
+}
+
+_lib = None
+
+
+def lib():
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m attention_sink_long_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise LgError(status, where)
+
+
+def _pat(p) -> _lg_pattern_t:
+    return _lg_pattern_t(int(p[0]), int(p[1]), int(p[2]), int(p[3]) if len(p) > 3 else 0)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+    return int(getattr(stream, "cuda_stream", stream))
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _expect(t, name, dtype, shape, device=None):
+    import torch
+
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name}: expected device {device}, got {t.device}")
+    return torch
+
+
+def lg_strerror(status: int) -> str:
+    return lib().lg_strerror(int(status)).decode()
+
+
+def lg_version() -> int:
+    return int(lib().lg_version())
+
+
+# ---------------------------------------------------------------- pattern
+def lg_pattern_expand(pattern, seqlen: int):
+    """CSR (row_ptr, col) as int32 numpy arrays."""
+    import numpy as np
+
+    p = _pat(pattern)
+    nnz = _c_i64(0)
+    _check(lib().lg_pattern_expand(ctypes.byref(p), seqlen, None, None, 0, ctypes.byref(nnz)), "lg_pattern_expand")
+    nqb = seqlen // p.block_size
+    row_ptr = np.zeros(nqb + 1, dtype=np.int32)
+    col = np.zeros(max(nnz.value, 1), dtype=np.int32)
+    _check(lib().lg_pattern_expand(ctypes.byref(p), seqlen, row_ptr.ctypes.data_as(_P(_c_i32)),
+                                   col.ctypes.data_as(_P(_c_i32)), col.size, ctypes.byref(nnz)), "lg_pattern_expand")
+    return row_ptr, col[: nnz.value]
+
+
+def lg_pattern_expand_t(pattern, seqlen: int):
+    """CSC (col_ptr, row) as int32 numpy arrays."""
+    import numpy as np
+
+    p = _pat(pattern)
+    nnz = _c_i64(0)
+    _check(lib().lg_pattern_expand_t(ctypes.byref(p), seqlen, None, None, 0, ctypes.byref(nnz)),
+           "lg_pattern_expand_t")
+    nqb = seqlen // p.block_size
+    col_ptr = np.zeros(nqb + 1, dtype=np.int32)
+    row = np.zeros(max(nnz.value, 1), dtype=np.int32)
+    _check(lib().lg_pattern_expand_t(ctypes.byref(p), seqlen, col_ptr.ctypes.data_as(_P(_c_i32)),
+                                     row.ctypes.data_as(_P(_c_i32)), row.size, ctypes.byref(nnz)),
+           "lg_pattern_expand_t")
+    return col_ptr, row[: nnz.value]
+
+
+def lg_pattern_pairs(pattern, seqlen: int) -> int:
+    p = _pat(pattern)
+    out = _c_i64(0)
+    _check(lib().lg_pattern_pairs(ctypes.byref(p), seqlen, ctypes.byref(out)), "lg_pattern_pairs")
+    return out.value
+
+
+def lg_pattern_iterate_device(pattern, seqlen: int, tile_blocks: int, transpose: int, out, cap: int, stream=None):
+    """Runs the kernels' block iterator on the device into ``out`` (int32 CUDA tensor)."""
+    p = _pat(pattern)
+    _check(lib().lg_pattern_iterate_device(ctypes.byref(p), seqlen, tile_blocks, transpose, out.data_ptr(), cap,
+                                           _stream(stream)), "lg_pattern_iterate_device")
+
+
+# ---------------------------------------------------------------- forward
+def lg_sparse_attn_fwd_workspace(pattern, B, S, H, Hkv, D) -> int:
+    p = _pat(pattern)
+    n = _c_sz(0)
+    _check(lib().lg_sparse_attn_fwd_workspace(ctypes.byref(p), B, S, H, Hkv, D, ctypes.byref(n)),
+           "lg_sparse_attn_fwd_workspace")
+    return n.value
+
+
+def lg_sparse_attn_fwd(pattern, q, k, v, o, lse, scale: float, workspace=None, stream=None):
+    """q [B,S,H,D], k/v [B,S,Hkv,D], o [B,S,H,D] bf16 CUDA tensors; lse [B,H,S] fp32 or None."""
+    import torch
+
+    B, S, H, D = q.shape
+    Hkv = k.shape[2]
+    _expect(q, "q", torch.bfloat16, (B, S, H, D))
+    _expect(k, "k", torch.bfloat16, (B, S, Hkv, D), q.device)
+    _expect(v, "v", torch.bfloat16, (B, S, Hkv, D), q.device)
+    _expect(o, "o", torch.bfloat16, (B, S, H, D), q.device)
+    if lse is not None:
+        _expect(lse, "lse", torch.float32, (B, H, S), q.device)
+    p = _pat(pattern)
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().lg_sparse_attn_fwd(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                    _ptr(lse), B, S, H, Hkv, D, float(scale), _ptr(workspace), ws, _stream(stream)),
+           "lg_sparse_attn_fwd")
+
+
+# ---------------------------------------------------------------- backward
+def lg_sparse_attn_bwd_workspace(pattern, B, S, H, Hkv, D) -> int:
+    p = _pat(pattern)
+    n = _c_sz(0)
+    _check(lib().lg_sparse_attn_bwd_workspace(ctypes.byref(p), B, S, H, Hkv, D, ctypes.byref(n)),
+           "lg_sparse_attn_bwd_workspace")
+    return n.value
+
+
+def lg_sparse_attn_bwd(pattern, q, k, v, o, dout, lse, dq, dk, dv, scale: float, workspace, stream=None):
+    """Gradients; dq/dk/dv bf16 outputs shaped like q/k/v; workspace a CUDA uint8 tensor."""
+    import torch
+
+    B, S, H, D = q.shape
+    Hkv = k.shape[2]
+    for name, t, shp in (("q", q, (B, S, H, D)), ("o", o, (B, S, H, D)), ("dout", dout, (B, S, H, D)),
+                         ("dq", dq, (B, S, H, D)), ("k", k, (B, S, Hkv, D)), ("v", v, (B, S, Hkv, D)),
+                         ("dk", dk, (B, S, Hkv, D)), ("dv", dv, (B, S, Hkv, D))):
+        _expect(t, name, torch.bfloat16, shp, q.device)
+    _expect(lse, "lse", torch.float32, (B, H, S), q.device)
+    p = _pat(pattern)
+    ws = workspace.numel() * workspace.element_size()
+    _check(lib().lg_sparse_attn_bwd(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                    dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                    B, S, H, Hkv, D, float(scale), workspace.data_ptr(), ws, _stream(stream)),
+           "lg_sparse_attn_bwd")
+
+
+# ---------------------------------------------------------------- decode
+def lg_sparse_decode_splits(B, H, Hkv, D, Lmax, num_splits=0) -> int:
+    n = _c_i32(0)
+    _check(lib().lg_sparse_decode_splits(B, H, Hkv, D, Lmax, num_splits, ctypes.byref(n)), "lg_sparse_decode_splits")
+    return n.value
+
+
+def lg_sparse_decode_workspace(B, H, Hkv, D, Lmax, num_splits=0) -> int:
+    n = _c_sz(0)
+    _check(lib().lg_sparse_decode_workspace(B, H, Hkv, D, Lmax, num_splits, ctypes.byref(n)),
+           "lg_sparse_decode_workspace")
+    return n.value
+
+
+def lg_sparse_decode(q, k_cache, v_cache, cache_lens, o, lse, scale: float, num_splits: int = 0, workspace=None,
+                     stream=None):
+    """q [B,H,D] bf16, caches [B,Lmax,Hkv,D] bf16, cache_lens [B] int32, o [B,H,D] bf16, lse [B,H] fp32 or None."""
+    import torch
+
+    B, H, D = q.shape
+    Lmax, Hkv = k_cache.shape[1], k_cache.shape[2]
+    _expect(q, "q", torch.bfloat16, (B, H, D))
+    _expect(k_cache, "k_cache", torch.bfloat16, (B, Lmax, Hkv, D), q.device)
+    _expect(v_cache, "v_cache", torch.bfloat16, (B, Lmax, Hkv, D), q.device)
+    _expect(cache_lens, "cache_lens", torch.int32, (B,), q.device)
+    _expect(o, "o", torch.bfloat16, (B, H, D), q.device)
+    if lse is not None:
+        _expect(lse, "lse", torch.float32, (B, H), q.device)
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().lg_sparse_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), cache_lens.data_ptr(),
+                                  o.data_ptr(), _ptr(lse), B, H, Hkv, D, Lmax, int(num_splits), float(scale),
+                                  _ptr(workspace), ws, _stream(stream)), "lg_sparse_decode")
+
+
+# ---------------------------------------------------------------- diagnostics
+def lg_device_status(device: int = 0) -> int:
+    """Reads and clears the device error flags (synchronises the device)."""
+    f = ctypes.c_uint32(0)
+    _check(lib().lg_device_status(int(device), ctypes.byref(f)), "lg_device_status")
+    return f.value

@@ -1,0 +1,401 @@
+// api.cu -- the extern "C" boundary (include/lg_attn.h): argument validation,
+// workspace sizing, TMA tensor-map construction and kernel launches.
+// Nothing here allocates or frees device memory or synchronises a stream,
+// except lg_device_status, which says so.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "lg_kernels.h"
+#include "lg_pattern.cuh"
+
+// Device error word written by bounded waits that ran out (see lg_device_status).
+__device__ unsigned int g_lg_error_word;
+
+namespace {
+
+using lg::imin;
+
+constexpr int kMaxDevices = 64;
+
+lg_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? LG_OK : LG_ERR_CUDA; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+lg_status_t check_pattern(const lg_pattern_t* p) {
+  if (p == nullptr) return LG_ERR_INVALID_ARG;
+  if (p->block_size <= 0 || p->sink_blocks < 0 || p->local_blocks < 1 || p->stride < 0) return LG_ERR_INVALID_ARG;
+  return LG_OK;
+}
+
+lg_status_t check_prefill_shape(const lg_pattern_t* p, int B, int S, int H, int Hkv, int D) {
+  lg_status_t st = check_pattern(p);
+  if (st != LG_OK) return st;
+  if (B <= 0 || S <= 0 || H <= 0 || Hkv <= 0 || D <= 0) return LG_ERR_INVALID_ARG;
+  if (H % Hkv != 0) return LG_ERR_INVALID_ARG;
+  if (p->block_size != 64) return LG_ERR_UNSUPPORTED;
+  if (S % 64 != 0) return LG_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128) return LG_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535) return LG_ERR_UNSUPPORTED;
+  return LG_OK;
+}
+
+// Device error word address, resolved once per device with that device current.
+unsigned int* error_word(lg_status_t* st) {
+  static std::mutex mu;
+  static unsigned int* addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *st = LG_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_lg_error_word) != cudaSuccess) {
+      *st = LG_ERR_CUDA;
+      return nullptr;
+    }
+    addr[dev] = static_cast<unsigned int*>(p);
+  }
+  *st = LG_OK;
+  return addr[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// 4-D bf16 tensor map over a contiguous [B, S, Hx, D] tensor: dims {D, Hx, S, B};
+// box {64, 1, rows, 1} with 128-byte swizzle, i.e. one [rows x 64] panel.
+lg_status_t make_map(CUtensorMap* m, const void* base, int B, int S, int Hx, int D, int rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (enc == nullptr) return LG_ERR_CUDA;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)Hx, (cuuint64_t)S, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)Hx * D * 2, (cuuint64_t)S * Hx * D * 2};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LG_OK : LG_ERR_CUDA;
+}
+
+// Decode split rule: about 256 KB of K+V per CTA, more splits when there are
+// too few (b, kv head) rows to fill the GPU.
+void decode_split_rule(int B, int Hkv, int D, int Lmax, int requested, int* ns_out, int* rps_out) {
+  int rps, ns;
+  if (requested > 0) {
+    ns = imin(requested, Lmax);
+    rps = (Lmax + ns - 1) / ns;
+  } else {
+    rps = (D == 128) ? 512 : 1024;
+    ns = (Lmax + rps - 1) / rps;
+    while (rps > 64 && (long long)B * Hkv * ns < 148LL * 8) {
+      rps /= 2;
+      ns = (Lmax + rps - 1) / rps;
+    }
+  }
+  if (ns < 1) ns = 1;
+  rps = (Lmax + ns - 1) / ns;
+  ns = (Lmax + rps - 1) / rps;
+  *ns_out = ns;
+  *rps_out = rps;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+extern "C" {
+
+const char* lg_strerror(lg_status_t s) {
+  switch (s) {
+    case LG_OK: return "ok";
+    case LG_ERR_INVALID_ARG: return "invalid argument";
+    case LG_ERR_UNSUPPORTED: return "unsupported shape, pattern or alignment";
+    case LG_ERR_WORKSPACE: return "workspace missing or too small";
+    case LG_ERR_CUDA: return "CUDA error";
+    case LG_ERR_INTERNAL: return "internal error";
+    case LG_ERR_CAPACITY: return "output capacity too small";
+  }
+  return "unknown status";
+}
+
+int32_t lg_version(void) { return (1 << 16) | 0; }
+
+// ---------------------------------------------------------------- pattern (host)
+lg_status_t lg_pattern_expand(const lg_pattern_t* p, int32_t seqlen, int32_t* row_ptr, int32_t* col, int64_t cap,
+                              int64_t* nnz) {
+  lg_status_t st = check_pattern(p);
+  if (st != LG_OK) return st;
+  if (nnz == nullptr || seqlen <= 0 || seqlen % p->block_size != 0) return LG_ERR_INVALID_ARG;
+  const int nqb = seqlen / p->block_size;
+  int64_t total = 0;
+  for (int i = 0; i < nqb; ++i) total += lg::KvIter(*p, i, i).count();
+  *nnz = total;
+  if (col == nullptr) return LG_OK;
+  if (row_ptr == nullptr) return LG_ERR_INVALID_ARG;
+  if (cap < total) return LG_ERR_CAPACITY;
+  int64_t e = 0;
+  for (int i = 0; i < nqb; ++i) {
+    row_ptr[i] = (int32_t)e;
+    const lg::KvIter it(*p, i, i);
+    for (int j = it.first(); j >= 0; j = it.next(j)) col[e++] = j;
+  }
+  row_ptr[nqb] = (int32_t)e;
+  return e == total ? LG_OK : LG_ERR_INTERNAL;
+}
+
+lg_status_t lg_pattern_expand_t(const lg_pattern_t* p, int32_t seqlen, int32_t* col_ptr, int32_t* row, int64_t cap,
+                                int64_t* nnz) {
+  lg_status_t st = check_pattern(p);
+  if (st != LG_OK) return st;
+  if (nnz == nullptr || seqlen <= 0 || seqlen % p->block_size != 0) return LG_ERR_INVALID_ARG;
+  const int nqb = seqlen / p->block_size;
+  int64_t total = 0;
+  for (int j = 0; j < nqb; ++j) total += lg::QIter(*p, j, j, nqb).count();
+  *nnz = total;
+  if (row == nullptr) return LG_OK;
+  if (col_ptr == nullptr) return LG_ERR_INVALID_ARG;
+  if (cap < total) return LG_ERR_CAPACITY;
+  int64_t e = 0;
+  for (int j = 0; j < nqb; ++j) {
+    col_ptr[j] = (int32_t)e;
+    const lg::QIter it(*p, j, j, nqb);
+    for (int i = it.first_blk; i <= it.last_blk; ++i) row[e++] = i;
+  }
+  col_ptr[nqb] = (int32_t)e;
+  return e == total ? LG_OK : LG_ERR_INTERNAL;
+}
+
+lg_status_t lg_pattern_pairs(const lg_pattern_t* p, int32_t seqlen, int64_t* pairs) {
+  lg_status_t st = check_pattern(p);
+  if (st != LG_OK) return st;
+  if (pairs == nullptr || seqlen <= 0 || seqlen % p->block_size != 0) return LG_ERR_INVALID_ARG;
+  const int64_t b = p->block_size;
+  const int nqb = seqlen / p->block_size;
+  int64_t total = 0;
+  // Every listed block below the diagonal is fully visible; the diagonal is causal.
+  for (int i = 0; i < nqb; ++i) total += (int64_t)(lg::KvIter(*p, i, i).count() - 1) * b * b + b * (b + 1) / 2;
+  *pairs = total;
+  return LG_OK;
+}
+
+lg_status_t lg_pattern_iterate_device(const lg_pattern_t* p, int32_t seqlen, int32_t tile_blocks, int32_t transpose,
+                                      int32_t* out, int32_t cap, lg_stream_t stream) {
+  lg_status_t st = check_pattern(p);
+  if (st != LG_OK) return st;
+  if (out == nullptr || seqlen <= 0 || seqlen % p->block_size != 0 || cap < 0) return LG_ERR_INVALID_ARG;
+  if (tile_blocks != 1 && tile_blocks != 2) return LG_ERR_UNSUPPORTED;
+  if (transpose != 0 && transpose != 1) return LG_ERR_INVALID_ARG;
+  return cuda_status(
+      lg::launch_pattern_iterate(*p, seqlen, tile_blocks, transpose, out, cap, static_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------- forward
+lg_status_t lg_sparse_attn_fwd_workspace(const lg_pattern_t* p, int32_t B, int32_t S, int32_t H, int32_t Hkv,
+                                         int32_t D, size_t* bytes) {
+  lg_status_t st = check_prefill_shape(p, B, S, H, Hkv, D);
+  if (st != LG_OK) return st;
+  if (bytes == nullptr) return LG_ERR_INVALID_ARG;
+  *bytes = 0;
+  return LG_OK;
+}
+
+lg_status_t lg_sparse_attn_fwd(const lg_pattern_t* p, const void* q, const void* k, const void* v, void* o,
+                               float* lse, int32_t B, int32_t S, int32_t H, int32_t Hkv, int32_t D, float scale,
+                               void* workspace, size_t workspace_bytes, lg_stream_t stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  lg_status_t st = check_prefill_shape(p, B, S, H, Hkv, D);
+  if (st != LG_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return LG_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return LG_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return LG_ERR_UNSUPPORTED;
+  unsigned int* err = error_word(&st);
+  if (st != LG_OK) return st;
+  CUtensorMap tq, tk, tv, to;
+  if ((st = make_map(&tq, q, B, S, H, D, 128)) != LG_OK) return st;
+  if ((st = make_map(&tk, k, B, S, Hkv, D, 64)) != LG_OK) return st;
+  if ((st = make_map(&tv, v, B, S, Hkv, D, 64)) != LG_OK) return st;
+  if ((st = make_map(&to, o, B, S, H, D, 128)) != LG_OK) return st;
+  lg::FwdParams prm;
+  prm.pat = *p;
+  prm.lse = lse;
+  prm.S = S;
+  prm.H = H;
+  prm.Hkv = Hkv;
+  prm.nqb = S / 64;
+  prm.nqt = (S + 127) / 128;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.err = err;
+  return cuda_status(lg::launch_fwd(D, tq, tk, tv, to, prm, B, static_cast<cudaStream_t>(stream)));
+}
+
+// ---------------------------------------------------------------- backward
+lg_status_t lg_sparse_attn_bwd_workspace(const lg_pattern_t* p, int32_t B, int32_t S, int32_t H, int32_t Hkv,
+                                         int32_t D, size_t* bytes) {
+  lg_status_t st = check_prefill_shape(p, B, S, H, Hkv, D);
+  if (st != LG_OK) return st;
+  if (bytes == nullptr) return LG_ERR_INVALID_ARG;
+  *bytes = round256((size_t)B * H * S * D * sizeof(float)) + round256((size_t)B * H * S * sizeof(float));
+  return LG_OK;
+}
+
+lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* p, const void* q, const void* k, const void* v, const void* o,
+                               const void* dout, const float* lse, void* dq, void* dk, void* dv, int32_t B, int32_t S,
+                               int32_t H, int32_t Hkv, int32_t D, float scale, void* workspace,
+                               size_t workspace_bytes, lg_stream_t stream) {
+  lg_status_t st = check_prefill_shape(p, B, S, H, Hkv, D);
+  if (st != LG_OK) return st;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return LG_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return LG_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return LG_ERR_UNSUPPORTED;
+  size_t need = 0;
+  lg_sparse_attn_bwd_workspace(p, B, S, H, Hkv, D, &need);
+  if (workspace == nullptr || workspace_bytes < need) return LG_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LG_ERR_UNSUPPORTED;
+  unsigned int* err = error_word(&st);
+  if (st != LG_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* dq_acc = static_cast<float*>(workspace);
+  float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + round256((size_t)B * H * S * D * 4));
+
+  CUtensorMap tq, tk, tv, tdo, tdk, tdv;
+  if ((st = make_map(&tq, q, B, S, H, D, 64)) != LG_OK) return st;
+  if ((st = make_map(&tk, k, B, S, Hkv, D, 128)) != LG_OK) return st;
+  if ((st = make_map(&tv, v, B, S, Hkv, D, 128)) != LG_OK) return st;
+  if ((st = make_map(&tdo, dout, B, S, H, D, 64)) != LG_OK) return st;
+  if ((st = make_map(&tdk, dk, B, S, Hkv, D, 128)) != LG_OK) return st;
+  if ((st = make_map(&tdv, dv, B, S, Hkv, D, 128)) != LG_OK) return st;
+
+  st = cuda_status(lg::launch_bwd_pre(o, dout, delta, dq_acc, B, S, H, D, s));
+  if (st != LG_OK) return st;
+  lg::BwdParams prm;
+  prm.pat = *p;
+  prm.lse = lse;
+  prm.delta = delta;
+  prm.dq_acc = dq_acc;
+  prm.S = S;
+  prm.H = H;
+  prm.Hkv = Hkv;
+  prm.D = D;
+  prm.nqb = S / 64;
+  prm.nkt = (S + 127) / 128;
+  prm.scale = scale;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.err = err;
+  st = cuda_status(lg::launch_bwd(D, tq, tk, tv, tdo, tdk, tdv, prm, B, s));
+  if (st != LG_OK) return st;
+  return cuda_status(lg::launch_bwd_dq(dq_acc, dq, scale, B, S, H, D, s));
+}
+
+// ---------------------------------------------------------------- decode
+lg_status_t lg_sparse_decode_splits(int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax, int32_t num_splits,
+                                    int32_t* splits) {
+  if (splits == nullptr || B <= 0 || H <= 0 || Hkv <= 0 || D <= 0 || Lmax <= 0 || num_splits < 0)
+    return LG_ERR_INVALID_ARG;
+  if (H % Hkv != 0) return LG_ERR_INVALID_ARG;
+  int ns, rps;
+  decode_split_rule(B, Hkv, D, Lmax, num_splits, &ns, &rps);
+  *splits = ns;
+  return LG_OK;
+}
+
+lg_status_t lg_sparse_decode_workspace(int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax, int32_t num_splits,
+                                       size_t* bytes) {
+  int32_t ns = 0;
+  lg_status_t st = lg_sparse_decode_splits(B, H, Hkv, D, Lmax, num_splits, &ns);
+  if (st != LG_OK) return st;
+  if (bytes == nullptr) return LG_ERR_INVALID_ARG;
+  if (ns == 1) {
+    *bytes = 0;
+    return LG_OK;
+  }
+  *bytes = round256((size_t)B * H * ns * D * 4) + round256((size_t)B * H * ns * 4) + round256((size_t)B * Hkv * 4);
+  return LG_OK;
+}
+
+lg_status_t lg_sparse_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* cache_lens,
+                             void* o, float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax,
+                             int32_t num_splits, float scale, void* workspace, size_t workspace_bytes,
+                             lg_stream_t stream) {
+  if (!q || !k_cache || !v_cache || !cache_lens || !o) return LG_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || Hkv <= 0 || D <= 0 || Lmax <= 0 || num_splits < 0) return LG_ERR_INVALID_ARG;
+  if (H % Hkv != 0) return LG_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return LG_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return LG_ERR_UNSUPPORTED;
+  const int G = H / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return LG_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv > 65535) return LG_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(cache_lens) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return LG_ERR_UNSUPPORTED;
+  int ns, rps;
+  decode_split_rule(B, Hkv, D, Lmax, num_splits, &ns, &rps);
+  size_t need = 0;
+  lg_sparse_decode_workspace(B, H, Hkv, D, Lmax, num_splits, &need);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LG_ERR_WORKSPACE;
+  if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LG_ERR_UNSUPPORTED;
+  lg_status_t st;
+  unsigned int* err = error_word(&st);
+  if (st != LG_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  lg::DecodeParams prm;
+  prm.q = q;
+  prm.k_cache = k_cache;
+  prm.v_cache = v_cache;
+  prm.lens = cache_lens;
+  prm.o = o;
+  prm.lse = lse;
+  prm.part_o = nullptr;
+  prm.part_lse = nullptr;
+  prm.tickets = nullptr;
+  if (ns > 1) {
+    char* w = static_cast<char*>(workspace);
+    prm.part_o = reinterpret_cast<float*>(w);
+    w += round256((size_t)B * H * ns * D * 4);
+    prm.part_lse = reinterpret_cast<float*>(w);
+    w += round256((size_t)B * H * ns * 4);
+    prm.tickets = reinterpret_cast<unsigned int*>(w);
+    st = cuda_status(cudaMemsetAsync(prm.tickets, 0, (size_t)B * Hkv * 4, s));
+    if (st != LG_OK) return st;
+  }
+  prm.B = B;
+  prm.H = H;
+  prm.Hkv = Hkv;
+  prm.Lmax = Lmax;
+  prm.ns = ns;
+  prm.rows_per_split = rps;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.err = err;
+  return cuda_status(lg::launch_decode(D, G, prm, s));
+}
+
+// ---------------------------------------------------------------- diagnostics
+lg_status_t lg_device_status(int32_t device, uint32_t* flags) {
+  if (flags == nullptr) return LG_ERR_INVALID_ARG;
+  int prev = 0;
+  if (cudaGetDevice(&prev) != cudaSuccess) return LG_ERR_CUDA;
+  if (cudaSetDevice(device) != cudaSuccess) return LG_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_lg_error_word, sizeof(v));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_lg_error_word, &zero, sizeof(zero));
+  cudaSetDevice(prev);
+  *flags = v;
+  return cuda_status(e);
+}
+
+}  // extern "C"

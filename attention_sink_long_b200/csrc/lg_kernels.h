@@ -1,0 +1,66 @@
+// lg_kernels.h -- launch interfaces between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/lg_attn.h"
+
+namespace lg {
+
+struct FwdParams {
+  lg_pattern_t pat;
+  float* lse;  // [B, H, S] or nullptr
+  int S, H, Hkv;
+  int nqb;  // S / 64
+  int nqt;  // ceil(S / 128)
+  float scale_log2;  // scale * log2(e)
+  unsigned int* err;
+};
+
+cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& to, const FwdParams& prm, int B, cudaStream_t stream);
+
+struct BwdParams {
+  lg_pattern_t pat;
+  const float* lse;      // [B, H, S]
+  const float* delta;    // [B, H, S] (workspace, written by the preprocess kernel)
+  float* dq_acc;         // [B, H, S, D] fp32 (workspace)
+  int S, H, Hkv, D;
+  int nqb;  // S / 64
+  int nkt;  // ceil(S / 128) KV tiles
+  float scale;       // softmax scale
+  float scale_log2;  // scale * log2(e)
+  unsigned int* err;
+};
+
+cudaError_t launch_bwd_pre(const void* o, const void* dout, float* delta, float* dq_acc, int B, int S, int H, int D,
+                           cudaStream_t stream);
+cudaError_t launch_bwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv, const BwdParams& prm,
+                       int B, cudaStream_t stream);
+cudaError_t launch_bwd_dq(const float* dq_acc, void* dq, float scale, int B, int S, int H, int D,
+                          cudaStream_t stream);
+
+struct DecodeParams {
+  const void* q;        // [B, H, D] bf16
+  const void* k_cache;  // [B, Lmax, Hkv, D] bf16
+  const void* v_cache;
+  const int32_t* lens;  // [B]
+  void* o;              // [B, H, D] bf16
+  float* lse;           // [B, H] or nullptr
+  float* part_o;        // [B, H, ns, D] fp32 (ns > 1)
+  float* part_lse;      // [B, H, ns] (log2 units)
+  unsigned int* tickets;  // [B, Hkv]
+  int B, H, Hkv, Lmax, ns, rows_per_split;
+  float scale_log2;
+  unsigned int* err;
+};
+
+cudaError_t launch_decode(int D, int G, const DecodeParams& prm, cudaStream_t stream);
+
+cudaError_t launch_pattern_iterate(const lg_pattern_t& p, int seqlen, int tile_blocks, int transpose, int32_t* out,
+                                   int cap, cudaStream_t stream);
+
+}  // namespace lg

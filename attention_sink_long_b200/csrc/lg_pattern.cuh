@@ -1,0 +1,91 @@
+// lg_pattern.cuh -- the static block pattern and its closed-form block iterators.
+//
+// "A Little Goes a Long Way" (LongGen), Abstract insight 1 and the atlas.scime.ai
+// summary, "Approach": sparse layers attend to sink blocks, a local window of
+// recent blocks and strided blocks, with static, block-wise access. Because the
+// pattern is static and made of at most three arithmetic ranges, the per-query-
+// block KV-block list (and its transpose) is enumerated here in closed form
+// instead of being stored: the kernels visit exactly the listed blocks, in
+// increasing order, and never touch a masked block.
+#pragma once
+
+#include <stdint.h>
+
+#include "../../include/lg_attn.h"
+
+#if defined(__CUDACC__)
+#define LG_HD __host__ __device__ __forceinline__
+#else
+#define LG_HD inline
+#endif
+
+namespace lg {
+
+LG_HD int imin(int a, int b) { return a < b ? a : b; }
+LG_HD int imax(int a, int b) { return a > b ? a : b; }
+LG_HD int ceil_div_nonneg(int a, int b) { return (a + b - 1) / b; }
+
+// Is KV block j in the list of query block i?
+LG_HD bool in_list(const lg_pattern_t& p, int i, int j) {
+  if (j < 0 || j > i) return false;
+  if (j < p.sink_blocks) return true;
+  if (i - j < p.local_blocks) return true;
+  if (p.stride > 0 && (j % p.stride) == 0) return true;
+  return false;
+}
+
+// Union of the KV-block lists of the consecutive query blocks [i_lo, i_hi], in
+// increasing order: sink blocks below the window, strided blocks below the
+// window, then the window [i_lo - local + 1, i_hi] (which covers every
+// diagonal). next(j) is the smallest listed block > j, or -1.
+struct KvIter {
+  int lo, hi, sink, stride;
+
+  LG_HD KvIter(const lg_pattern_t& p, int i_lo, int i_hi) {
+    const long long w = (long long)i_lo - (long long)p.local_blocks + 1;
+    lo = w < 0 ? 0 : (int)w;
+    hi = i_hi;
+    sink = p.sink_blocks;
+    stride = p.stride;
+  }
+  LG_HD int first() const { return next(-1); }
+  LG_HD int next(int j) const {
+    const int c = j + 1;
+    if (c >= lo) return c <= hi ? c : -1;
+    if (c < sink) return c;
+    if (stride > 0) {
+      const int m = ceil_div_nonneg(c, stride) * stride;
+      if (m < lo) return m;
+    }
+    return lo <= hi ? lo : -1;
+  }
+  LG_HD int count() const {
+    const int a = imin(imax(sink, 0), lo);  // sink blocks strictly below the window
+    int n = a;
+    if (stride > 0) n += ceil_div_nonneg(lo, stride) - ceil_div_nonneg(a, stride);
+    return n + (hi - lo + 1);
+  }
+};
+
+// Union of the query-block lists (transpose) of the consecutive KV blocks
+// [j_lo, j_hi], given nqb query blocks. A sink or strided KV block is seen by
+// every later query block; any other by the local_blocks query blocks starting
+// at itself. The union is the contiguous range [j_lo, last].
+struct QIter {
+  int first_blk, last_blk;
+
+  LG_HD QIter(const lg_pattern_t& p, int j_lo, int j_hi, int nqb) {
+    first_blk = j_lo;
+    int last = -1;
+    for (int j = j_lo; j <= j_hi; ++j) {
+      const bool global = (j < p.sink_blocks) || (p.stride > 0 && (j % p.stride) == 0);
+      const long long reach = global ? (long long)nqb - 1 : (long long)j + p.local_blocks - 1;
+      const int r = (int)(reach < (long long)nqb - 1 ? reach : (long long)nqb - 1);
+      last = imax(last, r);
+    }
+    last_blk = last;
+  }
+  LG_HD int count() const { return last_blk >= first_blk ? last_blk - first_blk + 1 : 0; }
+};
+
+}  // namespace lg

@@ -1,0 +1,220 @@
+/*
+ * lg_attn.h -- C ABI of the LongGen sparse-attention hot path for NVIDIA B200 (sm_100a).
+ *
+ * Method: "A Little Goes a Long Way: Efficient Long Context Training and
+ * Inference with Partial Contexts" (LongGen, arXiv 2410.01485).
+ *   - Abstract, insight 1: sparse layers keep the initial tokens (attention
+ *     sink), the recent tokens (window attention) and strided token blocks
+ *     (blockwise sparse attention), chosen for GPU-friendly memory access.
+ *   - Abstract, insight 2: the middle 1/3 of the layers keep full attention
+ *     (the all-blocks causal special case of the same kernels).
+ *   - atlas.scime.ai summary, "Approach": static, block-wise access; training
+ *     with a FlashAttention-2-based kernel (exact attention); serving over the
+ *     reduced KV cache of the sparse layers.
+ *   - Abstract / summary, "Key results": 1.67x prefill and 1.41x decode speedup
+ *     and KV cache 69.2 GB -> 26.5 GB at 128K (the decode entry point below is
+ *     the step those figures time).
+ *
+ * Conventions for every entry point:
+ *   - Every function returns lg_status_t (LG_OK == 0). Argument errors are
+ *     detected on the host before anything is launched; nothing is written.
+ *   - The caller owns every buffer. The library never allocates or frees
+ *     device memory and never synchronises the stream it is given (the one
+ *     exception, lg_device_status, says so). Pointers marked "device" must be
+ *     device memory of the current device, 16-byte aligned.
+ *   - Tensors are contiguous, row-major, with the layouts given per call:
+ *       q, o, dout, dq   [B, S, H, D]    bf16
+ *       k, v, dk, dv     [B, S, Hkv, D]  bf16
+ *       lse              [B, H, S]       fp32, natural log
+ *     Query head h reads KV head h / (H / Hkv).
+ *   - Launch errors map to LG_ERR_CUDA. Asynchronous device faults surface at
+ *     the caller's next synchronisation. Every device-side wait in the kernels
+ *     is bounded; a wait that runs out sets a flag readable with
+ *     lg_device_status and the kernel returns early (its outputs are then
+ *     undefined).
+ *   - Supported: D in {64, 128}; block_size == 64; S % 64 == 0; H % Hkv == 0;
+ *     1 <= local_blocks; sink_blocks >= 0; stride >= 0. Anything else returns
+ *     LG_ERR_UNSUPPORTED or LG_ERR_INVALID_ARG.
+ */
+#ifndef LG_ATTN_H_
+#define LG_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle (cudaStream_t / CUstream); NULL is the legacy default stream. */
+typedef void* lg_stream_t;
+
+typedef enum {
+  LG_OK = 0,
+  LG_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad pattern field */
+  LG_ERR_UNSUPPORTED = 2,  /* valid but outside the supported shapes / alignment */
+  LG_ERR_WORKSPACE = 3,    /* workspace missing or smaller than the query says */
+  LG_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed */
+  LG_ERR_INTERNAL = 5,
+  LG_ERR_CAPACITY = 6      /* an output buffer given with a capacity is too small */
+} lg_status_t;
+
+/*
+ * Static block pattern (atlas.scime.ai summary, "Approach": static, block-wise
+ * access; Abstract, insight 1: sink, window, strided blocks).
+ * Query block i = q / block_size attends to KV block j = k / block_size iff
+ *   j <= i  and  ( j < sink_blocks  or  i - j < local_blocks
+ *                  or (stride > 0 and j % stride == 0) ),
+ * with token-level causality (k <= q) inside the diagonal block.
+ * local_blocks counts the diagonal block; stride == 0 disables the strided
+ * term. Full causal attention is {64, 0, INT32_MAX, 0}.
+ */
+typedef struct {
+  int32_t block_size;
+  int32_t sink_blocks;
+  int32_t local_blocks;
+  int32_t stride;
+} lg_pattern_t;
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char* lg_strerror(lg_status_t status);
+
+/* ABI version of this library, (major << 16) | minor. */
+int32_t lg_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* Pattern expansion (host, pure integer)                                    */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * CSR of KV blocks per query block for a sequence of seqlen tokens
+ * (seqlen % block_size == 0, nqb = seqlen / block_size): row_ptr[nqb + 1] and
+ * col[nnz], each row sorted ascending without duplicates. Host pointers.
+ * Capacity idiom: with col == NULL only *nnz is written (row_ptr may also be
+ * NULL); otherwise cap is the length of col and LG_ERR_CAPACITY is returned
+ * (with *nnz set) when cap < nnz.
+ */
+lg_status_t lg_pattern_expand(const lg_pattern_t* pattern, int32_t seqlen, int32_t* row_ptr,
+                              int32_t* col, int64_t cap, int64_t* nnz);
+
+/* The transpose (CSC): query blocks per KV block, col_ptr[nqb + 1], row[nnz]. Same idiom. */
+lg_status_t lg_pattern_expand_t(const lg_pattern_t* pattern, int32_t seqlen, int32_t* col_ptr,
+                                int32_t* row, int64_t cap, int64_t* nnz);
+
+/* Number of unmasked (query, key) token pairs of one head: the unit of useful work. */
+lg_status_t lg_pattern_pairs(const lg_pattern_t* pattern, int32_t seqlen, int64_t* pairs);
+
+/*
+ * Runs, on the device, the block iterator the attention kernels use, and
+ * records what it visits, so tests can compare it bit for bit with the CSR.
+ * Tiles are tile_blocks (1 or 2) consecutive 64-token blocks. With
+ * transpose == 0 a tile is a range of query blocks and the iterator yields
+ * KV blocks (forward); with transpose == 1 it is a range of KV blocks and
+ * yields query blocks (backward). For tile u, out[u * (cap + 1)] receives the
+ * count n and out[u * (cap + 1) + 1 + e] the e-th visited block as
+ * (block << 2) | membership, where bit t of membership says whether the
+ * visited block is in the list of the tile's t-th block. Device pointer
+ * out holds ceil(nqb / tile_blocks) * (cap + 1) int32; entries beyond cap are
+ * not written (the count still is).
+ */
+lg_status_t lg_pattern_iterate_device(const lg_pattern_t* pattern, int32_t seqlen, int32_t tile_blocks,
+                                      int32_t transpose, int32_t* out, int32_t cap, lg_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Prefill forward                                                          */
+/* ------------------------------------------------------------------------ */
+
+/* Workspace bytes for lg_sparse_attn_fwd (currently 0: the block lists are generated in-kernel). */
+lg_status_t lg_sparse_attn_fwd_workspace(const lg_pattern_t* pattern, int32_t B, int32_t S, int32_t H,
+                                         int32_t Hkv, int32_t D, size_t* bytes);
+
+/*
+ * O = softmax_mask(scale * Q K^T) V for every (b, h), and LSE per query row.
+ * Abstract, insights 1-2; atlas.scime.ai summary, "Approach" (exact,
+ * FlashAttention-style attention under the static mask above).
+ * Device pointers: q [B,S,H,D] bf16, k/v [B,S,Hkv,D] bf16, o [B,S,H,D] bf16
+ * (written), lse [B,H,S] fp32 (written; may be NULL when not needed).
+ * KV blocks outside the pattern are never read.
+ */
+lg_status_t lg_sparse_attn_fwd(const lg_pattern_t* pattern, const void* q, const void* k, const void* v,
+                               void* o, float* lse, int32_t B, int32_t S, int32_t H, int32_t Hkv, int32_t D,
+                               float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Training backward                                                        */
+/* ------------------------------------------------------------------------ */
+
+/* Workspace bytes for lg_sparse_attn_bwd: fp32 dQ accumulator [B,H,S,D] plus Delta [B,H,S]. */
+lg_status_t lg_sparse_attn_bwd_workspace(const lg_pattern_t* pattern, int32_t B, int32_t S, int32_t H,
+                                         int32_t Hkv, int32_t D, size_t* bytes);
+
+/*
+ * Gradients of the forward above given dO (atlas.scime.ai summary, "Approach":
+ * the training kernel; "Key results": 1.55x training speedup at 128K):
+ *   P = exp(scale Q K^T - LSE) on the mask, Delta = rowsum(dO * O),
+ *   dV = P^T dO, dS = P * (dO V^T - Delta), dQ = scale dS K, dK = scale dS^T Q.
+ * Device pointers: q, k, v, o, dout, lse as produced/consumed by the forward;
+ * dq [B,S,H,D], dk/dv [B,S,Hkv,D] bf16 (written; dk/dv sum over the query
+ * heads of a KV group). workspace (device, 256-byte aligned) of at least the
+ * queried size; its contents on entry do not matter.
+ */
+lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* pattern, const void* q, const void* k, const void* v,
+                               const void* o, const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                               int32_t B, int32_t S, int32_t H, int32_t Hkv, int32_t D, float scale,
+                               void* workspace, size_t workspace_bytes, lg_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Decode over the reduced KV cache                                         */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * The number of KV splits lg_sparse_decode uses when num_splits == 0 (auto),
+ * written to *splits. Always >= 1.
+ */
+lg_status_t lg_sparse_decode_splits(int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax,
+                                    int32_t num_splits, int32_t* splits);
+
+/* Workspace bytes for lg_sparse_decode (per-split partial o and lse, plus one ticket per (b, kv head)). */
+lg_status_t lg_sparse_decode_workspace(int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax,
+                                       int32_t num_splits, size_t* bytes);
+
+/*
+ * Single-token attention of each sequence's query over its cached rows:
+ *   o[b,h] = sum_{r < cache_lens[b]} softmax_r(scale q[b,h] . K[b,r]) V[b,r],
+ *   lse[b,h] = log sum_r exp(scale q[b,h] . K[b,r]).
+ * The cache of a sparse layer holds only what its pattern can still reach
+ * (sink + window, + strided blocks), a full layer's holds every token
+ * (Abstract: KV cache reduction; summary, "Key results": 69.2 -> 26.5 GB and
+ * 1.41x decode). Row order does not matter (softmax is permutation
+ * invariant), so a ring-buffered window is fine.
+ * Device pointers: q [B,H,D] bf16; k_cache, v_cache [B,Lmax,Hkv,D] bf16;
+ * cache_lens [B] int32 with 1 <= cache_lens[b] <= Lmax (values are read on
+ * the device and clamped to [0, Lmax]; a zero length yields o = 0,
+ * lse = -inf); o [B,H,D] bf16 (written); lse [B,H] fp32 (written, may be NULL).
+ * The KV range of each (b, kv head) is cut into num_splits pieces (0 = auto,
+ * see lg_sparse_decode_splits); partial results are merged by
+ * log-sum-exp in the same launch by the last CTA to finish each (b, kv head).
+ * workspace (device, 256-byte aligned) of at least the queried size; its
+ * ticket region is cleared on the stream by every call.
+ */
+lg_status_t lg_sparse_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* cache_lens,
+                             void* o, float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax,
+                             int32_t num_splits, float scale, void* workspace, size_t workspace_bytes,
+                             lg_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Diagnostics                                                              */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Reads and clears the device-side error flags of the given device (bit 0:
+ * a forward wait ran out, bit 1: a backward wait ran out, bit 2: decode).
+ * SYNCHRONISES that device. *flags == 0 means no bounded wait ran out.
+ */
+lg_status_t lg_device_status(int32_t device, uint32_t* flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LG_ATTN_H_ */

@@ -54,3 +54,37 @@ def ragged_lens(B: int, Lmax: int, seed: int = SEED_BASE + 7):
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     return torch.randint(1, Lmax + 1, (B,), generator=g, dtype=torch.int64).tolist()
+
+
+def device_normal(shape, seed: int, device, dtype=torch.bfloat16) -> torch.Tensor:
+    """N(0, 1) drawn by torch's generator on ``device`` (used for inputs too large
+    to draw on the host, e.g. the 128K prefill and the 131072-row decode caches;
+    the oracle reads the sampled slices it needs back from the device)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    out = torch.empty(*shape, dtype=dtype, device=device)
+    chunk = 1 << 28  # elements per draw: bounds the fp32 temporary to 1 GiB
+    flat = out.view(-1)
+    for i, s in enumerate(range(0, flat.numel(), chunk)):
+        n = min(chunk, flat.numel() - s)
+        flat[s:s + n] = torch.randn(n, generator=g, device=device, dtype=torch.float32).to(dtype)
+    return out
+
+
+def prefill_inputs_device(B: int, S: int, H: int, Hkv: int, D: int, device, seed: int = SEED_BASE,
+                          with_dout: bool = False):
+    q = device_normal((B, S, H, D), seed + 0, device)
+    k = device_normal((B, S, Hkv, D), seed + 1, device)
+    v = device_normal((B, S, Hkv, D), seed + 2, device)
+    if with_dout:
+        return q, k, v, device_normal((B, S, H, D), seed + 3, device)
+    return q, k, v
+
+
+def decode_inputs_device(B: int, H: int, Hkv: int, D: int, Lmax: int, device, seed: int = SEED_BASE, lens=None):
+    q = device_normal((B, H, D), seed + 0, device)
+    kc = device_normal((B, Lmax, Hkv, D), seed + 1, device)
+    vc = device_normal((B, Lmax, Hkv, D), seed + 2, device)
+    if lens is None:
+        lens = [Lmax] * B
+    return q, kc, vc, torch.tensor(lens, dtype=torch.int32, device=device)

@@ -1,0 +1,146 @@
+"""Host-side tests of the C-ABI library: loading, exported symbols, the host
+pattern expansion (bit-exact against the oracle's token-level scan and the
+hand-derived counts) and argument validation. No GPU needed: every call here
+returns before any CUDA work."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import attention_sink_long_b200 as lg
+from attention_sink_long_b200 import build as lgbuild
+
+from test_oracle import load_golden
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lg_attn.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    lgbuild.build()
+    yield
+
+
+def header_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+char\s*\*|lg_status_t|int32_t)\s+(lg_\w+)\s*\(", text, re.M)))
+
+
+def test_exports_every_declared_symbol():
+    names = header_functions()
+    assert len(names) >= 14
+    L = ctypes.CDLL(lgbuild.LIB)
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(lg.EXPORTED_SYMBOLS) == names
+
+
+def test_strerror_and_version():
+    assert lg.lg_strerror(0) == "ok"
+    assert "workspace" in lg.lg_strerror(3)
+    assert lg.lg_version() >= (1 << 16)
+
+
+PATTERNS = [
+    lg.Pattern(64, 1, 4, 0), lg.Pattern(64, 1, 16, 32), lg.Pattern(64, 0, 1, 0), lg.Pattern(64, 0, 1, 3),
+    lg.Pattern(64, 3, 2, 5), lg.Pattern(64, 0, 7, 0), lg.Pattern.full(64), lg.Pattern(64, 100, 1, 0),
+    lg.Pattern(16, 2, 3, 4), lg.Pattern(8, 1, 1, 1),
+]
+
+
+@pytest.mark.parametrize("p", PATTERNS)
+@pytest.mark.parametrize("S_blocks", [1, 2, 7, 33])
+def test_host_expansion_bit_exact_vs_oracle(p, S_blocks):
+    S = p.block_size * S_blocks
+    op = oracle.Pattern(*p)
+    row_ptr, col = lg.lg_pattern_expand(p, S)
+    o_ptr, o_col = oracle.block_lists(S, op)
+    np.testing.assert_array_equal(row_ptr, o_ptr)
+    np.testing.assert_array_equal(col, o_col)
+    col_ptr, row = lg.lg_pattern_expand_t(p, S)
+    t_ptr, t_row = oracle.block_lists_t(S, op)
+    np.testing.assert_array_equal(col_ptr, t_ptr)
+    np.testing.assert_array_equal(row, t_row)
+    assert lg.lg_pattern_pairs(p, S) == oracle.pair_count(S, op)
+
+
+@pytest.mark.parametrize("name", ["c1_sink_local4", "c2_sink_window", "c2_dense", "c3_block_sparse",
+                                  "c3_analog_4096", "c4_sink_window"])
+def test_host_counts_match_hand_counts(name):
+    S, p, nnz, pairs = load_golden()[name]
+    lp = lg.Pattern(p.block_size, p.sink_blocks, p.local_blocks, p.stride)
+    row_ptr, col = lg.lg_pattern_expand(lp, S)
+    assert int(row_ptr[-1]) == nnz
+    assert np.all(np.diff(row_ptr) > 0)
+    assert lg.lg_pattern_pairs(lp, S) == pairs
+    col_ptr, row = lg.lg_pattern_expand_t(lp, S)
+    assert int(col_ptr[-1]) == nnz
+
+
+def test_expansion_capacity_idiom():
+    L = lg.lib()
+    p = lg._lg_pattern_t(64, 1, 4, 0)
+    nnz = ctypes.c_int64(0)
+    assert L.lg_pattern_expand(ctypes.byref(p), 1024, None, None, 0, ctypes.byref(nnz)) == 0
+    assert nnz.value == 70
+    rp = (ctypes.c_int32 * 17)()
+    col = (ctypes.c_int32 * 10)()
+    assert L.lg_pattern_expand(ctypes.byref(p), 1024, rp, col, 10, ctypes.byref(nnz)) == 6  # LG_ERR_CAPACITY
+    assert L.lg_pattern_expand(ctypes.byref(p), 1000, rp, col, 10, ctypes.byref(nnz)) == 1  # not a multiple
+
+
+def _fwd(**kw):
+    L = lg.lib()
+    a = dict(p=lg._lg_pattern_t(64, 1, 4, 0), q=0x10000, k=0x20000, v=0x30000, o=0x40000, lse=0x50000,
+             B=1, S=1024, H=4, Hkv=4, D=64, scale=0.125)
+    a.update(kw)
+    p = a["p"]
+    return L.lg_sparse_attn_fwd(None if p is None else ctypes.byref(p), a["q"], a["k"], a["v"], a["o"], a["lse"],
+                                a["B"], a["S"], a["H"], a["Hkv"], a["D"], a["scale"], None, 0, None)
+
+
+def test_fwd_argument_errors():
+    assert _fwd(p=None) == 1
+    assert _fwd(q=None) == 1
+    assert _fwd(B=0) == 1
+    assert _fwd(H=4, Hkv=3) == 1
+    assert _fwd(scale=0.0) == 1
+    assert _fwd(scale=float("nan")) == 1
+    assert _fwd(p=lg._lg_pattern_t(64, 1, 0, 0)) == 1      # local_blocks < 1
+    assert _fwd(p=lg._lg_pattern_t(64, -1, 1, 0)) == 1     # negative sink
+    assert _fwd(p=lg._lg_pattern_t(32, 1, 4, 0)) == 2      # block size other than 64
+    assert _fwd(S=1000) == 2                               # S not a multiple of 64
+    assert _fwd(D=96) == 2
+    assert _fwd(q=0x10008) == 2                            # misaligned
+    assert _fwd(lse=0x50004) == 2
+
+
+def test_bwd_and_decode_argument_errors():
+    L = lg.lib()
+    p = lg._lg_pattern_t(64, 1, 4, 0)
+    ptrs = [0x10000 * (i + 1) for i in range(9)]
+    assert L.lg_sparse_attn_bwd(ctypes.byref(p), *ptrs, 1, 1024, 4, 4, 64, 0.125, None, 0, None) == 3  # workspace
+    assert L.lg_sparse_attn_bwd(ctypes.byref(p), *ptrs, 1, 1024, 4, 4, 128, 0.125, 0x100000, 16, None) == 3
+    assert L.lg_sparse_attn_bwd(ctypes.byref(p), *([None] + ptrs[1:]), 1, 1024, 4, 4, 64, 0.125, None, 0, None) == 1
+    args = [0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0x60000]
+    assert L.lg_sparse_decode(*args, 32, 32, 32, 96, 4160, 0, 0.1, None, 0, None) == 2   # D
+    assert L.lg_sparse_decode(*args, 32, 24, 8, 128, 4160, 0, 0.1, None, 0, None) == 2   # G = 3
+    assert L.lg_sparse_decode(*args, 32, 32, 32, 128, 4160, 0, 0.1, None, 0, None) == 3  # workspace needed
+    assert L.lg_sparse_decode(*args, 32, 32, 32, 128, 0, 0, 0.1, None, 0, None) == 1
+
+
+def test_workspace_queries():
+    assert lg.lg_sparse_attn_fwd_workspace(lg.Pattern(64, 1, 64, 0), 1, 131072, 32, 32, 128) == 0
+    ws = lg.lg_sparse_attn_bwd_workspace(lg.Pattern(64, 1, 64, 0), 1, 131072, 32, 32, 128)
+    assert ws >= 131072 * 32 * 128 * 4 + 131072 * 32 * 4
+    assert lg.lg_sparse_decode_splits(32, 32, 32, 128, 4160) > 1
+    assert lg.lg_sparse_decode_splits(1, 1, 1, 128, 64, 1) == 1
+    assert lg.lg_sparse_decode_workspace(1, 1, 1, 128, 64, 1) == 0
+    ns = lg.lg_sparse_decode_splits(32, 32, 32, 128, 131072)
+    assert lg.lg_sparse_decode_workspace(32, 32, 32, 128, 131072) >= 32 * 32 * ns * 129 * 4
+    assert lg.lg_sparse_decode_splits(2, 8, 8, 128, 100, 7) == 7
