@@ -1,0 +1,577 @@
+#!/usr/bin/env python3
+"""Benchmark of the LongGen sparse-attention hot path on B200.
+
+One step = one pass of every kernel of the path over the Llama-2-7B-shaped 32K
+workload (B=1, H=Hkv=32, D=128, bf16, 64-token blocks):
+  * prefill forward, sink+window pattern {64, 1, 64, 0} (64 sink + 4096 window tokens);
+  * prefill forward, full causal pattern (the middle-layer dense case);
+  * training backward of the sink+window layer (preprocess, main, dQ convert);
+  * decode of one sparse layer over its reduced cache: batch 32, 32 heads,
+    4160 cached rows (64 sink + 4096 window), split-KV with the LSE merge.
+The block iterator (pattern expansion) runs inside the kernels.
+
+value = useful FLOPs of the whole step (unmasked pairs only: 4*D per pair
+forward, 10*D per pair backward, 4*D per cached row decode) / device time.
+Per-kernel rows (TFLOP/s, GB/s and roofline fractions) are in "rows".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
+                    [--workload step32k|fwd128k|bwd128k|decode]
+
+Multi-GPU (torchrun): every rank runs the same per-GPU workload on its own
+device (weak scaling, independent replicas -- the path has no exchange step);
+the time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn fwd/bwd useful TFLOP/s & decode GB/s; % of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SINK_WINDOW = (64, 1, 64, 0)
+FULL = (64, 0, 2**31 - 1, 0)
+BLOCK_SPARSE = (64, 1, 16, 32)
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--workload", choices=["step32k", "fwd128k", "bwd128k", "decode"], default="step32k")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
+    return ap.parse_args(argv)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------
+# Workload description (shared by both arms)
+# ----------------------------------------------------------------------------
+
+def workload(name):
+    D = 128
+    if name == "step32k":
+        return {
+            "workload": "llama2-7b-shaped 32K step: fwd sink+window + fwd dense + bwd sink+window + sparse-layer decode",
+            "prefill": {"B": 1, "S": 32768, "H": 32, "Hkv": 32, "D": D},
+            "fwd": [("sink+window", SINK_WINDOW), ("dense", FULL)],
+            "bwd": [("sink+window", SINK_WINDOW)],
+            "decode": {"B": 32, "H": 32, "Hkv": 32, "D": D, "L": 4160},
+        }
+    if name == "fwd128k":
+        return {"workload": "128K block-sparse prefill forward {64,1,16,32}",
+                "prefill": {"B": 1, "S": 131072, "H": 32, "Hkv": 32, "D": D},
+                "fwd": [("block-sparse", BLOCK_SPARSE)], "bwd": [], "decode": None}
+    if name == "bwd128k":
+        return {"workload": "128K sink+window training backward {64,1,64,0}",
+                "prefill": {"B": 1, "S": 131072, "H": 32, "Hkv": 32, "D": D},
+                "fwd": [], "bwd": [("sink+window", SINK_WINDOW)], "decode": None}
+    if name == "decode":
+        return {"workload": "32-layer hybrid decode step: 21 sparse layers (4160 rows) + 11 full layers (131072 rows)",
+                "prefill": None, "fwd": [], "bwd": [],
+                "decode": {"B": 32, "H": 32, "Hkv": 32, "D": D, "L": 4160, "L_full": 131072}}
+    raise ValueError(name)
+
+
+def pairs_of(pattern, S):
+    """Unmasked pairs per head, from the library's host expansion (closed form)."""
+    import attention_sink_long_b200 as lg
+
+    return lg.lg_pattern_pairs(pattern, S)
+
+
+# ----------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# CUDA arm
+# ----------------------------------------------------------------------------
+
+class CudaStep:
+    """Device buffers and the launch sequence of one step."""
+
+    def __init__(self, wl, device):
+        import torch
+
+        import attention_sink_long_b200 as lg
+        import synthetic_inputs as si
+
+        self.lg, self.torch, self.wl, self.dev = lg, torch, wl, device
+        self.stream = torch.cuda.current_stream(device)
+        self.parts = []  # (name, kind, useful_flops, useful_bytes, launches)
+        pf = wl["prefill"]
+        if pf is not None:
+            B, S, H, Hkv, D = pf["B"], pf["S"], pf["H"], pf["Hkv"], pf["D"]
+            self.scale = 1.0 / math.sqrt(D)
+            self.q, self.k, self.v, self.do = si.prefill_inputs_device(B, S, H, Hkv, D, device, with_dout=True)
+            self.o = {n: torch.empty_like(self.q) for n, _ in wl["fwd"]}
+            self.lse = {n: torch.empty(B, H, S, dtype=torch.float32, device=device) for n, _ in wl["fwd"]}
+            for n, p in wl["fwd"]:
+                self.parts.append((f"fwd {n}", "fwd", 4 * D * pairs_of(p, S) * B * H, None, 1))
+            if wl["bwd"] and not self._bwd_available(pf, wl["bwd"][0][1]):
+                wl = dict(wl, bwd=[], workload=wl["workload"] + " (backward not available in this build)")
+                self.wl = wl
+            if wl["bwd"]:
+                self.dq, self.dk, self.dv = torch.empty_like(self.q), torch.empty_like(self.k), torch.empty_like(self.v)
+                self.bwd_ws = torch.empty(max(lg.lg_sparse_attn_bwd_workspace(wl["bwd"][0][1], B, S, H, Hkv, D), 1),
+                                          dtype=torch.uint8, device=device)
+                for n, p in wl["bwd"]:
+                    if n not in self.o:  # the backward needs O and LSE of its own forward
+                        self.o[n] = torch.empty_like(self.q)
+                        self.lse[n] = torch.empty(B, H, S, dtype=torch.float32, device=device)
+                        lg.lg_sparse_attn_fwd(p, self.q, self.k, self.v, self.o[n], self.lse[n], self.scale)
+                    self.parts.append((f"bwd {n}", "bwd", 10 * D * pairs_of(p, S) * B * H, None, 3))
+        dc = wl["decode"]
+        if dc is not None:
+            B, H, Hkv, D, L = dc["B"], dc["H"], dc["Hkv"], dc["D"], dc["L"]
+            self.dq_in, self.kc, self.vc, self.lens = si.decode_inputs_device(B, H, Hkv, D, L, device)
+            self.do_out = torch.empty(B, H, D, dtype=torch.bfloat16, device=device)
+            self.dlse = torch.empty(B, H, dtype=torch.float32, device=device)
+            self.dws = torch.empty(max(lg.lg_sparse_decode_workspace(B, H, Hkv, D, L), 1), dtype=torch.uint8,
+                                   device=device)
+            nbytes = 2 * B * L * Hkv * D * 2 + 2 * B * H * D * 2
+            self.parts.append(("decode sparse layer", "decode", 4 * D * L * B * H, nbytes, 1))
+            if "L_full" in dc:
+                Lf = dc["L_full"]
+                self.fq, self.fkc, self.fvc, self.flens = si.decode_inputs_device(B, H, Hkv, D, Lf, device, seed=2000)
+                self.fws = torch.empty(max(lg.lg_sparse_decode_workspace(B, H, Hkv, D, Lf), 1), dtype=torch.uint8,
+                                       device=device)
+                fbytes = 2 * B * Lf * Hkv * D * 2 + 2 * B * H * D * 2
+                self.parts.append(("decode full layer", "decode_full", 4 * D * Lf * B * H, fbytes, 1))
+
+    def _bwd_available(self, pf, pattern):
+        """One tiny backward call: False when the library reports it unsupported."""
+        lg, torch = self.lg, self.torch
+        D = pf["D"]
+        t = torch.zeros(1, 128, 1, D, dtype=torch.bfloat16, device=self.dev)
+        lse = torch.zeros(1, 1, 128, dtype=torch.float32, device=self.dev)
+        ws = torch.empty(lg.lg_sparse_attn_bwd_workspace(pattern, 1, 128, 1, 1, D), dtype=torch.uint8,
+                         device=self.dev)
+        try:
+            lg.lg_sparse_attn_bwd(pattern, t, t, t, t, t, lse, torch.empty_like(t), torch.empty_like(t),
+                                  torch.empty_like(t), 0.1, ws)
+        except lg.LgError as e:
+            if e.status == 4:
+                return False
+            raise
+        return True
+
+    def run(self, events=None):
+        """Launch one step; if events is given, record one event after each part."""
+        lg, wl = self.lg, self.wl
+        i = 0
+        for n, p in wl["fwd"]:
+            lg.lg_sparse_attn_fwd(p, self.q, self.k, self.v, self.o[n], self.lse[n], self.scale)
+            if events is not None:
+                events[i].record(self.stream)
+            i += 1
+        for n, p in wl["bwd"]:
+            lg.lg_sparse_attn_bwd(p, self.q, self.k, self.v, self.o[n], self.do, self.lse[n], self.dq, self.dk,
+                                  self.dv, self.scale, self.bwd_ws)
+            if events is not None:
+                events[i].record(self.stream)
+            i += 1
+        if wl["decode"] is not None:
+            lg.lg_sparse_decode(self.dq_in, self.kc, self.vc, self.lens, self.do_out, self.dlse, self.scale_dec(),
+                                workspace=self.dws)
+            if events is not None:
+                events[i].record(self.stream)
+            i += 1
+            if "L_full" in wl["decode"]:
+                lg.lg_sparse_decode(self.fq, self.fkc, self.fvc, self.flens, self.do_out, self.dlse,
+                                    self.scale_dec(), workspace=self.fws)
+                if events is not None:
+                    events[i].record(self.stream)
+                i += 1
+
+    def scale_dec(self):
+        return 1.0 / math.sqrt(self.wl["decode"]["D"])
+
+    def launches_per_step(self):
+        return sum(p[4] for p in self.parts)
+
+    def step_weights(self):
+        """How many times each part counts per reported step (decode: 21 sparse + 11 full layers)."""
+        if self.wl["workload"].startswith("32-layer"):
+            return [21 if p[2] and p[1] == "decode" else 11 for p in self.parts]
+        return [1] * len(self.parts)
+
+
+def host_buffers(step):
+    """Pinned host copies of the step's inputs and outputs, for the end-to-end loop."""
+    torch = step.torch
+    pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu())  # noqa: E731
+    ins, outs = [], []
+    for name in ("q", "k", "v", "do", "dq_in", "kc", "vc", "lens"):
+        if hasattr(step, name):
+            ins.append((getattr(step, name), pin(getattr(step, name))))
+    for d in ("o", "lse"):
+        if hasattr(step, d):
+            for t in getattr(step, d).values():
+                outs.append((t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)))
+    for name in ("dq", "dk", "dv", "do_out", "dlse"):
+        if hasattr(step, name):
+            t = getattr(step, name)
+            outs.append((t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)))
+    return ins, outs
+
+
+def cuda_arm(args, rank, world, dist):
+    import torch
+
+    import attention_sink_long_b200 as lg
+    from attention_sink_long_b200 import build as lgbuild
+
+    lgbuild.build()
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    wl = workload(args.workload)
+    step = CudaStep(wl, device)
+    wl = step.wl
+    # Skip parts the library does not provide (e.g. a kernel not built yet): probe once.
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    assert lg.lg_device_status(local) == 0, "a bounded device wait ran out during warm-up"
+
+    nparts = len(step.parts)
+    per_part_ms = [[] for _ in range(nparts)]
+    clocks = ClockSampler(local)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nparts)] for _ in range(args.steps)]
+    t0.record(step.stream)
+    for k in range(args.steps):
+        step.run(evs[k])
+    t1.record(step.stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if dist is not None:
+        dist.barrier()
+    total_ms = t0.elapsed_time(t1)
+    for k in range(args.steps):
+        prev = t0 if k == 0 else evs[k - 1][-1]
+        for i in range(nparts):
+            per_part_ms[i].append(prev.elapsed_time(evs[k][i]))
+            prev = evs[k][i]
+    assert lg.lg_device_status(local) == 0, "a bounded device wait ran out during the timed region"
+
+    if dist is not None:
+        tt = torch.tensor([total_ms], device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+
+    weights = step.step_weights()
+    step_flops = sum(w * p[2] for w, p in zip(weights, step.parts))
+    ms_per_step = total_ms / args.steps
+    if wl["workload"].startswith("32-layer"):
+        # Reported decode step: 21 sparse-layer + 11 full-layer calls, from the per-call times.
+        ms_per_step = sum(w * statistics.mean(per_part_ms[i]) for i, w in enumerate(weights))
+    value = world * step_flops / (ms_per_step * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    rows = {}
+    dominant = None
+    for i, (name, kind, flops, nbytes, nl) in enumerate(step.parts):
+        ms = statistics.mean(per_part_ms[i])
+        r = {"ms": round(ms, 4), "useful_tflops": round(flops / (ms * 1e-3) / 1e12, 2)}
+        if kind.startswith("decode"):
+            r["gbs"] = round(nbytes / (ms * 1e-3) / 1e9, 1)
+            r["frac_hbm"] = round(r["gbs"] / peaks["hbm_gbs"], 4)
+        else:
+            r["frac_bf16"] = round(r["useful_tflops"] / peaks["bf16_tflops"], 4)
+        rows[name] = r
+        if dominant is None or ms * weights[i] > dominant[1]:
+            dominant = (i, ms * weights[i])
+    di = dominant[0]
+    dname, dkind, dflops, dbytes, _ = step.parts[di]
+    dms = statistics.mean(per_part_ms[di])
+    if dkind.startswith("decode"):
+        achieved = dbytes / (dms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None}
+    else:
+        achieved = dflops / (dms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None}
+    roof["kernel"] = dname
+    roof["peak_source"] = f"{peak_src} (burst)"
+
+    # End-to-end through the public API with pinned host buffers.
+    e2e = None
+    if not args.no_e2e:
+        ins, outs = host_buffers(step)
+        bi = sum(h.numel() * h.element_size() for _, h in ins)
+        bo = sum(h.numel() * h.element_size() for _, h in outs)
+        for _ in range(1):
+            for d, h in ins:
+                d.copy_(h, non_blocking=True)
+            step.run()
+            for d, h in outs:
+                h.copy_(d, non_blocking=True)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        ek = max(1, min(args.steps, 5))
+        e0.record(step.stream)
+        for _ in range(ek):
+            for d, h in ins:
+                d.copy_(h, non_blocking=True)
+            step.run()
+            for d, h in outs:
+                h.copy_(d, non_blocking=True)
+        e1.record(step.stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1) / ek
+        if dist is not None:
+            tt = torch.tensor([ems], device=device)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ems = float(tt.item())
+        e2e = {"value": round(world * step_flops / (ems * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(ems, 3), "steps": ek}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, args.cpu_seconds)
+
+    launches = args.steps * step.launches_per_step()
+    pf = wl["prefill"]
+    config = {"workload": wl["workload"], "l2": "inputs larger than L2 (126 MB), no flush",
+              "parallelism": f"dp{world} (independent replicas, no collective)"}
+    if pf:
+        config.update({"prefill_shape": pf, "patterns": {n: list(p) for n, p in wl["fwd"] + wl["bwd"]}})
+    if wl["decode"]:
+        config["decode_shape"] = wl["decode"]
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16; no dataset, no weights)",
+        "config": config, "roofline": roof, "rows": rows, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches, "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# Oracle on the host: the CPU baseline and the reference arm
+# ----------------------------------------------------------------------------
+
+def oracle_sample(wl, budget_s, seed=11):
+    """Runs the fp64 oracle on a bounded sample of the workload for about
+    budget_s seconds; returns (useful_flops, seconds, description)."""
+    import numpy as np
+
+    import oracle
+    import synthetic_inputs as si
+
+    rng = np.random.default_rng(seed)
+    flops = 0.0
+    t_used = 0.0
+    desc = []
+    pf = wl["prefill"]
+    jobs = []
+    if pf:
+        S, D = pf["S"], pf["D"]
+        B, H = pf["B"], pf["H"]
+        nqb = S // 64
+        # One head's inputs drawn on the host with the same seeds (head 0 of a 1-head draw).
+        q, k, v, do = si.prefill_inputs(1, S, 1, 1, D, with_dout=True)
+        qh, kh, vh, doh = (t[0, :, 0].double().numpy() for t in (q, k, v, do))
+        scale = 1.0 / math.sqrt(D)
+        for n, p in wl["fwd"]:
+            jobs.append(("fwd " + n, "fwd", p))
+        for n, p in wl["bwd"]:
+            jobs.append(("bwd " + n, "bwd", p))
+    if wl["decode"]:
+        jobs.append(("decode", "decode", None))
+    per_job = budget_s / max(1, len(jobs))
+    for name, kind, p in jobs:
+        t_start = time.perf_counter()
+        n_done = 0
+        job_flops = 0.0
+        while time.perf_counter() - t_start < per_job:
+            if kind in ("fwd", "bwd"):
+                blk = int(rng.integers(0, nqb))
+                rows = np.arange(blk * 64, blk * 64 + 64)
+                op = oracle.Pattern(*p)
+                pairs = int(oracle.allowed(rows[:, None], np.arange(S)[None, :], op).sum())
+                if kind == "fwd":
+                    oracle.attention_rows(qh, kh, vh, rows, op, scale)
+                    job_flops += 4 * D * pairs
+                else:
+                    oracle.attention_backward_rows(qh, kh, vh, doh, rows, op, scale)
+                    job_flops += 6 * D * pairs  # S, dP and dQ for these rows
+            else:
+                dc = wl["decode"]
+                L, D2 = dc["L"], dc["D"]
+                qq, kc, vc, cl = si.decode_inputs(1, 1, 1, D2, L, seed=1000 + int(rng.integers(0, 1000)))
+                oracle.decode(qq, kc, vc, cl.numpy(), 1.0 / math.sqrt(D2))
+                job_flops += 4 * D2 * L
+            n_done += 1
+        dt = time.perf_counter() - t_start
+        flops += job_flops
+        t_used += dt
+        desc.append(f"{name}: {n_done} {'query blocks of one head' if kind != 'decode' else '(b,h) rows'}")
+    return flops, t_used, "; ".join(desc)
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, budget_s):
+    from threadpoolctl import threadpool_limits
+
+    with threadpool_limits(limits=cpu_cores()):
+        flops, secs, desc = oracle_sample(wl, budget_s)
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle, {secs:.1f} s: {desc}; useful FLOPs credited 4D/pair fwd, "
+                      f"6D/pair bwd dQ rows, 4D/row decode"}
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return
+    wl = workload(args.workload)
+    per_step = 1.5
+    for _ in range(args.warmup):
+        oracle_sample(wl, per_step / 3)
+    tot_f, tot_s, desc = 0.0, 0.0, ""
+    for _ in range(args.steps):
+        f, s, desc = oracle_sample(wl, per_step)
+        tot_f += f
+        tot_s += s
+    value = tot_f / tot_s / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16 upcast to f64)",
+        "config": {"workload": wl["workload"], "sample": "bounded oracle sample per step (see cpu_baseline)"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        reference_arm(args, rank, world)
+        return 0
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        cuda_arm(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
