@@ -28,14 +28,14 @@ __all__ = [
     "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd",
     "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd",
     "lg_sparse_decode_splits", "lg_sparse_decode_workspace", "lg_sparse_decode",
-    "lg_device_status", "EXPORTED_SYMBOLS",
+    "lg_sparse_decode_noalloc", "lg_device_status", "EXPORTED_SYMBOLS",
 ]
 
 EXPORTED_SYMBOLS = (
     "lg_strerror", "lg_version", "lg_pattern_expand", "lg_pattern_expand_t", "lg_pattern_pairs",
     "lg_pattern_iterate_device", "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd",
     "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd", "lg_sparse_decode_splits",
-    "lg_sparse_decode_workspace", "lg_sparse_decode", "lg_device_status",
+    "lg_sparse_decode_workspace", "lg_sparse_decode", "lg_sparse_decode_noalloc", "lg_device_status",
 )
 
 
@@ -80,6 +80,7 @@ _SIGS = {
     "lg_sparse_decode_splits": (_c_i32, [_c_i32] * 6 + [_P(_c_i32)]),
     "lg_sparse_decode_workspace": (_c_i32, [_c_i32] * 6 + [_P(_c_sz)]),
     "lg_sparse_decode": (_c_i32, [_c_vp] * 6 + [_c_i32] * 6 + [_c_f, _c_vp, _c_sz, _c_vp]),
+    "lg_sparse_decode_noalloc": (_c_i32, [_c_vp] * 6 + [_c_i32] * 6 + [_c_f, _c_vp]),
     "lg_device_status": (_c_i32, [_c_i32, _P(ctypes.c_uint32)]),
 }
 
@@ -279,6 +280,30 @@ def lg_sparse_decode(q, k_cache, v_cache, cache_lens, o, lse, scale: float, num_
     _check(lib().lg_sparse_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), cache_lens.data_ptr(),
                                   o.data_ptr(), _ptr(lse), B, H, Hkv, D, Lmax, int(num_splits), float(scale),
                                   _ptr(workspace), ws, _stream(stream)), "lg_sparse_decode")
+
+
+def lg_sparse_decode_noalloc(q, k_cache, v_cache, cache_lens, o, lse, scale: float, num_splits: int = 0,
+                             stream=None):
+    """lg_sparse_decode for callers that cannot allocate device memory: no
+    workspace argument; the library's fixed 16 MiB device scratch array holds
+    the split partials. Calls that overlap on the GPU share that array and race,
+    so serialise them. The first call on a device resolves the array's address;
+    make it before any stream capture."""
+    import torch
+
+    B, H, D = q.shape
+    Lmax, Hkv = k_cache.shape[1], k_cache.shape[2]
+    _expect(q, "q", torch.bfloat16, (B, H, D))
+    _expect(k_cache, "k_cache", torch.bfloat16, (B, Lmax, Hkv, D), q.device)
+    _expect(v_cache, "v_cache", torch.bfloat16, (B, Lmax, Hkv, D), q.device)
+    _expect(cache_lens, "cache_lens", torch.int32, (B,), q.device)
+    _expect(o, "o", torch.bfloat16, (B, H, D), q.device)
+    if lse is not None:
+        _expect(lse, "lse", torch.float32, (B, H), q.device)
+    _check(lib().lg_sparse_decode_noalloc(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                          cache_lens.data_ptr(), o.data_ptr(), _ptr(lse), B, H, Hkv, D, Lmax,
+                                          int(num_splits), float(scale), _stream(stream)),
+           "lg_sparse_decode_noalloc")
 
 
 # ---------------------------------------------------------------- diagnostics

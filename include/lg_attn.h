@@ -202,6 +202,38 @@ lg_status_t lg_sparse_decode(const void* q, const void* k_cache, const void* v_c
                              int32_t num_splits, float scale, void* workspace, size_t workspace_bytes,
                              lg_stream_t stream);
 
+/*
+ * Size of the fixed device scratch array behind lg_sparse_decode_noalloc:
+ * 16 MiB on every device that loads the library, held until process exit.
+ */
+#define LG_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/*
+ * lg_sparse_decode without a workspace, for callers that cannot allocate
+ * device memory. The paper has no counterpart: this is a deployment
+ * convenience. Typical such callers are a plugin inside a host framework that
+ * owns all device memory through its own pool and forbids side allocations, a
+ * latency-critical decode loop where cudaMalloc / cudaFree would synchronise
+ * the device and stall every other stream, and a thin C / FFI caller with no
+ * device allocator of its own. Arguments and results are those of
+ * lg_sparse_decode minus the workspace; the caller still passes all inputs
+ * and outputs. Nothing is allocated or freed.
+ * The split partials and tickets live in one file-scope device array of
+ * LG_DECODE_NOALLOC_SCRATCH_BYTES. The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress, with that device current);
+ * make that first call before any stream capture. With num_splits == 0 the
+ * automatic split count is lowered until the partials fit the array; an
+ * explicit num_splits whose partials need more than the array holds
+ * (B * H * num_splits * (D + 1) * 4 bytes, roughly) returns LG_ERR_WORKSPACE
+ * and launches nothing. Every call shares the array: the tickets are cleared
+ * on the given stream at each call, and calls that overlap on the GPU (other
+ * streams, other host threads) race on it, so serialise them.
+ */
+lg_status_t lg_sparse_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* cache_lens, void* o, float* lse, int32_t B, int32_t H,
+                                     int32_t Hkv, int32_t D, int32_t Lmax, int32_t num_splits, float scale,
+                                     lg_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Diagnostics                                                              */
 /* ------------------------------------------------------------------------ */
