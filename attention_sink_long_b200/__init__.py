@@ -73,10 +73,11 @@ _SIGS = {
     "lg_pattern_pairs": (_c_i32, [_P(_lg_pattern_t), _c_i32, _P(_c_i64)]),
     "lg_pattern_iterate_device": (_c_i32, [_P(_lg_pattern_t), _c_i32, _c_i32, _c_i32, _c_vp, _c_i32, _c_vp]),
     "lg_sparse_attn_fwd_workspace": (_c_i32, [_P(_lg_pattern_t)] + [_c_i32] * 5 + [_P(_c_sz)]),
-    "lg_sparse_attn_fwd": (_c_i32, [_P(_lg_pattern_t), _c_vp, _c_vp, _c_vp, _c_vp, _c_vp] + [_c_i32] * 5
+    "lg_sparse_attn_fwd": (_c_i32, [_P(_lg_pattern_t), _c_vp, _c_vp, _c_vp, _c_vp, _c_i32, _c_vp] + [_c_i32] * 5
                            + [_c_f, _c_vp, _c_sz, _c_vp]),
     "lg_sparse_attn_bwd_workspace": (_c_i32, [_P(_lg_pattern_t)] + [_c_i32] * 5 + [_P(_c_sz)]),
-    "lg_sparse_attn_bwd": (_c_i32, [_P(_lg_pattern_t)] + [_c_vp] * 9 + [_c_i32] * 5 + [_c_f, _c_vp, _c_sz, _c_vp]),
+    "lg_sparse_attn_bwd": (_c_i32, [_P(_lg_pattern_t)] + [_c_vp] * 4 + [_c_i32] + [_c_vp] * 5 + [_c_i32] * 6
+                           + [_c_f, _c_vp, _c_sz, _c_vp]),
     "lg_sparse_decode_splits": (_c_i32, [_c_i32] * 6 + [_P(_c_i32)]),
     "lg_sparse_decode_workspace": (_c_i32, [_c_i32] * 6 + [_P(_c_sz)]),
     "lg_sparse_decode": (_c_i32, [_c_vp] * 6 + [_c_i32] * 6 + [_c_f, _c_vp, _c_sz, _c_vp]),
@@ -201,8 +202,19 @@ def lg_sparse_attn_fwd_workspace(pattern, B, S, H, Hkv, D) -> int:
     return n.value
 
 
+def _dtype_code(t, name):
+    import torch
+
+    if t.dtype == torch.bfloat16:
+        return 0
+    if t.dtype == torch.float32:
+        return 1
+    raise TypeError(f"{name}: expected bfloat16 or float32, got {t.dtype}")
+
+
 def lg_sparse_attn_fwd(pattern, q, k, v, o, lse, scale: float, workspace=None, stream=None):
-    """q [B,S,H,D], k/v [B,S,Hkv,D], o [B,S,H,D] bf16 CUDA tensors; lse [B,H,S] fp32 or None."""
+    """q [B,S,H,D], k/v [B,S,Hkv,D] bf16 CUDA tensors; o [B,S,H,D] bf16 or fp32
+    (written); lse [B,H,S] fp32 or None."""
     import torch
 
     B, S, H, D = q.shape
@@ -210,12 +222,13 @@ def lg_sparse_attn_fwd(pattern, q, k, v, o, lse, scale: float, workspace=None, s
     _expect(q, "q", torch.bfloat16, (B, S, H, D))
     _expect(k, "k", torch.bfloat16, (B, S, Hkv, D), q.device)
     _expect(v, "v", torch.bfloat16, (B, S, Hkv, D), q.device)
-    _expect(o, "o", torch.bfloat16, (B, S, H, D), q.device)
+    odt = _dtype_code(o, "o")
+    _expect(o, "o", o.dtype, (B, S, H, D), q.device)
     if lse is not None:
         _expect(lse, "lse", torch.float32, (B, H, S), q.device)
     p = _pat(pattern)
     ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib().lg_sparse_attn_fwd(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+    _check(lib().lg_sparse_attn_fwd(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), odt,
                                     _ptr(lse), B, S, H, Hkv, D, float(scale), _ptr(workspace), ws, _stream(stream)),
            "lg_sparse_attn_fwd")
 
@@ -230,20 +243,26 @@ def lg_sparse_attn_bwd_workspace(pattern, B, S, H, Hkv, D) -> int:
 
 
 def lg_sparse_attn_bwd(pattern, q, k, v, o, dout, lse, dq, dk, dv, scale: float, workspace, stream=None):
-    """Gradients; dq/dk/dv bf16 outputs shaped like q/k/v; workspace a CUDA uint8 tensor."""
+    """Gradients into dq/dk/dv (shaped like q/k/v; all bf16, or all fp32 for the
+    unrounded accumulators). o is the forward output (bf16 or fp32); workspace
+    is a CUDA uint8 tensor."""
     import torch
 
     B, S, H, D = q.shape
     Hkv = k.shape[2]
-    for name, t, shp in (("q", q, (B, S, H, D)), ("o", o, (B, S, H, D)), ("dout", dout, (B, S, H, D)),
-                         ("dq", dq, (B, S, H, D)), ("k", k, (B, S, Hkv, D)), ("v", v, (B, S, Hkv, D)),
-                         ("dk", dk, (B, S, Hkv, D)), ("dv", dv, (B, S, Hkv, D))):
+    for name, t, shp in (("q", q, (B, S, H, D)), ("dout", dout, (B, S, H, D)),
+                         ("k", k, (B, S, Hkv, D)), ("v", v, (B, S, Hkv, D))):
         _expect(t, name, torch.bfloat16, shp, q.device)
+    odt = _dtype_code(o, "o")
+    _expect(o, "o", o.dtype, (B, S, H, D), q.device)
+    gdt = _dtype_code(dq, "dq")
+    for name, t, shp in (("dq", dq, (B, S, H, D)), ("dk", dk, (B, S, Hkv, D)), ("dv", dv, (B, S, Hkv, D))):
+        _expect(t, name, dq.dtype, shp, q.device)
     _expect(lse, "lse", torch.float32, (B, H, S), q.device)
     p = _pat(pattern)
     ws = workspace.numel() * workspace.element_size()
-    _check(lib().lg_sparse_attn_bwd(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                    dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+    _check(lib().lg_sparse_attn_bwd(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), odt,
+                                    dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), gdt,
                                     B, S, H, Hkv, D, float(scale), workspace.data_ptr(), ws, _stream(stream)),
            "lg_sparse_attn_bwd")
 

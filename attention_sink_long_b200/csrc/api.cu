@@ -213,13 +213,14 @@ lg_status_t lg_sparse_attn_fwd_workspace(const lg_pattern_t* p, int32_t B, int32
 }
 
 lg_status_t lg_sparse_attn_fwd(const lg_pattern_t* p, const void* q, const void* k, const void* v, void* o,
-                               float* lse, int32_t B, int32_t S, int32_t H, int32_t Hkv, int32_t D, float scale,
-                               void* workspace, size_t workspace_bytes, lg_stream_t stream) {
+                               int32_t o_dtype, float* lse, int32_t B, int32_t S, int32_t H, int32_t Hkv, int32_t D,
+                               float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream) {
   (void)workspace;
   (void)workspace_bytes;
   lg_status_t st = check_prefill_shape(p, B, S, H, Hkv, D);
   if (st != LG_OK) return st;
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return LG_ERR_INVALID_ARG;
+  if (o_dtype != LG_BF16 && o_dtype != LG_F32) return LG_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return LG_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return LG_ERR_UNSUPPORTED;
   unsigned int* err = error_word(&st);
@@ -228,10 +229,13 @@ lg_status_t lg_sparse_attn_fwd(const lg_pattern_t* p, const void* q, const void*
   if ((st = make_map(&tq, q, B, S, H, D, 128)) != LG_OK) return st;
   if ((st = make_map(&tk, k, B, S, Hkv, D, 64)) != LG_OK) return st;
   if ((st = make_map(&tv, v, B, S, Hkv, D, 64)) != LG_OK) return st;
-  if ((st = make_map(&to, o, B, S, H, D, 128)) != LG_OK) return st;
+  // With an fp32 O the kernel stores rows directly; the bf16 map is then built
+  // over q only to have a valid (unused) descriptor.
+  if ((st = make_map(&to, o_dtype == LG_F32 ? q : o, B, S, H, D, 128)) != LG_OK) return st;
   lg::FwdParams prm;
   prm.pat = *p;
   prm.lse = lse;
+  prm.o_f32 = o_dtype == LG_F32 ? static_cast<float*>(o) : nullptr;
   prm.S = S;
   prm.H = H;
   prm.Hkv = Hkv;
@@ -253,12 +257,15 @@ lg_status_t lg_sparse_attn_bwd_workspace(const lg_pattern_t* p, int32_t B, int32
 }
 
 lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* p, const void* q, const void* k, const void* v, const void* o,
-                               const void* dout, const float* lse, void* dq, void* dk, void* dv, int32_t B, int32_t S,
-                               int32_t H, int32_t Hkv, int32_t D, float scale, void* workspace,
-                               size_t workspace_bytes, lg_stream_t stream) {
+                               int32_t o_dtype, const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                               int32_t grad_dtype, int32_t B, int32_t S, int32_t H, int32_t Hkv, int32_t D,
+                               float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream) {
   lg_status_t st = check_prefill_shape(p, B, S, H, Hkv, D);
   if (st != LG_OK) return st;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return LG_ERR_INVALID_ARG;
+  if (grad_dtype != LG_BF16 && grad_dtype != LG_F32) return LG_ERR_INVALID_ARG;
+  if (o_dtype != LG_BF16 && o_dtype != LG_F32) return LG_ERR_INVALID_ARG;
+  const int grad_f32 = grad_dtype == LG_F32;
   if (!(scale > 0.f) || !isfinite(scale)) return LG_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
@@ -278,10 +285,12 @@ lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* p, const void* q, const void*
   if ((st = make_map(&tk, k, B, S, Hkv, D, 128)) != LG_OK) return st;
   if ((st = make_map(&tv, v, B, S, Hkv, D, 128)) != LG_OK) return st;
   if ((st = make_map(&tdo, dout, B, S, H, D, 64)) != LG_OK) return st;
-  if ((st = make_map(&tdk, dk, B, S, Hkv, D, 128)) != LG_OK) return st;
-  if ((st = make_map(&tdv, dv, B, S, Hkv, D, 128)) != LG_OK) return st;
+  // With fp32 gradients the kernel stores dK / dV directly; the bf16 maps are
+  // then built over K / V only to have valid (unused) descriptors.
+  if ((st = make_map(&tdk, grad_f32 ? k : dk, B, S, Hkv, D, 128)) != LG_OK) return st;
+  if ((st = make_map(&tdv, grad_f32 ? v : dv, B, S, Hkv, D, 128)) != LG_OK) return st;
 
-  st = cuda_status(lg::launch_bwd_pre(o, dout, delta, dq_acc, B, S, H, D, s));
+  st = cuda_status(lg::launch_bwd_pre(o, o_dtype == LG_F32, dout, delta, dq_acc, B, S, H, D, s));
   if (st != LG_OK) return st;
   lg::BwdParams prm;
   prm.pat = *p;
@@ -296,10 +305,17 @@ lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* p, const void* q, const void*
   prm.nkt = (S + 127) / 128;
   prm.scale = scale;
   prm.scale_log2 = scale * 1.4426950408889634f;
+  // dK and dV of a KV head sum over its H / Hkv query heads, so their size
+  // grows with the group; the bf16 residuals of P and dS then keep the bf16
+  // rounding of those operands out of dV and dK.
+  prm.split_lo = (H / Hkv) > 1;
+  prm.grad_f32 = grad_f32;
+  prm.dk_f32 = grad_f32 ? static_cast<float*>(dk) : nullptr;
+  prm.dv_f32 = grad_f32 ? static_cast<float*>(dv) : nullptr;
   prm.err = err;
   st = cuda_status(lg::launch_bwd(D, tq, tk, tv, tdo, tdk, tdv, prm, B, s));
   if (st != LG_OK) return st;
-  return cuda_status(lg::launch_bwd_dq(dq_acc, dq, scale, B, S, H, D, s));
+  return cuda_status(lg::launch_bwd_dq(dq_acc, dq, grad_f32, scale, B, S, H, D, s));
 }
 
 // ---------------------------------------------------------------- decode

@@ -17,8 +17,8 @@ namespace lg {
 // ---------------------------------------------------------------------------
 // 1. Delta and dQ_acc clearing. One thread per 8 elements of a row.
 // ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(256) lg_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
+template <int D, bool OF32>
+__global__ void __launch_bounds__(256) lg_bwd_pre_kernel(const void* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dout,
                                                          float* __restrict__ delta, float* __restrict__ dq_acc,
                                                          int B, int S, int H) {
@@ -29,14 +29,27 @@ __global__ void __launch_bounds__(256) lg_bwd_pre_kernel(const __nv_bfloat16* __
   const int c = (int)(t % TPR);
   float acc = 0.f;
   if (row < rows) {
-    const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + 8 * c);
+    float of[8];
+    if constexpr (OF32) {
+      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(o) + row * D + 8 * c);
+      const float4 x0 = src[0], x1 = src[1];
+      of[0] = x0.x; of[1] = x0.y; of[2] = x0.z; of[3] = x0.w;
+      of[4] = x1.x; of[5] = x1.y; of[6] = x1.z; of[7] = x1.w;
+    } else {
+      const uint4 a = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(o) + row * D + 8 * c);
+      const uint32_t aa[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        of[2 * e] = __uint_as_float(aa[e] << 16);
+        of[2 * e + 1] = __uint_as_float(aa[e] & 0xffff0000u);
+      }
+    }
     const uint4 g = *reinterpret_cast<const uint4*>(dout + row * D + 8 * c);
-    const uint32_t aa[4] = {a.x, a.y, a.z, a.w};
     const uint32_t gg[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      acc = fmaf(__uint_as_float(aa[e] << 16), __uint_as_float(gg[e] << 16), acc);
-      acc = fmaf(__uint_as_float(aa[e] & 0xffff0000u), __uint_as_float(gg[e] & 0xffff0000u), acc);
+      acc = fmaf(of[2 * e], __uint_as_float(gg[e] << 16), acc);
+      acc = fmaf(of[2 * e + 1], __uint_as_float(gg[e] & 0xffff0000u), acc);
     }
   }
 #pragma unroll
@@ -54,17 +67,18 @@ __global__ void __launch_bounds__(256) lg_bwd_pre_kernel(const __nv_bfloat16* __
   }
 }
 
-cudaError_t launch_bwd_pre(const void* o, const void* dout, float* delta, float* dq_acc, int B, int S, int H, int D,
-                           cudaStream_t stream) {
+cudaError_t launch_bwd_pre(const void* o, int o_f32, const void* dout, float* delta, float* dq_acc, int B, int S,
+                           int H, int D, cudaStream_t stream) {
   const long long threads = (long long)B * S * H * (D / 8);
   const unsigned int blocks = (unsigned int)((threads + 255) / 256);
-  if (D == 64)
-    lg_bwd_pre_kernel<64><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
-                                                      static_cast<const __nv_bfloat16*>(dout), delta, dq_acc, B, S, H);
-  else
-    lg_bwd_pre_kernel<128><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
-                                                       static_cast<const __nv_bfloat16*>(dout), delta, dq_acc, B, S,
-                                                       H);
+  const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(dout);
+  if (D == 64) {
+    if (o_f32) lg_bwd_pre_kernel<64, true><<<blocks, 256, 0, stream>>>(o, g, delta, dq_acc, B, S, H);
+    else lg_bwd_pre_kernel<64, false><<<blocks, 256, 0, stream>>>(o, g, delta, dq_acc, B, S, H);
+  } else {
+    if (o_f32) lg_bwd_pre_kernel<128, true><<<blocks, 256, 0, stream>>>(o, g, delta, dq_acc, B, S, H);
+    else lg_bwd_pre_kernel<128, false><<<blocks, 256, 0, stream>>>(o, g, delta, dq_acc, B, S, H);
+  }
   return cudaGetLastError();
 }
 
@@ -73,8 +87,8 @@ cudaError_t launch_bwd_pre(const void* o, const void* dout, float* delta, float*
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) lg_bwd_dq_kernel(const float* __restrict__ dq_acc,
-                                                        __nv_bfloat16* __restrict__ dq, float scale, int B, int S,
-                                                        int H) {
+                                                        __nv_bfloat16* __restrict__ dq, float* __restrict__ dq_f32,
+                                                        float scale, int B, int S, int H) {
   constexpr int TPR = D / 8;
   const long long rows = (long long)B * S * H;
   const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -88,6 +102,12 @@ __global__ void __launch_bounds__(256) lg_bwd_dq_kernel(const float* __restrict_
   const long long srow = ((long long)b * H + h) * S + s;
   const float4* src = reinterpret_cast<const float4*>(dq_acc + srow * D + 8 * c);
   const float4 x0 = src[0], x1 = src[1];
+  if (dq_f32 != nullptr) {
+    float4* dst = reinterpret_cast<float4*>(dq_f32 + row * D + 8 * c);
+    dst[0] = make_float4(x0.x * scale, x0.y * scale, x0.z * scale, x0.w * scale);
+    dst[1] = make_float4(x1.x * scale, x1.y * scale, x1.z * scale, x1.w * scale);
+    return;
+  }
   uint4 out;
   out.x = pack_bf16x2(x0.x * scale, x0.y * scale);
   out.y = pack_bf16x2(x0.z * scale, x0.w * scale);
@@ -96,25 +116,456 @@ __global__ void __launch_bounds__(256) lg_bwd_dq_kernel(const float* __restrict_
   *reinterpret_cast<uint4*>(dq + row * D + 8 * c) = out;
 }
 
-cudaError_t launch_bwd_dq(const float* dq_acc, void* dq, float scale, int B, int S, int H, int D,
+cudaError_t launch_bwd_dq(const float* dq_acc, void* dq, int dq_f32, float scale, int B, int S, int H, int D,
                           cudaStream_t stream) {
   const long long threads = (long long)B * S * H * (D / 8);
   const unsigned int blocks = (unsigned int)((threads + 255) / 256);
+  __nv_bfloat16* qb = dq_f32 ? nullptr : static_cast<__nv_bfloat16*>(dq);
+  float* qf = dq_f32 ? static_cast<float*>(dq) : nullptr;
   if (D == 64)
-    lg_bwd_dq_kernel<64><<<blocks, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), scale, B, S, H);
+    lg_bwd_dq_kernel<64><<<blocks, 256, 0, stream>>>(dq_acc, qb, qf, scale, B, S, H);
   else
-    lg_bwd_dq_kernel<128><<<blocks, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), scale, B, S, H);
+    lg_bwd_dq_kernel<128><<<blocks, 256, 0, stream>>>(dq_acc, qb, qf, scale, B, S, H);
   return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
-// 2. main kernel -- not yet available.
+// 2. main kernel.
+//
+// CTA per (128-row KV tile = KV blocks 2u and 2u+1, KV head, batch); it walks
+// the union of the two blocks' query-block lists (a contiguous range, see
+// QIter) for every query head of the KV head's group, one 64-row query block
+// per step. Per step, all on tcgen05 with fp32 accumulation in TMEM:
+//   S^T  = K Q_i^T          (M=128 kv, N=64 q, K=D)
+//   dP^T = V dO_i^T         (M=128,    N=64,   K=D)
+//   dV  += P^T dO_i         (M=128,    N=D,    K=64; P^T as a bf16 hi + lo pair)
+//   dK  += dS^T Q_i         (M=128,    N=D,    K=64)
+//   dQ_i^T = K^T dS^T       (M=D,      N=64,   K=128)
+// with P^T = exp(scale S^T - LSE) on the mask and dS^T = P^T (dP^T - Delta),
+// computed by four warps that each own 32 KV rows (TMEM lanes), written to
+// shared memory as bf16 in the 128B-swizzled K-major layout the MMA reads.
+// With GQA (H / Hkv > 1) dV and dK sum over the group's query heads and grow
+// with it, so P^T and dS^T then go in twice, as bf16(x) and the residual
+// bf16(x - bf16(x)): dV and dK then carry no bf16 rounding of P or dS (a
+// single bf16 operand costs ~2^-9 relative per term, which at |dK| ~ 4 is the
+// whole 1e-2 error budget). Without GQA the plain five GEMMs are used.
+// dQ_i^T is read back by a second group of four warps, transposed through
+// shared memory and added to the fp32 dQ accumulator with one bulk
+// reduce-add per step. S/dP of step n+1 are issued before the gradient GEMMs
+// of step n, so the exponentials of one step overlap the GEMMs of the other.
+//
+// Warps: 0-3 P/dS + epilogue, 4 TMA producer, 5 TMEM owner + MMA issuer,
+// 6-9 dQ drain. TMEM columns: dV [0,D), dK [D,2D), S^T [2D,2D+64),
+// dP^T [2D+64,2D+128), dQ^T double buffer [2D+128, 2D+256).
 // ---------------------------------------------------------------------------
+template <int D>
+struct BwdLayout {
+  static constexpr int KV_BYTES = 128 * D * 2;  // K or V tile (128 rows)
+  static constexpr int QB_BYTES = 64 * D * 2;   // Q or dO block (64 rows)
+  static constexpr int PT_BYTES = 128 * 64 * 2;  // P^T or dS^T (bf16)
+  static constexpr int DQS_BYTES = 64 * D * 4;   // dQ staging (fp32, [q][d])
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + KV_BYTES;
+  static constexpr int OFF_Q = OFF_V + KV_BYTES;      // 2 stages
+  static constexpr int OFF_DO = OFF_Q + 2 * QB_BYTES;  // 2 stages
+  static constexpr int OFF_PT = OFF_DO + 2 * QB_BYTES;  // bf16(P^T)
+  static constexpr int OFF_PL = OFF_PT + PT_BYTES;       // bf16(P^T - bf16(P^T))
+  static constexpr int OFF_DST = OFF_PL + PT_BYTES;      // bf16(dS^T)
+  static constexpr int OFF_DSL = OFF_DST + PT_BYTES;     // bf16(dS^T - bf16(dS^T))
+  static constexpr int OFF_DQS = OFF_DSL + PT_BYTES;
+  static constexpr int OFF_LSE = OFF_DQS + DQS_BYTES;  // 2 stages x 64 fp32
+  static constexpr int OFF_DEL = OFF_LSE + 512;        // 2 stages x 64 fp32
+  static constexpr int OFF_BAR = OFF_DEL + 512;
+  static constexpr int NBAR = 16;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t T_DV = 0, T_DK = D, T_S = 2 * D, T_DP = 2 * D + 64, T_DQ = 2 * D + 128;
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    lg_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                  const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
+                  const BwdParams prm) {
+  using L = BwdLayout<D>;
+  constexpr int DP = D / 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;    // [2]
+  uint64_t* q_empty = bars + 3;   // [2]
+  uint64_t* s_full = bars + 5;
+  uint64_t* dp_full = bars + 6;
+  uint64_t* st_free = bars + 7;
+  uint64_t* p_full = bars + 8;
+  uint64_t* ds_full = bars + 9;
+  uint64_t* pds_free = bars + 10;
+  uint64_t* dq_full = bars + 11;  // [2]
+  uint64_t* dq_free = bars + 13;  // [2]
+  uint64_t* acc_done = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+  const float* s_lse = reinterpret_cast<const float*>(smem + L::OFF_LSE);
+  const float* s_del = reinterpret_cast<const float*>(smem + L::OFF_DEL);
+  float* s_dq = reinterpret_cast<float*>(smem + L::OFF_DQS);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int u = blockIdx.x;
+  const int kvh = blockIdx.y;
+  const int b = blockIdx.z;
+  const int G = prm.H / prm.Hkv;
+  const int j_lo = 2 * u;
+  const int j_hi = imin(2 * u + 1, prm.nqb - 1);
+  const QIter qit(prm.pat, j_lo, j_hi, prm.nqb);
+  const int cnt = qit.count();
+  const int N = G * cnt;
+  unsigned int* err = prm.err;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1 + 128);
+      mbar_init(&dq_full[s], 1);
+      mbar_init(&dq_free[s], 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(ds_full, 128);
+    mbar_init(pds_free, 1);
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(st_free, 128);
+    mbar_init(acc_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(kv_full, 2 * L::KV_BYTES);
+      for (int p = 0; p < DP; ++p) {
+        tma_load_4d(smem + L::OFF_K + p * 16384, &tmK, kv_full, 64 * p, kvh, 128 * u, b);
+        tma_load_4d(smem + L::OFF_V + p * 16384, &tmV, kv_full, 64 * p, kvh, 128 * u, b);
+      }
+      for (int n = 0; n < N; ++n) {
+        const int h = kvh * G + n / cnt;
+        const int i = qit.first_blk + n % cnt;
+        const int st = n & 1;
+        const uint32_t use = (uint32_t)(n >> 1);
+        if (use > 0 && !mbar_wait(&q_empty[st], (use - 1) & 1, abort_flag, err, kErrBwdWait)) break;
+        mbar_arrive_expect_tx(&q_full[st], 2 * L::QB_BYTES + 512);
+        for (int p = 0; p < DP; ++p) {
+          tma_load_4d(smem + L::OFF_Q + st * L::QB_BYTES + p * 8192, &tmQ, &q_full[st], 64 * p, h, 64 * i, b);
+          tma_load_4d(smem + L::OFF_DO + st * L::QB_BYTES + p * 8192, &tmdO, &q_full[st], 64 * p, h, 64 * i, b);
+        }
+        const size_t row = ((size_t)b * prm.H + h) * prm.S + 64 * (size_t)i;
+        bulk_load(smem + L::OFF_LSE + st * 256, prm.lse + row, 256, &q_full[st]);
+        bulk_load(smem + L::OFF_DEL + st * 256, prm.delta + row, 256, &q_full[st]);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(128, 64, false, false);
+      constexpr uint32_t idesc_g = idesc_bf16(128, D, false, true);
+      constexpr uint32_t idesc_q = idesc_bf16(D, 64, true, true);
+      const uint32_t aK = sbase + L::OFF_K, aV = sbase + L::OFF_V;
+      auto grad = [&](int m) -> bool {
+        const int bb = m & 1;
+        const uint32_t use = (uint32_t)(m >> 1);
+        const uint32_t aQ = sbase + L::OFF_Q + bb * L::QB_BYTES;
+        const uint32_t aDO = sbase + L::OFF_DO + bb * L::QB_BYTES;
+        const uint32_t aPT = sbase + L::OFF_PT;
+        const uint32_t aPL = sbase + L::OFF_PL;
+        const uint32_t aDS = sbase + L::OFF_DST;
+        if (!mbar_wait(p_full, (uint32_t)m & 1, abort_flag, err, kErrBwdWait)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_ss(tmem + L::T_DV, sdesc_sw128(aPT + kk * 32, 16, 1024), sdesc_sw128(aDO + kk * 2048, 8192, 1024),
+                    idesc_g, (m > 0 || kk > 0) ? 1u : 0u);
+        if (prm.split_lo) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_ss(tmem + L::T_DV, sdesc_sw128(aPL + kk * 32, 16, 1024),
+                      sdesc_sw128(aDO + kk * 2048, 8192, 1024), idesc_g, 1u);
+        }
+        if (!mbar_wait(ds_full, (uint32_t)m & 1, abort_flag, err, kErrBwdWait)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_ss(tmem + L::T_DK, sdesc_sw128(aDS + kk * 32, 16, 1024), sdesc_sw128(aQ + kk * 2048, 8192, 1024),
+                    idesc_g, (m > 0 || kk > 0) ? 1u : 0u);
+        if (prm.split_lo) {
+          const uint32_t aDL = sbase + L::OFF_DSL;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_ss(tmem + L::T_DK, sdesc_sw128(aDL + kk * 32, 16, 1024), sdesc_sw128(aQ + kk * 2048, 8192, 1024),
+                      idesc_g, 1u);
+        }
+        if (use > 0 && !mbar_wait(&dq_free[bb], (use - 1) & 1, abort_flag, err, kErrBwdWait)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_ss(tmem + L::T_DQ + 64 * bb, sdesc_sw128(aK + kk * 2048, 16384, 1024),
+                    sdesc_sw128(aDS + kk * 2048, 8192, 1024), idesc_q, kk > 0 ? 1u : 0u);
+        tc_commit(&dq_full[bb]);
+        tc_commit(pds_free);
+        tc_commit(&q_empty[bb]);
+        return true;
+      };
+      bool ok = mbar_wait(kv_full, 0, abort_flag, err, kErrBwdWait);
+      for (int n = 0; n < N && ok; ++n) {
+        const int st = n & 1;
+        const uint32_t use = (uint32_t)(n >> 1);
+        if (!mbar_wait(&q_full[st], use & 1, abort_flag, err, kErrBwdWait)) { ok = false; break; }
+        if (n >= 1 && !mbar_wait(st_free, (uint32_t)(n - 1) & 1, abort_flag, err, kErrBwdWait)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t aQ = sbase + L::OFF_Q + st * L::QB_BYTES;
+        const uint32_t aDO = sbase + L::OFF_DO + st * L::QB_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ka = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint32_t kb = (kk >> 2) * 8192 + (kk & 3) * 32;
+          tc_mma_ss(tmem + L::T_S, sdesc_sw128(aK + ka, 16, 1024), sdesc_sw128(aQ + kb, 16, 1024), idesc_s,
+                    kk > 0 ? 1u : 0u);
+        }
+        tc_commit(s_full);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ka = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint32_t kb = (kk >> 2) * 8192 + (kk & 3) * 32;
+          tc_mma_ss(tmem + L::T_DP, sdesc_sw128(aV + ka, 16, 1024), sdesc_sw128(aDO + kb, 16, 1024), idesc_s,
+                    kk > 0 ? 1u : 0u);
+        }
+        tc_commit(dp_full);
+        if (n >= 1 && !grad(n - 1)) { ok = false; break; }
+      }
+      if (ok && N > 0) ok = grad(N - 1);
+      tc_commit(acc_done);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ P / dS warps
+    const int r = threadIdx.x;  // KV row of the tile == TMEM lane
+    const int kvb = 2 * u + (r >> 6);
+    const int rr = r & 63;
+    const bool krow_live = kvb < prm.nqb;
+    const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
+    const float sl2 = prm.scale_log2;
+    constexpr float kLog2e = 1.4426950408889634f;
+    int n = 0;
+    for (; n < N; ++n) {
+      const int i = qit.first_blk + n % cnt;
+      const int st = n & 1;
+      const uint32_t use = (uint32_t)(n >> 1);
+      const bool vis = krow_live && in_list(prm.pat, i, kvb);
+      const bool diag = (i == kvb);
+      if (!__all_sync(0xffffffffu, mbar_wait(&q_full[st], use & 1, abort_flag, err, kErrBwdWait))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full, (uint32_t)n & 1, abort_flag, err, kErrBwdWait))) break;
+      tc_fence_after();
+      float pf[64];
+      {
+        uint32_t sr[64];
+        tmem_ld64(t_lane + L::T_S, sr);
+        const float* lse = s_lse + st * 64;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float x = fmaf(__uint_as_float(sr[c]), sl2, -lse[c] * kLog2e);
+          const bool keep = vis && (!diag || rr <= c);
+          pf[c] = keep ? ex2_approx(x) : 0.f;
+        }
+      }
+      // P^T / dS^T buffers are free once the gradient GEMMs of step n-1 completed.
+      if (n >= 1 &&
+          !__all_sync(0xffffffffu, mbar_wait(pds_free, (uint32_t)(n - 1) & 1, abort_flag, err, kErrBwdWait)))
+        break;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p0 = pf[8 * c + 2 * e], p1 = pf[8 * c + 2 * e + 1];
+          hi[e] = pack_bf16x2(p0, p1);
+          lo[e] = pack_bf16x2(p0 - __uint_as_float(hi[e] << 16), p1 - __uint_as_float(hi[e] & 0xffff0000u));
+        }
+        const uint32_t off = sw128_offset(r, c);
+        st_shared_v4(sbase + L::OFF_PT + off, hi[0], hi[1], hi[2], hi[3]);
+        if (prm.split_lo) st_shared_v4(sbase + L::OFF_PL + off, lo[0], lo[1], lo[2], lo[3]);
+      }
+      fence_async_smem();
+      mbar_arrive(p_full);
+      if (!__all_sync(0xffffffffu, mbar_wait(dp_full, (uint32_t)n & 1, abort_flag, err, kErrBwdWait))) break;
+      tc_fence_after();
+      uint32_t dpr[64];
+      tmem_ld64(t_lane + L::T_DP, dpr);
+      tc_fence_before();
+      mbar_arrive(st_free);
+      const float* del = s_del + st * 64;
+      const uint32_t drow = sbase + L::OFF_DST;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float d8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) d8[e] = pf[8 * c + e] * (__uint_as_float(dpr[8 * c + e]) - del[8 * c + e]);
+        uint32_t hi[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) hi[e] = pack_bf16x2(d8[2 * e], d8[2 * e + 1]);
+        st_shared_v4(drow + sw128_offset(r, c), hi[0], hi[1], hi[2], hi[3]);
+        if (prm.split_lo) {
+          uint32_t lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            lo[e] = pack_bf16x2(d8[2 * e] - __uint_as_float(hi[e] << 16),
+                                d8[2 * e + 1] - __uint_as_float(hi[e] & 0xffff0000u));
+          st_shared_v4(sbase + L::OFF_DSL + sw128_offset(r, c), lo[0], lo[1], lo[2], lo[3]);
+        }
+      }
+      fence_async_smem();
+      mbar_arrive(ds_full);
+      mbar_arrive(&q_empty[st]);
+    }
+
+    // ------------------------------------------------------------ dK, dV epilogue
+    bool ok = (n == N) && !*abort_flag;
+    if (ok) ok = mbar_wait(acc_done, 0, abort_flag, err, kErrBwdWait);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok && prm.grad_f32) {
+      // fp32 gradients: each thread stores its KV row straight from TMEM.
+      tc_fence_after();
+      const int krow = 128 * u + r;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tcol = which == 0 ? L::T_DV : L::T_DK;
+        const float mul = which == 0 ? 1.f : prm.scale;
+        float* dst = (which == 0 ? prm.dv_f32 : prm.dk_f32) + (((size_t)b * prm.S + krow) * prm.Hkv + kvh) * D;
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t o[32];
+          tmem_ld32(t_lane + tcol + 32 * ch, o);
+          if (krow < prm.S) {
+            float4* d4 = reinterpret_cast<float4*>(dst + 32 * ch);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              d4[e] = make_float4(__uint_as_float(o[4 * e]) * mul, __uint_as_float(o[4 * e + 1]) * mul,
+                                  __uint_as_float(o[4 * e + 2]) * mul, __uint_as_float(o[4 * e + 3]) * mul);
+          }
+        }
+      }
+    } else if (ok) {
+      tc_fence_after();
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tcol = which == 0 ? L::T_DV : L::T_DK;
+        const float mul = which == 0 ? 1.f : prm.scale;
+        const uint32_t dst = sbase + (which == 0 ? L::OFF_V : L::OFF_K);
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t o[32];
+          tmem_ld32(t_lane + tcol + 32 * ch, o);
+          const uint32_t panel = dst + (uint32_t)((32 * ch) >> 6) * 16384;
+          const int c0 = ((32 * ch) & 63) >> 3;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const float* f = reinterpret_cast<const float*>(&o[8 * q4]);
+            st_shared_v4(panel + sw128_offset(r, c0 + q4), pack_bf16x2(f[0] * mul, f[1] * mul),
+                         pack_bf16x2(f[2] * mul, f[3] * mul), pack_bf16x2(f[4] * mul, f[5] * mul),
+                         pack_bf16x2(f[6] * mul, f[7] * mul));
+          }
+        }
+      }
+    }
+    fence_async_smem();
+    named_bar_sync(1, 128);
+    if (r == 0 && !*abort_flag && !prm.grad_f32) {
+      for (int p = 0; p < DP; ++p) {
+        tma_store_4d(&tmdV, smem + L::OFF_V + p * 16384, 64 * p, kvh, 128 * u, b);
+        tma_store_4d(&tmdK, smem + L::OFF_K + p * 16384, 64 * p, kvh, 128 * u, b);
+      }
+      bulk_commit();
+      bulk_wait_all();
+    }
+  } else {
+    // ------------------------------------------------------------ dQ drain warps 6-9
+    const int t = threadIdx.x - 192;
+    const int quarter = warp & 3;
+    // dQ^T row (= d) held by this thread: M = D rows; for M = 64 the rows sit in
+    // lanes 0-15 of each 32-lane quarter.
+    const int d = (D == 128) ? quarter * 32 + lane : quarter * 16 + lane;
+    const bool dvalid = (D == 128) || lane < 16;
+    const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
+    bool ok = true;
+    for (int n = 0; n < N; ++n) {
+      const int h = kvh * G + n / cnt;
+      const int i = qit.first_blk + n % cnt;
+      const int bb = n & 1;
+      const uint32_t use = (uint32_t)(n >> 1);
+      ok = ok && mbar_wait(&dq_full[bb], use & 1, abort_flag, err, kErrBwdWait);
+      const bool wok = __all_sync(0xffffffffu, ok);
+      if (wok) {
+        tc_fence_after();
+        uint32_t v[64];
+        tmem_ld64(t_lane + L::T_DQ + 64 * bb, v);
+        tc_fence_before();
+        mbar_arrive(&dq_free[bb]);
+        if (dvalid) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s_dq[c * D + d] = __uint_as_float(v[c]);
+        }
+      }
+      fence_async_smem();
+      named_bar_sync(2, 128);
+      if (t == 0 && !*abort_flag) {
+        float* dst = prm.dq_acc + (((size_t)b * prm.H + h) * prm.S + 64 * (size_t)i) * D;
+        bulk_reduce_add_f32(dst, s_dq, 64 * D * 4);
+        bulk_commit();
+        bulk_wait_read_all();
+      }
+      named_bar_sync(2, 128);
+    }
+    if (t == 0) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+template <int D>
+static cudaError_t launch_bwd_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                   const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
+                                   const BwdParams& prm, int B, cudaStream_t stream) {
+  using L = BwdLayout<D>;
+  cudaError_t e = cudaFuncSetAttribute(lg_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+  if (e != cudaSuccess) return e;
+  dim3 grid(prm.nkt, prm.Hkv, B);
+  lg_bwd_kernel<D><<<grid, 320, L::ALLOC, stream>>>(tq, tk, tv, tdo, tdk, tdv, prm);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_bwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv, const BwdParams& prm,
                        int B, cudaStream_t stream) {
-  (void)D; (void)tq; (void)tk; (void)tv; (void)tdo; (void)tdk; (void)tdv; (void)prm; (void)B; (void)stream;
-  return cudaErrorNotSupported;
+  if (D == 64) return launch_bwd_impl<64>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
+  return launch_bwd_impl<128>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
 }
 
 }  // namespace lg

@@ -284,7 +284,25 @@ __global__ void __launch_bounds__(192, 1)
       ok = mbar_wait(&pv_done[lb], lu & 1, abort_flag, err, kErrFwdWait);
     }
     ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
+    const int srow = 128 * tile + r;
+    if (ok && prm.o_f32 != nullptr) {
+      // fp32 output: each thread stores its row straight from TMEM.
+      tc_fence_after();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      float* dst = prm.o_f32 + (((size_t)b * prm.S + srow) * prm.H + h) * D;
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t o[32];
+        tmem_ld32(t_lane + (uint32_t)(32 * ch), o);
+        if (row_live && srow < prm.S) {
+          float4* d4 = reinterpret_cast<float4*>(dst + 32 * ch);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            d4[e] = make_float4(__uint_as_float(o[4 * e]) * inv_l, __uint_as_float(o[4 * e + 1]) * inv_l,
+                                __uint_as_float(o[4 * e + 2]) * inv_l, __uint_as_float(o[4 * e + 3]) * inv_l);
+        }
+      }
+    } else if (ok) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
@@ -301,15 +319,14 @@ __global__ void __launch_bounds__(192, 1)
                        pack_bf16x2(f[6] * inv_l, f[7] * inv_l));
         }
       }
-      const int srow = 128 * tile + r;
-      if (prm.lse != nullptr && row_live && srow < prm.S) {
-        const float lse = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-        prm.lse[((size_t)b * prm.H + h) * prm.S + srow] = lse;
-      }
+    }
+    if (ok && prm.lse != nullptr && row_live && srow < prm.S) {
+      const float lse = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      prm.lse[((size_t)b * prm.H + h) * prm.S + srow] = lse;
     }
     fence_async_smem();
     named_bar_sync(1, 128);
-    if (r == 0 && !*abort_flag) {
+    if (r == 0 && !*abort_flag && prm.o_f32 == nullptr) {
       for (int p = 0; p < L::DP; ++p) tma_store_4d(&tmO, smem + L::OFF_Q + p * 16384, 64 * p, h, 128 * tile, b);
       bulk_commit();
       bulk_wait_all();

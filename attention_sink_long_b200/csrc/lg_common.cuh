@@ -112,6 +112,18 @@ __device__ __forceinline__ void bulk_reduce_add_f32(float* gdst, const void* sme
                : "memory");
 }
 
+// Contiguous global -> shared copy completing on an mbarrier (addresses 16-byte
+// aligned, bytes % 16 == 0); no multicast.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
 // Generic-proxy writes to shared memory become visible to the async proxy (TMA, tcgen05).
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 

@@ -11,7 +11,8 @@ namespace lg {
 
 struct FwdParams {
   lg_pattern_t pat;
-  float* lse;  // [B, H, S] or nullptr
+  float* lse;    // [B, H, S] or nullptr
+  float* o_f32;  // [B, S, H, D] fp32 output, or nullptr for the bf16 TMA-stored output
   int S, H, Hkv;
   int nqb;  // S / 64
   int nqt;  // ceil(S / 128)
@@ -32,15 +33,19 @@ struct BwdParams {
   int nkt;  // ceil(S / 128) KV tiles
   float scale;       // softmax scale
   float scale_log2;  // scale * log2(e)
+  int split_lo;      // 1: P and dS also enter dV / dK as bf16 residuals (GQA groups)
+  int grad_f32;      // 1: dK / dV written as fp32 straight from the accumulators
+  float* dk_f32;     // [B, S, Hkv, D] when grad_f32
+  float* dv_f32;
   unsigned int* err;
 };
 
-cudaError_t launch_bwd_pre(const void* o, const void* dout, float* delta, float* dq_acc, int B, int S, int H, int D,
-                           cudaStream_t stream);
+cudaError_t launch_bwd_pre(const void* o, int o_f32, const void* dout, float* delta, float* dq_acc, int B, int S,
+                           int H, int D, cudaStream_t stream);
 cudaError_t launch_bwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv, const BwdParams& prm,
                        int B, cudaStream_t stream);
-cudaError_t launch_bwd_dq(const float* dq_acc, void* dq, float scale, int B, int S, int H, int D,
+cudaError_t launch_bwd_dq(const float* dq_acc, void* dq, int dq_f32, float scale, int B, int S, int H, int D,
                           cudaStream_t stream);
 
 struct DecodeParams {

@@ -23,8 +23,8 @@
  *     exception, lg_device_status, says so). Pointers marked "device" must be
  *     device memory of the current device, 16-byte aligned.
  *   - Tensors are contiguous, row-major, with the layouts given per call:
- *       q, o, dout, dq   [B, S, H, D]    bf16
- *       k, v, dk, dv     [B, S, Hkv, D]  bf16
+ *       q, o, dout, dq   [B, S, H, D]    bf16 (o, dq may be fp32, see lg_dtype_t)
+ *       k, v, dk, dv     [B, S, Hkv, D]  bf16 (dk, dv may be fp32)
  *       lse              [B, H, S]       fp32, natural log
  *     Query head h reads KV head h / (H / Hkv).
  *   - Launch errors map to LG_ERR_CUDA. Asynchronous device faults surface at
@@ -82,6 +82,15 @@ const char* lg_strerror(lg_status_t status);
 /* ABI version of this library, (major << 16) | minor. */
 int32_t lg_version(void);
 
+/*
+ * Element type of the forward output O (and of O as an input of the
+ * backward) and of the gradient outputs. LG_BF16 rounds to nearest even and
+ * is the training format; LG_F32 keeps the fp32 accumulators as they are --
+ * the backward's Delta = rowsum(dO * O) is then exact to fp32, and parity can
+ * be checked apart from the output rounding.
+ */
+typedef enum { LG_BF16 = 0, LG_F32 = 1 } lg_dtype_t;
+
 /* ------------------------------------------------------------------------ */
 /* Pattern expansion (host, pure integer)                                    */
 /* ------------------------------------------------------------------------ */
@@ -132,13 +141,14 @@ lg_status_t lg_sparse_attn_fwd_workspace(const lg_pattern_t* pattern, int32_t B,
  * O = softmax_mask(scale * Q K^T) V for every (b, h), and LSE per query row.
  * Abstract, insights 1-2; atlas.scime.ai summary, "Approach" (exact,
  * FlashAttention-style attention under the static mask above).
- * Device pointers: q [B,S,H,D] bf16, k/v [B,S,Hkv,D] bf16, o [B,S,H,D] bf16
- * (written), lse [B,H,S] fp32 (written; may be NULL when not needed).
- * KV blocks outside the pattern are never read.
+ * Device pointers: q [B,S,H,D] bf16, k/v [B,S,Hkv,D] bf16, o [B,S,H,D]
+ * (written) of element type o_dtype (LG_BF16 or LG_F32), lse [B,H,S] fp32
+ * (written; may be NULL when not needed). KV blocks outside the pattern are
+ * never read.
  */
 lg_status_t lg_sparse_attn_fwd(const lg_pattern_t* pattern, const void* q, const void* k, const void* v,
-                               void* o, float* lse, int32_t B, int32_t S, int32_t H, int32_t Hkv, int32_t D,
-                               float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream);
+                               void* o, int32_t o_dtype, float* lse, int32_t B, int32_t S, int32_t H, int32_t Hkv,
+                               int32_t D, float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Training backward                                                        */
@@ -153,15 +163,18 @@ lg_status_t lg_sparse_attn_bwd_workspace(const lg_pattern_t* pattern, int32_t B,
  * the training kernel; "Key results": 1.55x training speedup at 128K):
  *   P = exp(scale Q K^T - LSE) on the mask, Delta = rowsum(dO * O),
  *   dV = P^T dO, dS = P * (dO V^T - Delta), dQ = scale dS K, dK = scale dS^T Q.
- * Device pointers: q, k, v, o, dout, lse as produced/consumed by the forward;
- * dq [B,S,H,D], dk/dv [B,S,Hkv,D] bf16 (written; dk/dv sum over the query
- * heads of a KV group). workspace (device, 256-byte aligned) of at least the
- * queried size; its contents on entry do not matter.
+ * Device pointers: q, k, v, dout bf16; o as written by the forward, of
+ * element type o_dtype; lse as written by the forward; dq [B,S,H,D], dk/dv
+ * [B,S,Hkv,D] (written; dk/dv sum over the query heads of a KV group) of
+ * element type grad_dtype. P enters the dV product as a bf16 hi + lo pair
+ * (dV is exact to fp32 accumulation); dS enters dK and dQ as bf16.
+ * workspace (device, 256-byte aligned) of at least the queried size; its
+ * contents on entry do not matter.
  */
 lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* pattern, const void* q, const void* k, const void* v,
-                               const void* o, const void* dout, const float* lse, void* dq, void* dk, void* dv,
-                               int32_t B, int32_t S, int32_t H, int32_t Hkv, int32_t D, float scale,
-                               void* workspace, size_t workspace_bytes, lg_stream_t stream);
+                               const void* o, int32_t o_dtype, const void* dout, const float* lse, void* dq,
+                               void* dk, void* dv, int32_t grad_dtype, int32_t B, int32_t S, int32_t H, int32_t Hkv,
+                               int32_t D, float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Decode over the reduced KV cache                                         */

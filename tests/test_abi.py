@@ -100,8 +100,9 @@ def _fwd(**kw):
              B=1, S=1024, H=4, Hkv=4, D=64, scale=0.125)
     a.update(kw)
     p = a["p"]
-    return L.lg_sparse_attn_fwd(None if p is None else ctypes.byref(p), a["q"], a["k"], a["v"], a["o"], a["lse"],
-                                a["B"], a["S"], a["H"], a["Hkv"], a["D"], a["scale"], None, 0, None)
+    return L.lg_sparse_attn_fwd(None if p is None else ctypes.byref(p), a["q"], a["k"], a["v"], a["o"],
+                                a.get("odt", 0), a["lse"], a["B"], a["S"], a["H"], a["Hkv"], a["D"], a["scale"],
+                                None, 0, None)
 
 
 def test_fwd_argument_errors():
@@ -118,15 +119,23 @@ def test_fwd_argument_errors():
     assert _fwd(D=96) == 2
     assert _fwd(q=0x10008) == 2                            # misaligned
     assert _fwd(lse=0x50004) == 2
+    assert _fwd(odt=2) == 1                                # O dtype
 
 
 def test_bwd_and_decode_argument_errors():
     L = lg.lib()
     p = lg._lg_pattern_t(64, 1, 4, 0)
-    ptrs = [0x10000 * (i + 1) for i in range(9)]
-    assert L.lg_sparse_attn_bwd(ctypes.byref(p), *ptrs, 1, 1024, 4, 4, 64, 0.125, None, 0, None) == 3  # workspace
-    assert L.lg_sparse_attn_bwd(ctypes.byref(p), *ptrs, 1, 1024, 4, 4, 128, 0.125, 0x100000, 16, None) == 3
-    assert L.lg_sparse_attn_bwd(ctypes.byref(p), *([None] + ptrs[1:]), 1, 1024, 4, 4, 64, 0.125, None, 0, None) == 1
+    P = [0x10000 * (i + 1) for i in range(9)]
+
+    def bwd(ptrs, odt=0, gdt=0, D=64, ws=None, wsb=0):
+        return L.lg_sparse_attn_bwd(ctypes.byref(p), *ptrs[:4], odt, *ptrs[4:], gdt, 1, 1024, 4, 4, D, 0.125, ws,
+                                    wsb, None)
+
+    assert bwd(P) == 3                                  # workspace missing
+    assert bwd(P, D=128, ws=0x100000, wsb=16) == 3      # workspace too small
+    assert bwd([None] + P[1:]) == 1
+    assert bwd(P, gdt=2) == 1                           # gradient dtype
+    assert bwd(P, odt=5) == 1                           # O dtype
     args = [0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0x60000]
     assert L.lg_sparse_decode(*args, 32, 32, 32, 96, 4160, 0, 0.1, None, 0, None) == 2   # D
     assert L.lg_sparse_decode(*args, 32, 24, 8, 128, 4160, 0, 0.1, None, 0, None) == 2   # G = 3

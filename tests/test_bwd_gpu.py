@@ -1,0 +1,109 @@
+"""Backward parity: the tcgen05 backward (preprocess, main, dQ convert) through
+the C-ABI vs the fp64 oracle's analytic gradients.
+
+O and LSE come from the library's own forward (they are inputs of the
+backward); the oracle computes its gradients from Q, K, V and dO alone.
+Parity is checked on the fp32 gradient outputs (the accumulators before any
+output rounding), at max |err| <= 1e-2 and mean |err| <= 1e-3; the bf16
+outputs are checked to be those fp32 values rounded to nearest even (within
+one bf16 ulp, since the order of the dQ reduce-adds varies between runs).
+The benchmark workloads (1K attention-sink, 128K sink+window) run the
+training configuration: bf16 O from the forward. The other shapes take the
+forward's fp32 O, which makes Delta = rowsum(dO * O) exact to fp32: with a
+bf16 O, Delta alone carries ~1e-3 relative error, which reaches the 1e-2
+bound on dQ / dK for shapes with large gradients (GQA groups).
+Small shapes are compared in full; the 128K sink+window training workload on
+sampled query blocks (dQ) and KV blocks (dK, dV -- the sink block gathers
+every query of the sequence).
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import attention_sink_long_b200 as lg
+import synthetic_inputs as si
+from parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+def run_fwd_bwd(pattern, q, k, v, do, scale, grad_dtype=torch.float32, o_dtype=torch.bfloat16):
+    B, S, H, D = q.shape
+    Hkv = k.shape[2]
+    o = torch.empty(q.shape, dtype=o_dtype, device=q.device)
+    lse = torch.empty(B, H, S, dtype=torch.float32, device=q.device)
+    lg.lg_sparse_attn_fwd(pattern, q, k, v, o, lse, scale)
+    dq = torch.empty(q.shape, dtype=grad_dtype, device=q.device)
+    dk = torch.empty(k.shape, dtype=grad_dtype, device=q.device)
+    dv = torch.empty(v.shape, dtype=grad_dtype, device=q.device)
+    ws = torch.empty(lg.lg_sparse_attn_bwd_workspace(pattern, B, S, H, Hkv, D), dtype=torch.uint8, device=q.device)
+    ws.fill_(0xFF)  # poisoned: the backward must not depend on the workspace contents
+    lg.lg_sparse_attn_bwd(pattern, q, k, v, o, do, lse, dq, dk, dv, scale, ws)
+    torch.cuda.synchronize()
+    assert lg.lg_device_status(q.device.index or 0) == 0
+    return dq, dk, dv
+
+
+def assert_bf16_rounding_of(name, got_bf16, ref_f32):
+    """got_bf16 equals ref_f32 rounded to bf16, within one bf16 ulp."""
+    r = ref_f32.to(torch.bfloat16).float()
+    g = got_bf16.float()
+    ulp = torch.where(r == 0, torch.full_like(r, 2.0 ** -133), torch.abs(r) * 2.0 ** -7)
+    bad = (torch.abs(g - r) > ulp * 1.0001).sum().item()
+    assert bad == 0, (name, bad)
+
+
+SMALL = [
+    # B, S, H, Hkv, D, pattern, O dtype
+    (1, 1024, 4, 4, 64, lg.Pattern(64, 1, 4, 0), torch.bfloat16),   # the 1K attention-sink workload
+    (1, 1024, 4, 4, 64, lg.Pattern(64, 1, 4, 0), torch.float32),
+    (1, 192, 2, 2, 128, lg.Pattern(64, 1, 1, 0), torch.float32),    # ragged 64-row tail KV tile
+    (2, 384, 4, 2, 128, lg.Pattern(64, 0, 2, 3), torch.float32),    # GQA, strided, no sink
+    (1, 512, 2, 2, 64, lg.Pattern.full(64), torch.float32),         # dense causal
+    (1, 640, 4, 1, 128, lg.Pattern(64, 2, 3, 0), torch.float32),    # 4 query heads per KV head
+    (1, 64, 1, 1, 128, lg.Pattern(64, 1, 1, 0), torch.float32),     # a single block
+    (1, 2048, 2, 2, 128, lg.Pattern(64, 1, 16, 4), torch.float32),
+    (1, 1280, 2, 2, 128, lg.Pattern(64, 0, 1, 0), torch.float32),   # diagonal only
+]
+
+
+@pytest.mark.parametrize("B,S,H,Hkv,D,pat,odt", SMALL)
+def test_bwd_matches_oracle_small(B, S, H, Hkv, D, pat, odt):
+    q, k, v, do = si.prefill_inputs(B, S, H, Hkv, D, with_dout=True)
+    scale = 1.0 / math.sqrt(D)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    dq, dk, dv = run_fwd_bwd(pat, qd, kd, vd, dod, scale, o_dtype=odt)
+    rdq, rdk, rdv, _ = oracle.attention_backward(q, k, v, do, oracle.Pattern(*pat), scale)
+    assert_close("dQ", dq.cpu().numpy(), rdq)
+    assert_close("dK", dk.cpu().numpy(), rdk)
+    assert_close("dV", dv.cpu().numpy(), rdv)
+    bq, bk, bv = run_fwd_bwd(pat, qd, kd, vd, dod, scale, torch.bfloat16, o_dtype=odt)
+    assert_bf16_rounding_of("dQ", bq, dq)
+    assert_bf16_rounding_of("dK", bk, dk)
+    assert_bf16_rounding_of("dV", bv, dv)
+
+
+def test_bwd_128k_sink_window_sampled():
+    B, S, H, D = 1, 131072, 32, 128
+    pat = lg.Pattern(64, 1, 64, 0)
+    op = oracle.Pattern(*pat)
+    dev = torch.device("cuda")
+    q, k, v, do = si.prefill_inputs_device(B, S, H, H, D, dev, with_dout=True)
+    scale = 1.0 / math.sqrt(D)
+    dq, dk, dv = run_fwd_bwd(pat, q, k, v, do, scale)
+    nqb = S // 64
+    rng = np.random.default_rng(7)
+    qblocks = sorted({0, 1, nqb - 2, nqb - 1, *rng.choice(np.arange(2, nqb - 2), 6, replace=False).tolist()})
+    qrows = np.concatenate([np.arange(i * 64, i * 64 + 64) for i in qblocks])
+    for h, kvblocks in ((0, [0, 1, nqb // 2, nqb - 1]), (H - 1, [1, nqb // 2, nqb - 1])):
+        qh, kh, vh, doh = (t[0, :, h].float().cpu().numpy() for t in (q, k, v, do))
+        rdq, _ = oracle.attention_backward_rows(qh, kh, vh, doh, qrows, op, scale)
+        assert_close(f"dQ h{h}", dq[0, qrows, h].cpu().numpy(), rdq)
+        krows = np.concatenate([np.arange(j * 64, j * 64 + 64) for j in kvblocks])
+        rdk, rdv = oracle.attention_backward_kv_rows(qh, kh, vh, doh, krows, op, scale, chunk=256)
+        assert_close(f"dK h{h}", dk[0, krows, h].cpu().numpy(), rdk)
+        assert_close(f"dV h{h}", dv[0, krows, h].cpu().numpy(), rdv)

@@ -20,9 +20,9 @@ from parity import assert_close, assert_lse
 pytestmark = pytest.mark.gpu
 
 
-def run_fwd(pattern, q, k, v, scale):
+def run_fwd(pattern, q, k, v, scale, o_dtype=torch.bfloat16):
     B, S, H, D = q.shape
-    o = torch.empty_like(q)
+    o = torch.empty(q.shape, dtype=o_dtype, device=q.device)
     lse = torch.empty(B, H, S, dtype=torch.float32, device=q.device)
     lg.lg_sparse_attn_fwd(pattern, q, k, v, o, lse, scale)
     torch.cuda.synchronize()
@@ -48,10 +48,16 @@ SMALL = [
 def test_fwd_matches_oracle_small(B, S, H, Hkv, D, pat):
     q, k, v = si.prefill_inputs(B, S, H, Hkv, D)
     scale = 1.0 / math.sqrt(D)
-    o, lse = run_fwd(pat, q.cuda(), k.cuda(), v.cuda(), scale)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o, lse = run_fwd(pat, qd, kd, vd, scale)
     ro, rlse = oracle.attention_forward(q, k, v, oracle.Pattern(*pat), scale)
     assert_close("O", o.float().cpu().numpy(), ro)
     assert_lse("LSE", lse.cpu().numpy(), rlse)
+    # fp32 output: the same accumulators without the bf16 rounding.
+    o32, lse32 = run_fwd(pat, qd, kd, vd, scale, torch.float32)
+    assert_close("O fp32", o32.cpu().numpy(), ro)
+    assert torch.equal(lse32, lse)
+    assert torch.equal(o32.to(torch.bfloat16), o)
 
 
 def test_fwd_repeatable():
