@@ -240,7 +240,7 @@ lg_status_t lg_sparse_attn_fwd(const lg_pattern_t* p, const void* q, const void*
   prm.H = H;
   prm.Hkv = Hkv;
   prm.nqb = S / 64;
-  prm.nqt = (S + 127) / 128;
+  prm.nqt = (S + 255) / 256;  // 256-row query spans (two 128-row tiles per CTA)
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.err = err;
   return cuda_status(lg::launch_fwd(D, tq, tk, tv, to, prm, B, static_cast<cudaStream_t>(stream)));

@@ -15,7 +15,7 @@ struct FwdParams {
   float* o_f32;  // [B, S, H, D] fp32 output, or nullptr for the bf16 TMA-stored output
   int S, H, Hkv;
   int nqb;  // S / 64
-  int nqt;  // ceil(S / 128)
+  int nqt;  // ceil(S / 256): CTAs along the sequence
   float scale_log2;  // scale * log2(e)
   unsigned int* err;
 };
