@@ -8,21 +8,27 @@
 // blocks, computes S = Q K^T and O += P V on the tcgen05 tensor cores with the
 // accumulators in TMEM, and keeps an online softmax per row.
 //
-// CTA = 10 warps, two 128-row query tiles that share every K/V block:
+// KV blocks are consumed in chunks of one block, or two adjacent listed blocks
+// (KvChunks), so most MMAs run with N = 128 (S) and K = 128 (PV).
+//
+// CTA = 10 warps, two 128-row query tiles that share every K/V chunk:
 //   warps 0-3 / 4-7  softmax + epilogue of tile 0 / tile 1; thread r of a group
 //                    owns row r of its tile, which is TMEM lane r (a warp may
 //                    only touch its own 32-lane quarter);
-//   warp 8           TMA producer (both Q tiles once, then K/V blocks through a
-//                    ring of stages);
+//   warp 8           TMA producer (both Q tiles once, then K/V chunks through a
+//                    two-stage ring);
 //   warp 9           TMEM allocation and the single MMA-issuing thread.
-// TMEM columns: O of tile t at [t*D, (t+1)*D); S of tile t, buffer sb at
-// 2D + 128t + 64sb (64 columns each).
-// Shared memory (128B-swizzled, as TMA writes it): Q tiles [128 x D], K/V
-// stages [64 x D], P double buffer per tile [128 x 64] bf16.
-// Per KV block the MMA thread issues, per tile, QK(n+1) before PV(n) so the
-// tensor core works on the next block while that tile's softmax finishes the
-// current one; the two tiles interleave. O is rescaled lazily, only when a
-// row's running max grows by more than 2^8.
+// TMEM columns: O of tile t at [t*D, (t+1)*D); S of tile t at 2D + 128t
+// (128 columns). The softmax writes P back over the first 64 columns of its S
+// (bf16, two per column) and the PV product reads it from there (A operand in
+// TMEM), so P never touches shared memory.
+// The MMA thread ping-pongs the tiles: PV_0(c), S_0(c+1), PV_1(c), S_1(c+1) --
+// the tensor core runs one tile's GEMMs while the other tile's softmax works.
+// Issue order also protects the P/S aliasing: S_t(c+1) is issued after
+// PV_t(c), and tcgen05 MMAs of one thread execute in order. When a tile's
+// softmax sees S_t(c) complete, PV_t(c-1) is complete too (same commit), so O
+// can be rescaled right away. O is rescaled lazily, only when a row's running
+// max grows by more than 2^8.
 #include "lg_common.cuh"
 #include "lg_kernels.h"
 #include "lg_pattern.cuh"
@@ -31,18 +37,16 @@ namespace lg {
 
 template <int D>
 struct FwdLayout {
-  static constexpr int DP = D / 64;               // 64-element (128-byte) panels per row
-  static constexpr int NT = 2;                    // 128-row query tiles per CTA
-  static constexpr int NS = (D == 128) ? 3 : 4;   // K/V ring depth
-  static constexpr int Q_BYTES = 128 * D * 2;     // one query tile
-  static constexpr int KV_BYTES = 64 * D * 2;     // one K or V block
-  static constexpr int P_BYTES = 128 * 64 * 2;
-  static constexpr int OFF_Q = 0;                 // NT tiles
+  static constexpr int DP = D / 64;              // 64-element (128-byte) panels per row
+  static constexpr int NT = 2;                   // 128-row query tiles per CTA
+  static constexpr int NS = 2;                   // K/V chunk stages
+  static constexpr int Q_BYTES = 128 * D * 2;    // one query tile
+  static constexpr int KVC_BYTES = 128 * D * 2;  // one K or V chunk (up to 128 rows)
+  static constexpr int OFF_Q = 0;                // NT tiles
   static constexpr int OFF_K = OFF_Q + NT * Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + NS * KV_BYTES;  // NT tiles x 2 buffers
-  static constexpr int OFF_BAR = OFF_P + NT * 2 * P_BYTES;
-  static constexpr int NBAR = 1 + 4 * NS + NT * 8;
+  static constexpr int OFF_V = OFF_K + NS * KVC_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NS * KVC_BYTES;
+  static constexpr int NBAR = 1 + 3 * NS + NT * 3;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;  // room to align the base to 1024 bytes
@@ -65,10 +69,9 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = bars + 1 + NS;
-  uint64_t* v_full = bars + 1 + 2 * NS;
-  uint64_t* v_empty = bars + 1 + 3 * NS;
-  uint64_t* tile_bars = bars + 1 + 4 * NS;  // per tile: s_full[2], s_empty[2], p_full[2], pv_done[2]
+  uint64_t* v_full = bars + 1 + NS;
+  uint64_t* kv_empty = bars + 1 + 2 * NS;
+  uint64_t* tile_bars = bars + 1 + 3 * NS;  // per tile: s_full, p_full, pv_done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -78,28 +81,20 @@ __global__ void __launch_bounds__(320, 1)
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const int kvh = h / (prm.H / prm.Hkv);
-  const int i_lo = 4 * span;
-  const int i_hi = imin(4 * span + 3, prm.nqb - 1);
-  const KvIter it(prm.pat, i_lo, i_hi);
-  const int N = it.count();
+  const KvChunks chunks(prm.pat, 4 * span, imin(4 * span + 3, prm.nqb - 1));
   unsigned int* err = prm.err;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], 1);
+      mbar_init(&kv_empty[s], 1);
     }
     for (int t = 0; t < NT; ++t) {
-      uint64_t* tb = tile_bars + 8 * t;
-      for (int s = 0; s < 2; ++s) {
-        mbar_init(&tb[0 + s], 1);    // s_full
-        mbar_init(&tb[2 + s], 128);  // s_empty
-        mbar_init(&tb[4 + s], 128);  // p_full
-        mbar_init(&tb[6 + s], 1);    // pv_done
-      }
+      mbar_init(&tile_bars[3 * t + 0], 1);    // s_full
+      mbar_init(&tile_bars[3 * t + 1], 128);  // p_full
+      mbar_init(&tile_bars[3 * t + 2], 1);    // pv_done
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -127,23 +122,29 @@ __global__ void __launch_bounds__(320, 1)
         for (int p = 0; p < L::DP; ++p)
           tma_load_4d(smem + L::OFF_Q + t * L::Q_BYTES + p * 16384, &tmQ, q_full, 64 * p, h, 256 * span + 128 * t,
                       b);
-      int n = 0;
-      for (int j = it.first(); j >= 0; j = it.next(j), ++n) {
-        const int st = n % NS;
-        const uint32_t use = (uint32_t)(n / NS);
-        if (use > 0 && !mbar_wait(&k_empty[st], (use - 1) & 1, abort_flag, err, kErrFwdWait)) break;
-        mbar_arrive_expect_tx(&k_full[st], L::KV_BYTES);
-        for (int p = 0; p < L::DP; ++p)
-          tma_load_4d(smem + L::OFF_K + st * L::KV_BYTES + p * 8192, &tmK, &k_full[st], 64 * p, kvh, 64 * j, b);
-        if (use > 0 && !mbar_wait(&v_empty[st], (use - 1) & 1, abort_flag, err, kErrFwdWait)) break;
-        mbar_arrive_expect_tx(&v_full[st], L::KV_BYTES);
-        for (int p = 0; p < L::DP; ++p)
-          tma_load_4d(smem + L::OFF_V + st * L::KV_BYTES + p * 8192, &tmV, &v_full[st], 64 * p, kvh, 64 * j, b);
+      int c = 0;
+      int nb = 1;
+      for (int j = chunks.first(); j >= 0; ++c) {
+        const int jn = chunks.span(j, &nb);
+        const int st = c % NS;
+        const uint32_t use = (uint32_t)(c / NS);
+        if (use > 0 && !mbar_wait(&kv_empty[st], (use - 1) & 1, abort_flag, err, kErrFwdWait)) break;
+        mbar_arrive_expect_tx(&k_full[st], nb * 64 * D * 2);
+        for (int hb = 0; hb < nb; ++hb)
+          for (int p = 0; p < L::DP; ++p)
+            tma_load_4d(smem + L::OFF_K + st * L::KVC_BYTES + p * 16384 + hb * 8192, &tmK, &k_full[st], 64 * p, kvh,
+                        64 * (j + hb), b);
+        mbar_arrive_expect_tx(&v_full[st], nb * 64 * D * 2);
+        for (int hb = 0; hb < nb; ++hb)
+          for (int p = 0; p < L::DP; ++p)
+            tma_load_4d(smem + L::OFF_V + st * L::KVC_BYTES + p * 16384 + hb * 8192, &tmV, &v_full[st], 64 * p, kvh,
+                        64 * (j + hb), b);
+        j = jn;
       }
       if (*abort_flag) {
         // Let copies already in flight land before the CTA's shared memory goes away.
-        for (int s = 0; s < NS && s < n; ++s) {
-          const int last = n - 1 - ((n - 1 - s) % NS);
+        for (int s = 0; s < NS && s < c; ++s) {
+          const int last = c - 1 - ((c - 1 - s) % NS);
           const uint32_t u = (uint32_t)(last / NS);
           const long long t0 = clock64();
           while (!(mbar_try_wait(&k_full[s], u & 1) && mbar_try_wait(&v_full[s], u & 1)) &&
@@ -155,104 +156,104 @@ __global__ void __launch_bounds__(320, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16(128, 64, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
       bool ok = mbar_wait(q_full, 0, abort_flag, err, kErrFwdWait);
       tc_fence_after();
-      // S_t(n) = Q_t K(n)^T into the tile's S buffer n % 2.
-      auto issue_qk = [&](int n, int t) -> bool {
-        const int st = n % NS;
-        const int sb = n & 1;
-        const uint32_t su = (uint32_t)(n >> 1);
-        uint64_t* tb = tile_bars + 8 * t;
-        if (!mbar_wait(&k_full[st], (uint32_t)(n / NS) & 1, abort_flag, err, kErrFwdWait)) return false;
-        if (n >= 2 && !mbar_wait(&tb[2 + sb], (su - 1) & 1, abort_flag, err, kErrFwdWait)) return false;
+      // S_t(c) = Q_t K(c)^T, N = 64 * nb, into the tile's S columns.
+      auto issue_s = [&](int c, int nb, int t) -> bool {
+        const int st = c % NS;
+        if (t == 0 && !mbar_wait(&k_full[st], (uint32_t)(c / NS) & 1, abort_flag, err, kErrFwdWait)) return false;
         tc_fence_after();
-        const uint32_t d_tmem = tmem + L::T_S + (uint32_t)(128 * t + 64 * sb);
+        const uint32_t idesc = idesc_bf16(128, 64 * nb, false, false);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t a = sbase + L::OFF_Q + t * L::Q_BYTES + (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t bb = sbase + L::OFF_K + st * L::KV_BYTES + (kk >> 2) * 8192 + (kk & 3) * 32;
-          tc_mma_ss(d_tmem, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          const uint32_t bb = sbase + L::OFF_K + st * L::KVC_BYTES + (kk >> 2) * 16384 + (kk & 3) * 32;
+          tc_mma_ss(tmem + L::T_S + 128 * t, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 16, 1024), idesc,
+                    kk > 0 ? 1u : 0u);
         }
-        tc_commit(&tb[0 + sb]);
+        tc_commit(&tile_bars[3 * t + 0]);
         return true;
       };
-      // O_t += P_t(n) V(n).
-      auto issue_pv = [&](int n, int t) -> bool {
-        const int st = n % NS;
-        const int sb = n & 1;
-        uint64_t* tb = tile_bars + 8 * t;
-        if (!mbar_wait(&tb[4 + sb], (uint32_t)(n >> 1) & 1, abort_flag, err, kErrFwdWait)) return false;
-        if (!mbar_wait(&v_full[st], (uint32_t)(n / NS) & 1, abort_flag, err, kErrFwdWait)) return false;
+      // O_t += P_t(c) V(c), K = 64 * nb, P from TMEM.
+      auto issue_pv = [&](int c, int nb, int t) -> bool {
+        const int st = c % NS;
+        if (!mbar_wait(&tile_bars[3 * t + 1], (uint32_t)c & 1, abort_flag, err, kErrFwdWait)) return false;
+        if (t == 0 && !mbar_wait(&v_full[st], (uint32_t)(c / NS) & 1, abort_flag, err, kErrFwdWait)) return false;
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint32_t a = sbase + L::OFF_P + (2 * t + sb) * L::P_BYTES + kk * 32;
-          const uint32_t bb = sbase + L::OFF_V + st * L::KV_BYTES + kk * 2048;
-          tc_mma_ss(tmem + (uint32_t)(t * D), sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 8192, 1024), idesc_pv,
-                    (n > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 4 * nb; ++kk) {
+          const uint32_t bb = sbase + L::OFF_V + st * L::KVC_BYTES + kk * 2048;
+          tc_mma_ts(tmem + (uint32_t)(t * D), tmem + L::T_S + 128 * t + 8 * kk, sdesc_sw128(bb, 16384, 1024),
+                    idesc_pv, (c > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(&tb[6 + sb]);
+        tc_commit(&tile_bars[3 * t + 2]);
         return true;
       };
-      for (int t = 0; t < NT && ok; ++t) ok = issue_qk(0, t);
-      if (ok && N > 0) tc_commit(&k_empty[0]);
-      for (int n = 0; n < N && ok; ++n) {
+      int nb = 1;
+      int j = chunks.first();
+      int jn = j >= 0 ? chunks.span(j, &nb) : -1;
+      for (int t = 0; t < NT && ok && j >= 0; ++t) ok = issue_s(0, nb, t);
+      for (int c = 0; j >= 0 && ok; ++c) {
+        int nb_next = 1;
+        const int jnn = jn >= 0 ? chunks.span(jn, &nb_next) : -1;
         for (int t = 0; t < NT && ok; ++t) {
-          if (n + 1 < N) ok = issue_qk(n + 1, t);
-          if (ok) ok = issue_pv(n, t);
+          ok = issue_pv(c, nb, t);
+          if (ok && jn >= 0) ok = issue_s(c + 1, nb_next, t);
         }
         if (!ok) break;
-        if (n + 1 < N) tc_commit(&k_empty[(n + 1) % NS]);
-        tc_commit(&v_empty[n % NS]);
+        tc_commit(&kv_empty[c % NS]);
+        j = jn;
+        jn = jnn;
+        nb = nb_next;
       }
     }
   } else {
     // ------------------------------------------------------------ softmax warps 0-7
-    const int t = warp >> 2;                 // query tile of this warp group
-    const int r = threadIdx.x & 127;         // tile row == TMEM lane
+    const int t = warp >> 2;          // query tile of this warp group
+    const int r = threadIdx.x & 127;  // tile row == TMEM lane
     const int i = 4 * span + 2 * t + (r >> 6);
     const int rr = r & 63;
     const bool row_live = i < prm.nqb;
-    uint64_t* tb = tile_bars + 8 * t;
+    uint64_t* s_full = &tile_bars[3 * t + 0];
+    uint64_t* p_full = &tile_bars[3 * t + 1];
+    uint64_t* pv_done = &tile_bars[3 * t + 2];
     const uint32_t t_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t t_o = t_lane + (uint32_t)(t * D);
     const uint32_t t_s = t_lane + L::T_S + (uint32_t)(128 * t);
     const float sl2 = prm.scale_log2;
     float m = -INFINITY;  // running max in log2 units of the scaled scores
     float l = 0.f;
-    int n = 0;
-    for (int j = it.first(); j >= 0; j = it.next(j), ++n) {
-      const int sb = n & 1;
-      const uint32_t su = (uint32_t)(n >> 1);
-      if (!__all_sync(0xffffffffu, mbar_wait(&tb[0 + sb], su & 1, abort_flag, err, kErrFwdWait))) break;
+    int c = 0;
+    int nb = 1;
+    for (int j = chunks.first(); j >= 0; ++c) {
+      const int jn = chunks.span(j, &nb);
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full, (uint32_t)c & 1, abort_flag, err, kErrFwdWait))) break;
       tc_fence_after();
-      uint32_t sr[64];
-      tmem_ld64(t_s + (uint32_t)(64 * sb), sr);
-      tc_fence_before();
-      mbar_arrive(&tb[2 + sb]);
-
-      float x[64];
+      // Pass 1: row max over the chunk, 64 columns at a time straight from TMEM,
+      // masked per 64-column half (blocks outside this row's list, causality
+      // inside the diagonal block). Pass 2 reloads the columns for the
+      // exponentials, which keeps only 64 row values in registers.
+      bool vis[2], diag[2];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(sr[c]);
-      const bool vis = row_live && in_list(prm.pat, i, j);
-      if (!vis) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) x[c] = -INFINITY;
-      } else if (j == i) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c > rr) x[c] = -INFINITY;
+      for (int hb = 0; hb < 2; ++hb) {
+        vis[hb] = hb < nb && row_live && in_list(prm.pat, i, j + hb);
+        diag[hb] = (j + hb == i);
       }
-      // Row max as a tree (short dependency chains keep the pipes busy).
       float mx8[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(x[e], x[e + 8]);
+      for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
 #pragma unroll
-      for (int c = 16; c < 64; c += 8)
+      for (int hb = 0; hb < 2; ++hb) {
+        if (vis[hb]) {
+          uint32_t xs[64];
+          tmem_ld64(t_s + 64 * hb, xs);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], x[c + e]);
+          for (int e = 0; e < 64; ++e) {
+            const float v = (diag[hb] && e > rr) ? -INFINITY : __uint_as_float(xs[e]);
+            mx8[e & 7] = fmaxf(mx8[e & 7], v);
+          }
+        }
+      }
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_blk = mx * sl2;
@@ -263,36 +264,40 @@ __global__ void __launch_bounds__(320, 1)
         m = m_blk;
       }
       const float m_use = (m == -INFINITY) ? 0.f : m;
-      uint32_t pk[32];
       float rs8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) rs8[e] = 0.f;
+      // Pass 2: P = 2^(x * scale * log2 e - m), packed to bf16 and written back
+      // over the first half of this tile's S columns.
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        const float p0 = ex2_approx(fmaf(x[c], sl2, -m_use));
-        const float p1 = ex2_approx(fmaf(x[c + 1], sl2, -m_use));
-        rs8[(c >> 1) & 7] += p0 + p1;
-        pk[c >> 1] = pack_bf16x2(p0, p1);
+      for (int hb = 0; hb < 2; ++hb) {
+        if (hb < nb) {
+          uint32_t pk[32];
+          if (vis[hb]) {
+            uint32_t xs[64];
+            tmem_ld64(t_s + 64 * hb, xs);
+#pragma unroll
+            for (int e = 0; e < 64; e += 2) {
+              const float x0 = (diag[hb] && e > rr) ? -INFINITY : __uint_as_float(xs[e]);
+              const float x1 = (diag[hb] && e + 1 > rr) ? -INFINITY : __uint_as_float(xs[e + 1]);
+              const float p0 = ex2_approx(fmaf(x0, sl2, -m_use));
+              const float p1 = ex2_approx(fmaf(x1, sl2, -m_use));
+              rs8[(e >> 1) & 7] += p0 + p1;
+              pk[e >> 1] = pack_bf16x2(p0, p1);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) pk[e] = 0u;
+          }
+          tmem_st32(t_s + 32 * hb, pk);
+        }
       }
       const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       l = l * alpha + rs;
 
-      // P buffer sb is free once PV(n-2) of this tile has completed.
-      if (n >= 2 &&
-          !__all_sync(0xffffffffu, mbar_wait(&tb[6 + sb], (su - 1) & 1, abort_flag, err, kErrFwdWait)))
-        break;
-      const uint32_t prow = sbase + L::OFF_P + (2 * t + sb) * L::P_BYTES;
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        st_shared_v4(prow + sw128_offset(r, c), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      fence_async_smem();
-
-      // Lazy rescale of O (warp-uniform because tcgen05.ld/st are warp-collective).
-      if (__any_sync(0xffffffffu, need && n > 0)) {
-        const int pb = (n - 1) & 1;
-        const uint32_t pu = (uint32_t)((n - 1) >> 1);
-        if (!__all_sync(0xffffffffu, mbar_wait(&tb[6 + pb], pu & 1, abort_flag, err, kErrFwdWait))) break;
-        tc_fence_after();
+      // Lazy rescale of O (warp-uniform: tcgen05.ld/st are warp-collective).
+      // PV_t(c-1) completed before S_t(c) did, so O is stable here.
+      if (__any_sync(0xffffffffu, need && c > 0)) {
 #pragma unroll
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t o[32];
@@ -303,16 +308,14 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&tb[4 + sb]);
+      mbar_arrive(p_full);
+      j = jn;
     }
+    const int NC = c;
 
     // ------------------------------------------------------------ epilogue
-    bool ok = (n == N) && !*abort_flag;
-    if (ok) {
-      const int lb = (N - 1) & 1;
-      const uint32_t lu = (uint32_t)((N - 1) >> 1);
-      ok = mbar_wait(&tb[6 + lb], lu & 1, abort_flag, err, kErrFwdWait);
-    }
+    bool ok = !*abort_flag && NC > 0;
+    if (ok) ok = mbar_wait(pv_done, (uint32_t)(NC - 1) & 1, abort_flag, err, kErrFwdWait);
     ok = __all_sync(0xffffffffu, ok);
     const int row0 = 256 * span + 128 * t;  // first sequence row of this tile
     const int srow = row0 + r;

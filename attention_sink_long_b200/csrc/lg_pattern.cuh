@@ -67,6 +67,25 @@ struct KvIter {
   }
 };
 
+// The KvIter sequence grouped into chunks of one listed block, or two when the
+// next listed block is adjacent (window and sink runs pair up, isolated strided
+// blocks stay single). span(j, &nb) takes a chunk start j, sets nb to its
+// block count and returns the next chunk start (or -1).
+struct KvChunks {
+  KvIter it;
+  LG_HD KvChunks(const lg_pattern_t& p, int i_lo, int i_hi) : it(p, i_lo, i_hi) {}
+  LG_HD int first() const { return it.first(); }
+  LG_HD int span(int j, int* nb) const {
+    const int j2 = it.next(j);
+    if (j2 == j + 1) {
+      *nb = 2;
+      return it.next(j2);
+    }
+    *nb = 1;
+    return j2;
+  }
+};
+
 // Union of the query-block lists (transpose) of the consecutive KV blocks
 // [j_lo, j_hi], given nqb query blocks. A sink or strided KV block is seen by
 // every later query block; any other by the local_blocks query blocks starting
