@@ -28,14 +28,15 @@ __all__ = [
     "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd",
     "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd",
     "lg_sparse_decode_splits", "lg_sparse_decode_workspace", "lg_sparse_decode",
-    "lg_sparse_decode_noalloc", "lg_device_status", "EXPORTED_SYMBOLS",
+    "lg_sparse_decode_noalloc", "lg_exp2_device", "lg_device_status", "EXPORTED_SYMBOLS",
 ]
 
 EXPORTED_SYMBOLS = (
     "lg_strerror", "lg_version", "lg_pattern_expand", "lg_pattern_expand_t", "lg_pattern_pairs",
     "lg_pattern_iterate_device", "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd",
     "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd", "lg_sparse_decode_splits",
-    "lg_sparse_decode_workspace", "lg_sparse_decode", "lg_sparse_decode_noalloc", "lg_device_status",
+    "lg_sparse_decode_workspace", "lg_sparse_decode", "lg_sparse_decode_noalloc", "lg_exp2_device",
+    "lg_device_status",
 )
 
 
@@ -82,6 +83,7 @@ _SIGS = {
     "lg_sparse_decode_workspace": (_c_i32, [_c_i32] * 6 + [_P(_c_sz)]),
     "lg_sparse_decode": (_c_i32, [_c_vp] * 6 + [_c_i32] * 6 + [_c_f, _c_vp, _c_sz, _c_vp]),
     "lg_sparse_decode_noalloc": (_c_i32, [_c_vp] * 6 + [_c_i32] * 6 + [_c_f, _c_vp]),
+    "lg_exp2_device": (_c_i32, [_c_vp, _c_vp, _c_i64, _c_i32, _c_vp]),
     "lg_device_status": (_c_i32, [_c_i32, _P(ctypes.c_uint32)]),
 }
 
@@ -323,6 +325,17 @@ def lg_sparse_decode_noalloc(q, k_cache, v_cache, cache_lens, o, lse, scale: flo
                                           cache_lens.data_ptr(), o.data_ptr(), _ptr(lse), B, H, Hkv, D, Lmax,
                                           int(num_splits), float(scale), _stream(stream)),
            "lg_sparse_decode_noalloc")
+
+
+# ---------------------------------------------------------------- numerics
+def lg_exp2_device(x, y, method: int, stream=None):
+    """y = 2^x on the device with the softmax's exponential (0: ex2.approx, 1: polynomial)."""
+    import torch
+
+    _expect(x, "x", torch.float32, tuple(x.shape))
+    _expect(y, "y", torch.float32, tuple(x.shape), x.device)
+    _check(lib().lg_exp2_device(x.data_ptr(), y.data_ptr(), x.numel(), int(method), _stream(stream)),
+           "lg_exp2_device")
 
 
 # ---------------------------------------------------------------- diagnostics

@@ -244,13 +244,15 @@ __global__ void __launch_bounds__(320, 1)
       for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
 #pragma unroll
       for (int hb = 0; hb < 2; ++hb) {
-        if (vis[hb]) {
+        if (vis[hb]) {  // vis and diag are warp-uniform (a warp's rows share a query block)
           uint32_t xs[64];
           tmem_ld64(t_s + 64 * hb, xs);
+          if (diag[hb]) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e) {
-            const float v = (diag[hb] && e > rr) ? -INFINITY : __uint_as_float(xs[e]);
-            mx8[e & 7] = fmaxf(mx8[e & 7], v);
+            for (int e = 0; e < 64; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], e > rr ? -INFINITY : __uint_as_float(xs[e]));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 64; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(xs[e]));
           }
         }
       }
@@ -268,7 +270,9 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
       for (int e = 0; e < 8; ++e) rs8[e] = 0.f;
       // Pass 2: P = 2^(x * scale * log2 e - m), packed to bf16 and written back
-      // over the first half of this tile's S columns.
+      // over the first half of this tile's S columns. Columns e with
+      // (e & 7) >= 6 -- a quarter -- take the FMA-pipe polynomial, the rest the
+      // special-function unit, so neither pipe alone sets the pace.
 #pragma unroll
       for (int hb = 0; hb < 2; ++hb) {
         if (hb < nb) {
@@ -276,12 +280,16 @@ __global__ void __launch_bounds__(320, 1)
           if (vis[hb]) {
             uint32_t xs[64];
             tmem_ld64(t_s + 64 * hb, xs);
+            if (diag[hb]) {
+#pragma unroll
+              for (int e = 0; e < 64; ++e) xs[e] = e > rr ? 0xff800000u : xs[e];  // -inf above the diagonal
+            }
 #pragma unroll
             for (int e = 0; e < 64; e += 2) {
-              const float x0 = (diag[hb] && e > rr) ? -INFINITY : __uint_as_float(xs[e]);
-              const float x1 = (diag[hb] && e + 1 > rr) ? -INFINITY : __uint_as_float(xs[e + 1]);
-              const float p0 = ex2_approx(fmaf(x0, sl2, -m_use));
-              const float p1 = ex2_approx(fmaf(x1, sl2, -m_use));
+              const float a0 = fmaf(__uint_as_float(xs[e]), sl2, -m_use);
+              const float a1 = fmaf(__uint_as_float(xs[e + 1]), sl2, -m_use);
+              const float p0 = ((e & 7) >= 6) ? ex2_poly(a0) : ex2_approx(a0);
+              const float p1 = ((e & 7) >= 6) ? ex2_poly(a1) : ex2_approx(a1);
               rs8[(e >> 1) & 7] += p0 + p1;
               pk[e >> 1] = pack_bf16x2(p0, p1);
             }

@@ -252,6 +252,27 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe, for the share of the softmax exponentials that is kept
+// off the special-function unit. Cody-Waite additive range reduction x = n + f
+// with n = round(x) (adding and subtracting 1.5 * 2^23 rounds to an integer)
+// and f in [-1/2, 1/2]; 2^f by a degree-4 polynomial, the Remez minimax fit
+// of the relative error on [-1/2, 1/2] made by csrc/exp2_poly_fit.py (max
+// relative error 2.7e-6 over [-126, 64]); 2^n enters through the exponent
+// bits. Exactly 0 for x <= -127 (masked entries arrive as -inf).
+__device__ __forceinline__ float ex2_poly(float x) {
+  const float xc = fmaxf(x, -127.0f);
+  const float y = xc + 12582912.0f;
+  const float n = y - 12582912.0f;
+  const float f = xc - n;
+  float p = 0.009570102207362652f;
+  p = fmaf(p, f, 0.05591785907745361f);
+  p = fmaf(p, f, 0.240247443318367f);
+  p = fmaf(p, f, 0.6931217908859253f);
+  p = fmaf(p, f, 0.9999992847442627f);
+  const float r = __uint_as_float(__float_as_uint(p) + (__float_as_uint(y) << 23));
+  return xc <= -127.0f ? 0.0f : r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
