@@ -138,82 +138,89 @@ cudaError_t launch_bwd_dq(const float* dq_acc, void* dq, int dq_f32, float scale
 // per step. Per step, all on tcgen05 with fp32 accumulation in TMEM:
 //   S^T  = K Q_i^T          (M=128 kv, N=64 q, K=D)
 //   dP^T = V dO_i^T         (M=128,    N=64,   K=D)
-//   dV  += P^T dO_i         (M=128,    N=D,    K=64; P^T as a bf16 hi + lo pair)
-//   dK  += dS^T Q_i         (M=128,    N=D,    K=64)
-//   dQ_i^T = K^T dS^T       (M=D,      N=64,   K=128)
+//   dV  += P^T dO_i         (M=128,    N=D,    K=64; P^T read from TMEM)
+//   dK  += dS^T Q_i         (M=128,    N=D,    K=64; dS^T read from TMEM)
+//   dQ_i^T = K^T dS^T       (M=D,      N=64,   K=128; dS^T from shared memory)
 // with P^T = exp(scale S^T - LSE) on the mask and dS^T = P^T (dP^T - Delta),
-// computed by four warps that each own 32 KV rows (TMEM lanes), written to
-// shared memory as bf16 in the 128B-swizzled K-major layout the MMA reads.
+// computed by four warps that each own 32 KV rows (TMEM lanes). They write
+// bf16 P^T and dS^T back into TMEM over the S^T / dP^T columns they have
+// read (A operands of the dV / dK products), and dS^T also to shared memory
+// (B operand of dQ^T). dQ_i^T lands in the middle 64 columns of the same
+// step's TMEM buffer, which the P^T / dS^T writes leave free; four more warps
+// read it and add it to the fp32 dQ accumulator with coalesced global
+// reductions (a warp's 32 lanes cover 32 consecutive dQ elements of one row).
+// The per-step TMEM buffer (S^T | dP^T) is double-buffered, so S^T / dP^T of
+// step n+1 run while the warps work on step n, and the gradient GEMMs of
+// step n run while they work on step n+1.
 // With GQA (H / Hkv > 1) dV and dK sum over the group's query heads and grow
-// with it, so P^T and dS^T then go in twice, as bf16(x) and the residual
-// bf16(x - bf16(x)): dV and dK then carry no bf16 rounding of P or dS (a
-// single bf16 operand costs ~2^-9 relative per term, which at |dK| ~ 4 is the
-// whole 1e-2 error budget). Without GQA the plain five GEMMs are used.
-// dQ_i^T is read back by a second group of four warps, transposed through
-// shared memory and added to the fp32 dQ accumulator with one bulk
-// reduce-add per step. S/dP of step n+1 are issued before the gradient GEMMs
-// of step n, so the exponentials of one step overlap the GEMMs of the other.
+// with it, so P^T and dS^T then also enter dV / dK as the bf16 residual
+// bf16(x - bf16(x)) from shared memory: dV and dK then carry no bf16 rounding
+// of P or dS (a single bf16 operand costs ~2^-9 relative per term, which at
+// |dK| ~ 4 is the whole 1e-2 error budget). Without GQA the plain five GEMMs
+// are used.
 //
 // Warps: 0-3 P/dS + epilogue, 4 TMA producer, 5 TMEM owner + MMA issuer,
-// 6-9 dQ drain. TMEM columns: dV [0,D), dK [D,2D), S^T [2D,2D+64),
-// dP^T [2D+64,2D+128), dQ^T double buffer [2D+128, 2D+256).
+// 6-9 dQ drain. TMEM columns: dV [0,D), dK [D,2D), step buffer b at
+// 2D + 128b: S^T [0,64) then P^T in [0,32); dP^T [64,128) then dS^T in
+// [96,128); dQ^T in [32,96).
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool SPLIT>
 struct BwdLayout {
-  static constexpr int KV_BYTES = 128 * D * 2;  // K or V tile (128 rows)
-  static constexpr int QB_BYTES = 64 * D * 2;   // Q or dO block (64 rows)
-  static constexpr int PT_BYTES = 128 * 64 * 2;  // P^T or dS^T (bf16)
-  static constexpr int DQS_BYTES = 64 * D * 4;   // dQ staging (fp32, [q][d])
+  static constexpr int QS = 3;                   // Q / dO stages
+  static constexpr int KV_BYTES = 128 * D * 2;   // K or V tile (128 rows)
+  static constexpr int QB_BYTES = 64 * D * 2;    // Q or dO block (64 rows)
+  static constexpr int PT_BYTES = 128 * 64 * 2;  // a [128 x 64] bf16 tile
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KV_BYTES;
-  static constexpr int OFF_Q = OFF_V + KV_BYTES;      // 2 stages
-  static constexpr int OFF_DO = OFF_Q + 2 * QB_BYTES;  // 2 stages
-  static constexpr int OFF_PT = OFF_DO + 2 * QB_BYTES;  // bf16(P^T)
-  static constexpr int OFF_PL = OFF_PT + PT_BYTES;       // bf16(P^T - bf16(P^T))
-  static constexpr int OFF_DST = OFF_PL + PT_BYTES;      // bf16(dS^T)
-  static constexpr int OFF_DSL = OFF_DST + PT_BYTES;     // bf16(dS^T - bf16(dS^T))
-  static constexpr int OFF_DQS = OFF_DSL + PT_BYTES;
-  static constexpr int OFF_LSE = OFF_DQS + DQS_BYTES;  // 2 stages x 64 fp32
-  static constexpr int OFF_DEL = OFF_LSE + 512;        // 2 stages x 64 fp32
-  static constexpr int OFF_BAR = OFF_DEL + 512;
-  static constexpr int NBAR = 16;
+  static constexpr int OFF_Q = OFF_V + KV_BYTES;          // QS stages
+  static constexpr int OFF_DO = OFF_Q + QS * QB_BYTES;    // QS stages
+  static constexpr int OFF_DST = OFF_DO + QS * QB_BYTES;  // bf16(dS^T), 2 buffers
+  static constexpr int OFF_PL = OFF_DST + 2 * PT_BYTES;   // GQA: bf16(P^T - bf16(P^T))
+  static constexpr int OFF_DSL = OFF_PL + PT_BYTES;       // GQA: bf16(dS^T - bf16(dS^T))
+  static constexpr int OFF_LSE = OFF_DSL + (SPLIT ? PT_BYTES : 0) - (SPLIT ? 0 : PT_BYTES);  // QS x 64 fp32
+  static constexpr int OFF_DEL = OFF_LSE + QS * 256;      // QS stages x 64 fp32
+  static constexpr int OFF_BAR = OFF_DEL + QS * 256;
+  static constexpr int NBAR = 1 + 2 * QS + 15;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t T_DV = 0, T_DK = D, T_S = 2 * D, T_DP = 2 * D + 64, T_DQ = 2 * D + 128;
+  static constexpr uint32_t T_DV = 0, T_DK = D, T_BUF = 2 * D;
 };
 
-template <int D>
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+  asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
+template <int D, bool SPLIT>
 __global__ void __launch_bounds__(320, 1)
     lg_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                   const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
                   const BwdParams prm) {
-  using L = BwdLayout<D>;
+  using L = BwdLayout<D, SPLIT>;
   constexpr int DP = D / 64;
+  constexpr int QS = L::QS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* kv_full = bars + 0;
-  uint64_t* q_full = bars + 1;    // [2]
-  uint64_t* q_empty = bars + 3;   // [2]
-  uint64_t* s_full = bars + 5;
-  uint64_t* dp_full = bars + 6;
-  uint64_t* st_free = bars + 7;
-  uint64_t* p_full = bars + 8;
-  uint64_t* ds_full = bars + 9;
-  uint64_t* pds_free = bars + 10;
-  uint64_t* dq_full = bars + 11;  // [2]
-  uint64_t* dq_free = bars + 13;  // [2]
-  uint64_t* acc_done = bars + 15;
+  uint64_t* q_full = bars + 1;        // [QS]
+  uint64_t* q_empty = bars + 1 + QS;  // [QS]
+  uint64_t* s_full = bars + 1 + 2 * QS;  // [2]
+  uint64_t* dp_full = s_full + 2;        // [2]
+  uint64_t* p_full = s_full + 4;         // [2]
+  uint64_t* ds_full = s_full + 6;        // [2]
+  uint64_t* dq_full = s_full + 8;        // [2]
+  uint64_t* dq_free = s_full + 10;       // [2]
+  uint64_t* dss_free = s_full + 12;      // [2]
+  uint64_t* acc_done = s_full + 14;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
   const float* s_lse = reinterpret_cast<const float*>(smem + L::OFF_LSE);
   const float* s_del = reinterpret_cast<const float*>(smem + L::OFF_DEL);
-  float* s_dq = reinterpret_cast<float*>(smem + L::OFF_DQS);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -226,22 +233,24 @@ __global__ void __launch_bounds__(320, 1)
   const QIter qit(prm.pat, j_lo, j_hi, prm.nqb);
   const int cnt = qit.count();
   const int N = G * cnt;
+  constexpr bool split = SPLIT;
   unsigned int* err = prm.err;
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < QS; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1 + 128);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&dp_full[s], 1);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&ds_full[s], 128);
       mbar_init(&dq_full[s], 1);
       mbar_init(&dq_free[s], 128);
+      mbar_init(&dss_free[s], 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(ds_full, 128);
-    mbar_init(pds_free, 1);
-    mbar_init(s_full, 1);
-    mbar_init(dp_full, 1);
-    mbar_init(st_free, 128);
     mbar_init(acc_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -266,8 +275,8 @@ __global__ void __launch_bounds__(320, 1)
       for (int n = 0; n < N; ++n) {
         const int h = kvh * G + n / cnt;
         const int i = qit.first_blk + n % cnt;
-        const int st = n & 1;
-        const uint32_t use = (uint32_t)(n >> 1);
+        const int st = n % QS;
+        const uint32_t use = (uint32_t)(n / QS);
         if (use > 0 && !mbar_wait(&q_empty[st], (use - 1) & 1, abort_flag, err, kErrBwdWait)) break;
         mbar_arrive_expect_tx(&q_full[st], 2 * L::QB_BYTES + 512);
         for (int p = 0; p < DP; ++p) {
@@ -288,54 +297,56 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t aK = sbase + L::OFF_K, aV = sbase + L::OFF_V;
       auto grad = [&](int m) -> bool {
         const int bb = m & 1;
+        const int st = m % QS;
         const uint32_t use = (uint32_t)(m >> 1);
-        const uint32_t aQ = sbase + L::OFF_Q + bb * L::QB_BYTES;
-        const uint32_t aDO = sbase + L::OFF_DO + bb * L::QB_BYTES;
-        const uint32_t aPT = sbase + L::OFF_PT;
-        const uint32_t aPL = sbase + L::OFF_PL;
-        const uint32_t aDS = sbase + L::OFF_DST;
-        if (!mbar_wait(p_full, (uint32_t)m & 1, abort_flag, err, kErrBwdWait)) return false;
+        const uint32_t tb = tmem + L::T_BUF + 128 * bb;
+        const uint32_t aQ = sbase + L::OFF_Q + st * L::QB_BYTES;
+        const uint32_t aDO = sbase + L::OFF_DO + st * L::QB_BYTES;
+        const uint32_t aDS = sbase + L::OFF_DST + bb * L::PT_BYTES;
+        if (!mbar_wait(&p_full[bb], use & 1, abort_flag, err, kErrBwdWait)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          tc_mma_ss(tmem + L::T_DV, sdesc_sw128(aPT + kk * 32, 16, 1024), sdesc_sw128(aDO + kk * 2048, 8192, 1024),
-                    idesc_g, (m > 0 || kk > 0) ? 1u : 0u);
-        if (prm.split_lo) {
+          tc_mma_ts(tmem + L::T_DV, tb + 8 * kk, sdesc_sw128(aDO + kk * 2048, 8192, 1024), idesc_g,
+                    (m > 0 || kk > 0) ? 1u : 0u);
+        if (split) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            tc_mma_ss(tmem + L::T_DV, sdesc_sw128(aPL + kk * 32, 16, 1024),
+            tc_mma_ss(tmem + L::T_DV, sdesc_sw128(sbase + L::OFF_PL + kk * 32, 16, 1024),
                       sdesc_sw128(aDO + kk * 2048, 8192, 1024), idesc_g, 1u);
         }
-        if (!mbar_wait(ds_full, (uint32_t)m & 1, abort_flag, err, kErrBwdWait)) return false;
+        if (!mbar_wait(&ds_full[bb], use & 1, abort_flag, err, kErrBwdWait)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          tc_mma_ss(tmem + L::T_DK, sdesc_sw128(aDS + kk * 32, 16, 1024), sdesc_sw128(aQ + kk * 2048, 8192, 1024),
-                    idesc_g, (m > 0 || kk > 0) ? 1u : 0u);
-        if (prm.split_lo) {
-          const uint32_t aDL = sbase + L::OFF_DSL;
+          tc_mma_ts(tmem + L::T_DK, tb + 96 + 8 * kk, sdesc_sw128(aQ + kk * 2048, 8192, 1024), idesc_g,
+                    (m > 0 || kk > 0) ? 1u : 0u);
+        if (split) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            tc_mma_ss(tmem + L::T_DK, sdesc_sw128(aDL + kk * 32, 16, 1024), sdesc_sw128(aQ + kk * 2048, 8192, 1024),
-                      idesc_g, 1u);
+            tc_mma_ss(tmem + L::T_DK, sdesc_sw128(sbase + L::OFF_DSL + kk * 32, 16, 1024),
+                      sdesc_sw128(aQ + kk * 2048, 8192, 1024), idesc_g, 1u);
         }
-        if (use > 0 && !mbar_wait(&dq_free[bb], (use - 1) & 1, abort_flag, err, kErrBwdWait)) return false;
-        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          tc_mma_ss(tmem + L::T_DQ + 64 * bb, sdesc_sw128(aK + kk * 2048, 16384, 1024),
-                    sdesc_sw128(aDS + kk * 2048, 8192, 1024), idesc_q, kk > 0 ? 1u : 0u);
+          tc_mma_ss(tb + 32, sdesc_sw128(aK + kk * 2048, 16384, 1024), sdesc_sw128(aDS + kk * 2048, 8192, 1024),
+                    idesc_q, kk > 0 ? 1u : 0u);
         tc_commit(&dq_full[bb]);
-        tc_commit(pds_free);
-        tc_commit(&q_empty[bb]);
+        tc_commit(&dss_free[bb]);
+        tc_commit(&q_empty[st]);
         return true;
       };
       bool ok = mbar_wait(kv_full, 0, abort_flag, err, kErrBwdWait);
       for (int n = 0; n < N && ok; ++n) {
-        const int st = n & 1;
-        const uint32_t use = (uint32_t)(n >> 1);
-        if (!mbar_wait(&q_full[st], use & 1, abort_flag, err, kErrBwdWait)) { ok = false; break; }
-        if (n >= 1 && !mbar_wait(st_free, (uint32_t)(n - 1) & 1, abort_flag, err, kErrBwdWait)) { ok = false; break; }
+        const int bb = n & 1;
+        const int st = n % QS;
+        const uint32_t tb = tmem + L::T_BUF + 128 * bb;
+        if (!mbar_wait(&q_full[st], (uint32_t)(n / QS) & 1, abort_flag, err, kErrBwdWait)) { ok = false; break; }
+        // Buffer bb last held step n-2: its dQ^T must have been drained.
+        if (n >= 2 && !mbar_wait(&dq_free[bb], (uint32_t)((n >> 1) - 1) & 1, abort_flag, err, kErrBwdWait)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t aQ = sbase + L::OFF_Q + st * L::QB_BYTES;
         const uint32_t aDO = sbase + L::OFF_DO + st * L::QB_BYTES;
@@ -343,18 +354,17 @@ __global__ void __launch_bounds__(320, 1)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ka = (kk >> 2) * 16384 + (kk & 3) * 32;
           const uint32_t kb = (kk >> 2) * 8192 + (kk & 3) * 32;
-          tc_mma_ss(tmem + L::T_S, sdesc_sw128(aK + ka, 16, 1024), sdesc_sw128(aQ + kb, 16, 1024), idesc_s,
-                    kk > 0 ? 1u : 0u);
+          tc_mma_ss(tb, sdesc_sw128(aK + ka, 16, 1024), sdesc_sw128(aQ + kb, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
-        tc_commit(s_full);
+        tc_commit(&s_full[bb]);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ka = (kk >> 2) * 16384 + (kk & 3) * 32;
           const uint32_t kb = (kk >> 2) * 8192 + (kk & 3) * 32;
-          tc_mma_ss(tmem + L::T_DP, sdesc_sw128(aV + ka, 16, 1024), sdesc_sw128(aDO + kb, 16, 1024), idesc_s,
+          tc_mma_ss(tb + 64, sdesc_sw128(aV + ka, 16, 1024), sdesc_sw128(aDO + kb, 16, 1024), idesc_s,
                     kk > 0 ? 1u : 0u);
         }
-        tc_commit(dp_full);
+        tc_commit(&dp_full[bb]);
         if (n >= 1 && !grad(n - 1)) { ok = false; break; }
       }
       if (ok && N > 0) ok = grad(N - 1);
@@ -372,72 +382,89 @@ __global__ void __launch_bounds__(320, 1)
     int n = 0;
     for (; n < N; ++n) {
       const int i = qit.first_blk + n % cnt;
-      const int st = n & 1;
+      const int st = n % QS;
+      const int bb = n & 1;
       const uint32_t use = (uint32_t)(n >> 1);
-      const bool vis = krow_live && in_list(prm.pat, i, kvb);
+      const uint32_t tl = t_lane + L::T_BUF + 128 * bb;
+      const bool vis = krow_live && in_list(prm.pat, i, kvb);  // warp-uniform
       const bool diag = (i == kvb);
-      if (!__all_sync(0xffffffffu, mbar_wait(&q_full[st], use & 1, abort_flag, err, kErrBwdWait))) break;
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full, (uint32_t)n & 1, abort_flag, err, kErrBwdWait))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&q_full[st], (uint32_t)(n / QS) & 1, abort_flag, err, kErrBwdWait)))
+        break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[bb], use & 1, abort_flag, err, kErrBwdWait))) break;
       tc_fence_after();
       float pf[64];
       {
         uint32_t sr[64];
-        tmem_ld64(t_lane + L::T_S, sr);
+        tmem_ld64(tl, sr);
         const float* lse = s_lse + st * 64;
+        if (vis) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float x = fmaf(__uint_as_float(sr[c]), sl2, -lse[c] * kLog2e);
-          const bool keep = vis && (!diag || rr <= c);
-          pf[c] = keep ? ex2_approx(x) : 0.f;
+          for (int c = 0; c < 64; ++c) {
+            const float p = ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -lse[c] * kLog2e));
+            pf[c] = (diag && c < rr) ? 0.f : p;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) pf[c] = 0.f;
         }
       }
-      // P^T / dS^T buffers are free once the gradient GEMMs of step n-1 completed.
-      if (n >= 1 &&
-          !__all_sync(0xffffffffu, mbar_wait(pds_free, (uint32_t)(n - 1) & 1, abort_flag, err, kErrBwdWait)))
-        break;
+      {
+        uint32_t hi[32];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t hi[4], lo[4];
+        for (int c = 0; c < 32; ++c) hi[c] = pack_bf16x2(pf[2 * c], pf[2 * c + 1]);
+        tmem_st32(tl, hi);  // P^T over S^T columns [0, 32)
+        if (split) {
+          // The single residual buffer is free once the gradient GEMMs of step n-1 completed.
+          if (n >= 1 && !__all_sync(0xffffffffu, mbar_wait(&dss_free[bb ^ 1], (uint32_t)((n - 1) >> 1) & 1,
+                                                           abort_flag, err, kErrBwdWait)))
+            break;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = pf[8 * c + 2 * e], p1 = pf[8 * c + 2 * e + 1];
-          hi[e] = pack_bf16x2(p0, p1);
-          lo[e] = pack_bf16x2(p0 - __uint_as_float(hi[e] << 16), p1 - __uint_as_float(hi[e] & 0xffff0000u));
+          for (int c = 0; c < 8; ++c) {
+            uint32_t lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              lo[e] = pack_bf16x2(pf[8 * c + 2 * e] - __uint_as_float(hi[4 * c + e] << 16),
+                                  pf[8 * c + 2 * e + 1] - __uint_as_float(hi[4 * c + e] & 0xffff0000u));
+            st_shared_v4(sbase + L::OFF_PL + sw128_offset(r, c), lo[0], lo[1], lo[2], lo[3]);
+          }
+          fence_async_smem();
         }
-        const uint32_t off = sw128_offset(r, c);
-        st_shared_v4(sbase + L::OFF_PT + off, hi[0], hi[1], hi[2], hi[3]);
-        if (prm.split_lo) st_shared_v4(sbase + L::OFF_PL + off, lo[0], lo[1], lo[2], lo[3]);
       }
-      fence_async_smem();
-      mbar_arrive(p_full);
-      if (!__all_sync(0xffffffffu, mbar_wait(dp_full, (uint32_t)n & 1, abort_flag, err, kErrBwdWait))) break;
-      tc_fence_after();
-      uint32_t dpr[64];
-      tmem_ld64(t_lane + L::T_DP, dpr);
       tc_fence_before();
-      mbar_arrive(st_free);
-      const float* del = s_del + st * 64;
-      const uint32_t drow = sbase + L::OFF_DST;
+      mbar_arrive(&p_full[bb]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&dp_full[bb], use & 1, abort_flag, err, kErrBwdWait))) break;
+      tc_fence_after();
+      {
+        uint32_t dpr[64];
+        tmem_ld64(tl + 64, dpr);
+        const float* del = s_del + st * 64;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) pf[c] = pf[c] * (__uint_as_float(dpr[c]) - del[c]);  // pf now holds dS^T
+      }
+      uint32_t hi[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) hi[c] = pack_bf16x2(pf[2 * c], pf[2 * c + 1]);
+      tmem_st32(tl + 96, hi);  // dS^T over dP^T columns [32, 64)
+      // The shared dS^T buffer bb last fed dQ^T of step n-2.
+      if (n >= 2 &&
+          !__all_sync(0xffffffffu, mbar_wait(&dss_free[bb], (use - 1) & 1, abort_flag, err, kErrBwdWait)))
+        break;
+      const uint32_t drow = sbase + L::OFF_DST + bb * L::PT_BYTES;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        float d8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) d8[e] = pf[8 * c + e] * (__uint_as_float(dpr[8 * c + e]) - del[8 * c + e]);
-        uint32_t hi[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) hi[e] = pack_bf16x2(d8[2 * e], d8[2 * e + 1]);
-        st_shared_v4(drow + sw128_offset(r, c), hi[0], hi[1], hi[2], hi[3]);
-        if (prm.split_lo) {
+        st_shared_v4(drow + sw128_offset(r, c), hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+        if (split) {
           uint32_t lo[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            lo[e] = pack_bf16x2(d8[2 * e] - __uint_as_float(hi[e] << 16),
-                                d8[2 * e + 1] - __uint_as_float(hi[e] & 0xffff0000u));
+            lo[e] = pack_bf16x2(pf[8 * c + 2 * e] - __uint_as_float(hi[4 * c + e] << 16),
+                                pf[8 * c + 2 * e + 1] - __uint_as_float(hi[4 * c + e] & 0xffff0000u));
           st_shared_v4(sbase + L::OFF_DSL + sw128_offset(r, c), lo[0], lo[1], lo[2], lo[3]);
         }
       }
       fence_async_smem();
-      mbar_arrive(ds_full);
+      tc_fence_before();
+      mbar_arrive(&ds_full[bb]);
       mbar_arrive(&q_empty[st]);
     }
 
@@ -502,43 +529,29 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else {
     // ------------------------------------------------------------ dQ drain warps 6-9
-    const int t = threadIdx.x - 192;
     const int quarter = warp & 3;
     // dQ^T row (= d) held by this thread: M = D rows; for M = 64 the rows sit in
     // lanes 0-15 of each 32-lane quarter.
     const int d = (D == 128) ? quarter * 32 + lane : quarter * 16 + lane;
     const bool dvalid = (D == 128) || lane < 16;
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
-    bool ok = true;
     for (int n = 0; n < N; ++n) {
       const int h = kvh * G + n / cnt;
       const int i = qit.first_blk + n % cnt;
       const int bb = n & 1;
-      const uint32_t use = (uint32_t)(n >> 1);
-      ok = ok && mbar_wait(&dq_full[bb], use & 1, abort_flag, err, kErrBwdWait);
-      const bool wok = __all_sync(0xffffffffu, ok);
-      if (wok) {
-        tc_fence_after();
-        uint32_t v[64];
-        tmem_ld64(t_lane + L::T_DQ + 64 * bb, v);
-        tc_fence_before();
-        mbar_arrive(&dq_free[bb]);
-        if (dvalid) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&dq_full[bb], (uint32_t)(n >> 1) & 1, abort_flag, err, kErrBwdWait)))
+        break;
+      tc_fence_after();
+      uint32_t v[64];
+      tmem_ld64(t_lane + L::T_BUF + 128 * bb + 32, v);
+      tc_fence_before();
+      mbar_arrive(&dq_free[bb]);
+      if (dvalid) {
+        float* dst = prm.dq_acc + (((size_t)b * prm.H + h) * prm.S + 64 * (size_t)i) * D + d;
 #pragma unroll
-          for (int c = 0; c < 64; ++c) s_dq[c * D + d] = __uint_as_float(v[c]);
-        }
+        for (int c = 0; c < 64; ++c) red_add_f32(dst + (size_t)c * D, __uint_as_float(v[c]));
       }
-      fence_async_smem();
-      named_bar_sync(2, 128);
-      if (t == 0 && !*abort_flag) {
-        float* dst = prm.dq_acc + (((size_t)b * prm.H + h) * prm.S + 64 * (size_t)i) * D;
-        bulk_reduce_add_f32(dst, s_dq, 64 * D * 4);
-        bulk_commit();
-        bulk_wait_read_all();
-      }
-      named_bar_sync(2, 128);
     }
-    if (t == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -549,23 +562,29 @@ __global__ void __launch_bounds__(320, 1)
   }
 }
 
-template <int D>
+template <int D, bool SPLIT>
 static cudaError_t launch_bwd_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                    const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
                                    const BwdParams& prm, int B, cudaStream_t stream) {
-  using L = BwdLayout<D>;
-  cudaError_t e = cudaFuncSetAttribute(lg_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+  using L = BwdLayout<D, SPLIT>;
+  static_assert(L::ALLOC <= 232448, "shared memory budget");
+  cudaError_t e =
+      cudaFuncSetAttribute(lg_bwd_kernel<D, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (e != cudaSuccess) return e;
   dim3 grid(prm.nkt, prm.Hkv, B);
-  lg_bwd_kernel<D><<<grid, 320, L::ALLOC, stream>>>(tq, tk, tv, tdo, tdk, tdv, prm);
+  lg_bwd_kernel<D, SPLIT><<<grid, 320, L::ALLOC, stream>>>(tq, tk, tv, tdo, tdk, tdv, prm);
   return cudaGetLastError();
 }
 
 cudaError_t launch_bwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv, const BwdParams& prm,
                        int B, cudaStream_t stream) {
-  if (D == 64) return launch_bwd_impl<64>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
-  return launch_bwd_impl<128>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
+  if (prm.split_lo) {
+    if (D == 64) return launch_bwd_impl<64, true>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
+    return launch_bwd_impl<128, true>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
+  }
+  if (D == 64) return launch_bwd_impl<64, false>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
+  return launch_bwd_impl<128, false>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
 }
 
 }  // namespace lg
