@@ -142,7 +142,7 @@ cudaError_t launch_bwd_dq(const float* dq_acc, void* dq, int dq_f32, float scale
 //   dK  += dS^T Q_i         (M=128,    N=D,    K=64; dS^T read from TMEM)
 //   dQ_i^T = K^T dS^T       (M=D,      N=64,   K=128; dS^T from shared memory)
 // with P^T = exp(scale S^T - LSE) on the mask and dS^T = P^T (dP^T - Delta),
-// computed by four warps that each own 32 KV rows (TMEM lanes). They write
+// computed by eight warps, two per 32 KV rows (TMEM lanes). They write
 // bf16 P^T and dS^T back into TMEM over the S^T / dP^T columns they have
 // read (A operands of the dV / dK products), and dS^T also to shared memory
 // (B operand of dQ^T). dQ_i^T lands in the middle 64 columns of the same
@@ -159,8 +159,8 @@ cudaError_t launch_bwd_dq(const float* dq_acc, void* dq, int dq_f32, float scale
 // |dK| ~ 4 is the whole 1e-2 error budget). Without GQA the plain five GEMMs
 // are used.
 //
-// Warps: 0-3 P/dS + epilogue, 4 TMA producer, 5 TMEM owner + MMA issuer,
-// 6-9 dQ drain. TMEM columns: dV [0,D), dK [D,2D), step buffer b at
+// Warps: 0-7 P/dS + epilogue (two per TMEM lane quarter, 32 query columns
+// each), 8 TMA producer, 9 TMEM owner + MMA issuer, 10-13 dQ drain. TMEM columns: dV [0,D), dK [D,2D), step buffer b at
 // 2D + 128b: S^T [0,64) then P^T in [0,32); dP^T [64,128) then dS^T in
 // [96,128); dQ^T in [32,96).
 // ---------------------------------------------------------------------------
@@ -180,7 +180,7 @@ struct BwdLayout {
   static constexpr int OFF_LSE = OFF_DSL + (SPLIT ? PT_BYTES : 0) - (SPLIT ? 0 : PT_BYTES);  // QS x 64 fp32
   static constexpr int OFF_DEL = OFF_LSE + QS * 256;      // QS stages x 64 fp32
   static constexpr int OFF_BAR = OFF_DEL + QS * 256;
-  static constexpr int NBAR = 1 + 2 * QS + 15;
+  static constexpr int NBAR = 1 + 2 * QS + 19;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;
@@ -193,7 +193,7 @@ __device__ __forceinline__ void red_add_f32(float* p, float v) {
 }
 
 template <int D, bool SPLIT>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
     lg_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                   const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
@@ -217,6 +217,8 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* dq_free = s_full + 10;       // [2]
   uint64_t* dss_free = s_full + 12;      // [2]
   uint64_t* acc_done = s_full + 14;
+  uint64_t* s_read = s_full + 15;   // [2] every P/dS warp has read S^T of the buffer
+  uint64_t* dp_read = s_full + 17;  // [2] every P/dS warp has read dP^T of the buffer
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
   const float* s_lse = reinterpret_cast<const float*>(smem + L::OFF_LSE);
@@ -240,22 +242,24 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(kv_full, 1);
     for (int s = 0; s < QS; ++s) {
       mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 1 + 128);
+      mbar_init(&q_empty[s], 1 + 256);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&dp_full[s], 1);
-      mbar_init(&p_full[s], 128);
-      mbar_init(&ds_full[s], 128);
+      mbar_init(&p_full[s], 256);
+      mbar_init(&ds_full[s], 256);
       mbar_init(&dq_full[s], 1);
       mbar_init(&dq_free[s], 128);
       mbar_init(&dss_free[s], 1);
+      mbar_init(&s_read[s], 256);
+      mbar_init(&dp_read[s], 256);
     }
     mbar_init(acc_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, L::TMEM_COLS);
     tmem_relinquish();
   }
@@ -264,7 +268,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       mbar_arrive_expect_tx(kv_full, 2 * L::KV_BYTES);
@@ -288,7 +292,7 @@ __global__ void __launch_bounds__(320, 1)
         bulk_load(smem + L::OFF_DEL + st * 256, prm.delta + row, 256, &q_full[st]);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(128, 64, false, false);
@@ -370,13 +374,17 @@ __global__ void __launch_bounds__(320, 1)
       if (ok && N > 0) ok = grad(N - 1);
       tc_commit(acc_done);
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ P / dS warps
-    const int r = threadIdx.x;  // KV row of the tile == TMEM lane
+    // Two warps per TMEM lane quarter: warp w owns KV rows 32 (w % 4) .. +31
+    // and query columns [32 (w / 4), +32) of the step.
+    const int hf = warp >> 2;
+    const int c0 = 32 * hf;
+    const int r = (warp & 3) * 32 + lane;  // KV row of the tile == TMEM lane
     const int kvb = 2 * u + (r >> 6);
     const int rr = r & 63;
     const bool krow_live = kvb < prm.nqb;
-    const uint32_t t_lane = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t t_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const float sl2 = prm.scale_log2;
     constexpr float kLog2e = 1.4426950408889634f;
     int n = 0;
@@ -392,40 +400,46 @@ __global__ void __launch_bounds__(320, 1)
         break;
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[bb], use & 1, abort_flag, err, kErrBwdWait))) break;
       tc_fence_after();
-      float pf[64];
+      float pf[32];
       {
-        uint32_t sr[64];
-        tmem_ld64(tl, sr);
-        const float* lse = s_lse + st * 64;
+        uint32_t sr[32];
+        tmem_ld32(tl + c0, sr);
+        tc_fence_before();
+        mbar_arrive(&s_read[bb]);
+        const float* lse = s_lse + st * 64 + c0;
         if (vis) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const float p = ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -lse[c] * kLog2e));
-            pf[c] = (diag && c < rr) ? 0.f : p;
+          for (int e = 0; e < 32; ++e) {
+            const float p = ex2_approx(fmaf(__uint_as_float(sr[e]), sl2, -lse[e] * kLog2e));
+            pf[e] = (diag && c0 + e < rr) ? 0.f : p;
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) pf[c] = 0.f;
+          for (int e = 0; e < 32; ++e) pf[e] = 0.f;
         }
       }
+      // P^T goes over S^T columns [0, 32), which hold S^T the other warp of this
+      // lane quarter may still be reading: wait until every warp has read S^T.
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_read[bb], use & 1, abort_flag, err, kErrBwdWait))) break;
+      tc_fence_after();
       {
-        uint32_t hi[32];
+        uint32_t hi[16];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) hi[c] = pack_bf16x2(pf[2 * c], pf[2 * c + 1]);
-        tmem_st32(tl, hi);  // P^T over S^T columns [0, 32)
+        for (int e = 0; e < 16; ++e) hi[e] = pack_bf16x2(pf[2 * e], pf[2 * e + 1]);
+        tmem_st16(tl + 16 * hf, hi);  // P^T over S^T columns [0, 32)
         if (split) {
           // The single residual buffer is free once the gradient GEMMs of step n-1 completed.
           if (n >= 1 && !__all_sync(0xffffffffu, mbar_wait(&dss_free[bb ^ 1], (uint32_t)((n - 1) >> 1) & 1,
                                                            abort_flag, err, kErrBwdWait)))
             break;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < 4; ++c) {
             uint32_t lo[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e)
               lo[e] = pack_bf16x2(pf[8 * c + 2 * e] - __uint_as_float(hi[4 * c + e] << 16),
                                   pf[8 * c + 2 * e + 1] - __uint_as_float(hi[4 * c + e] & 0xffff0000u));
-            st_shared_v4(sbase + L::OFF_PL + sw128_offset(r, c), lo[0], lo[1], lo[2], lo[3]);
+            st_shared_v4(sbase + L::OFF_PL + sw128_offset(r, 4 * hf + c), lo[0], lo[1], lo[2], lo[3]);
           }
           fence_async_smem();
         }
@@ -435,31 +449,36 @@ __global__ void __launch_bounds__(320, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(&dp_full[bb], use & 1, abort_flag, err, kErrBwdWait))) break;
       tc_fence_after();
       {
-        uint32_t dpr[64];
-        tmem_ld64(tl + 64, dpr);
-        const float* del = s_del + st * 64;
+        uint32_t dpr[32];
+        tmem_ld32(tl + 64 + c0, dpr);
+        tc_fence_before();
+        mbar_arrive(&dp_read[bb]);
+        const float* del = s_del + st * 64 + c0;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) pf[c] = pf[c] * (__uint_as_float(dpr[c]) - del[c]);  // pf now holds dS^T
+        for (int e = 0; e < 32; ++e) pf[e] = pf[e] * (__uint_as_float(dpr[e]) - del[e]);  // pf now holds dS^T
       }
-      uint32_t hi[32];
+      // dS^T goes over dP^T columns [32, 64): same hazard as for P^T.
+      if (!__all_sync(0xffffffffu, mbar_wait(&dp_read[bb], use & 1, abort_flag, err, kErrBwdWait))) break;
+      tc_fence_after();
+      uint32_t hi[16];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) hi[c] = pack_bf16x2(pf[2 * c], pf[2 * c + 1]);
-      tmem_st32(tl + 96, hi);  // dS^T over dP^T columns [32, 64)
+      for (int e = 0; e < 16; ++e) hi[e] = pack_bf16x2(pf[2 * e], pf[2 * e + 1]);
+      tmem_st16(tl + 96 + 16 * hf, hi);  // dS^T over dP^T columns [32, 64)
       // The shared dS^T buffer bb last fed dQ^T of step n-2.
       if (n >= 2 &&
           !__all_sync(0xffffffffu, mbar_wait(&dss_free[bb], (use - 1) & 1, abort_flag, err, kErrBwdWait)))
         break;
       const uint32_t drow = sbase + L::OFF_DST + bb * L::PT_BYTES;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        st_shared_v4(drow + sw128_offset(r, c), hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
+      for (int c = 0; c < 4; ++c) {
+        st_shared_v4(drow + sw128_offset(r, 4 * hf + c), hi[4 * c], hi[4 * c + 1], hi[4 * c + 2], hi[4 * c + 3]);
         if (split) {
           uint32_t lo[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             lo[e] = pack_bf16x2(pf[8 * c + 2 * e] - __uint_as_float(hi[4 * c + e] << 16),
                                 pf[8 * c + 2 * e + 1] - __uint_as_float(hi[4 * c + e] & 0xffff0000u));
-          st_shared_v4(sbase + L::OFF_DSL + sw128_offset(r, c), lo[0], lo[1], lo[2], lo[3]);
+          st_shared_v4(sbase + L::OFF_DSL + sw128_offset(r, 4 * hf + c), lo[0], lo[1], lo[2], lo[3]);
         }
       }
       fence_async_smem();
@@ -469,11 +488,13 @@ __global__ void __launch_bounds__(320, 1)
     }
 
     // ------------------------------------------------------------ dK, dV epilogue
+    // Warp (quarter, half) writes rows of its quarter, columns [half * D/2, +D/2).
     bool ok = (n == N) && !*abort_flag;
     if (ok) ok = mbar_wait(acc_done, 0, abort_flag, err, kErrBwdWait);
     ok = __all_sync(0xffffffffu, ok);
+    constexpr int CH = D / 64;  // 32-column chunks per half
     if (ok && prm.grad_f32) {
-      // fp32 gradients: each thread stores its KV row straight from TMEM.
+      // fp32 gradients: each thread stores its part of a KV row straight from TMEM.
       tc_fence_after();
       const int krow = 128 * u + r;
 #pragma unroll
@@ -482,11 +503,12 @@ __global__ void __launch_bounds__(320, 1)
         const float mul = which == 0 ? 1.f : prm.scale;
         float* dst = (which == 0 ? prm.dv_f32 : prm.dk_f32) + (((size_t)b * prm.S + krow) * prm.Hkv + kvh) * D;
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
+        for (int q = 0; q < CH; ++q) {
+          const int col = hf * (D / 2) + 32 * q;
           uint32_t o[32];
-          tmem_ld32(t_lane + tcol + 32 * ch, o);
+          tmem_ld32(t_lane + tcol + col, o);
           if (krow < prm.S) {
-            float4* d4 = reinterpret_cast<float4*>(dst + 32 * ch);
+            float4* d4 = reinterpret_cast<float4*>(dst + col);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
               d4[e] = make_float4(__uint_as_float(o[4 * e]) * mul, __uint_as_float(o[4 * e + 1]) * mul,
@@ -502,15 +524,16 @@ __global__ void __launch_bounds__(320, 1)
         const float mul = which == 0 ? 1.f : prm.scale;
         const uint32_t dst = sbase + (which == 0 ? L::OFF_V : L::OFF_K);
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
+        for (int q = 0; q < CH; ++q) {
+          const int col = hf * (D / 2) + 32 * q;
           uint32_t o[32];
-          tmem_ld32(t_lane + tcol + 32 * ch, o);
-          const uint32_t panel = dst + (uint32_t)((32 * ch) >> 6) * 16384;
-          const int c0 = ((32 * ch) & 63) >> 3;
+          tmem_ld32(t_lane + tcol + col, o);
+          const uint32_t panel = dst + (uint32_t)(col >> 6) * 16384;
+          const int cq = (col & 63) >> 3;
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             const float* f = reinterpret_cast<const float*>(&o[8 * q4]);
-            st_shared_v4(panel + sw128_offset(r, c0 + q4), pack_bf16x2(f[0] * mul, f[1] * mul),
+            st_shared_v4(panel + sw128_offset(r, cq + q4), pack_bf16x2(f[0] * mul, f[1] * mul),
                          pack_bf16x2(f[2] * mul, f[3] * mul), pack_bf16x2(f[4] * mul, f[5] * mul),
                          pack_bf16x2(f[6] * mul, f[7] * mul));
           }
@@ -518,8 +541,8 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     fence_async_smem();
-    named_bar_sync(1, 128);
-    if (r == 0 && !*abort_flag && !prm.grad_f32) {
+    named_bar_sync(1, 256);
+    if (threadIdx.x == 0 && !*abort_flag && !prm.grad_f32) {
       for (int p = 0; p < DP; ++p) {
         tma_store_4d(&tmdV, smem + L::OFF_V + p * 16384, 64 * p, kvh, 128 * u, b);
         tma_store_4d(&tmdK, smem + L::OFF_K + p * 16384, 64 * p, kvh, 128 * u, b);
@@ -528,7 +551,7 @@ __global__ void __launch_bounds__(320, 1)
       bulk_wait_all();
     }
   } else {
-    // ------------------------------------------------------------ dQ drain warps 6-9
+    // ------------------------------------------------------------ dQ drain warps 10-13
     const int quarter = warp & 3;
     // dQ^T row (= d) held by this thread: M = D rows; for M = 64 the rows sit in
     // lanes 0-15 of each 32-lane quarter.
@@ -556,7 +579,7 @@ __global__ void __launch_bounds__(320, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);
   }
@@ -572,7 +595,7 @@ static cudaError_t launch_bwd_impl(const CUtensorMap& tq, const CUtensorMap& tk,
       cudaFuncSetAttribute(lg_bwd_kernel<D, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (e != cudaSuccess) return e;
   dim3 grid(prm.nkt, prm.Hkv, B);
-  lg_bwd_kernel<D, SPLIT><<<grid, 320, L::ALLOC, stream>>>(tq, tk, tv, tdo, tdk, tdv, prm);
+  lg_bwd_kernel<D, SPLIT><<<grid, 448, L::ALLOC, stream>>>(tq, tk, tv, tdo, tdk, tdv, prm);
   return cudaGetLastError();
 }
 
