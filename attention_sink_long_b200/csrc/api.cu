@@ -4,7 +4,9 @@
 // except lg_device_status, which says so.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "lg_kernels.h"
 #include "lg_pattern.cuh"
@@ -36,7 +38,7 @@ lg_status_t check_prefill_shape(const lg_pattern_t* p, int B, int S, int H, int 
   if (p->block_size != 64) return LG_ERR_UNSUPPORTED;
   if (S % 64 != 0) return LG_ERR_UNSUPPORTED;
   if (D != 64 && D != 128) return LG_ERR_UNSUPPORTED;
-  if (B > 65535 || H > 65535) return LG_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535 || (long long)((S + 127) / 128) * H > 2147483647LL) return LG_ERR_UNSUPPORTED;
   return LG_OK;
 }
 
@@ -305,6 +307,19 @@ lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* p, const void* q, const void*
   prm.nkt = (S + 127) / 128;
   prm.scale = scale;
   prm.scale_log2 = scale * 1.4426950408889634f;
+  // Heavy KV tiles: query-list length above twice the median (e.g. the sink
+  // tile, seen by every query). Scheduled first; at most 128 of them.
+  {
+    std::vector<int> counts(prm.nkt);
+    for (int t = 0; t < prm.nkt; ++t)
+      counts[t] = lg::QIter(*p, 2 * t, imin(2 * t + 1, prm.nqb - 1), prm.nqb).count();
+    std::vector<int> sorted_counts(counts);
+    std::nth_element(sorted_counts.begin(), sorted_counts.begin() + prm.nkt / 2, sorted_counts.end());
+    const int median = sorted_counts[prm.nkt / 2];
+    prm.n_heavy = 0;
+    for (int t = 0; t < prm.nkt && prm.n_heavy < 128; ++t)
+      if (counts[t] > 2 * median) prm.heavy[prm.n_heavy++] = t;
+  }
   // dK and dV of a KV head sum over its H / Hkv query heads, so their size
   // grows with the group; the bf16 residuals of P and dS then keep the bf16
   // rounding of those operands out of dV and dK.

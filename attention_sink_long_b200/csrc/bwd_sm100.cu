@@ -226,9 +226,27 @@ __global__ void __launch_bounds__(448, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int u = blockIdx.x;
-  const int kvh = blockIdx.y;
-  const int b = blockIdx.z;
+  // Launch order: first the heavy KV tiles (those a sink or strided block makes
+  // visible to many more queries, listed by the host) of every head, then the
+  // other tiles head by head in ascending order -- so the long CTAs start in
+  // the first waves while CTAs running together still share one head's Q, dO
+  // and dQ accumulator rows in L2.
+  int u, kvh;
+  {
+    const int L = blockIdx.x;
+    const int nh = prm.n_heavy;
+    if (L < nh * prm.Hkv) {
+      u = prm.heavy[L / prm.Hkv];
+      kvh = L % prm.Hkv;
+    } else {
+      const int rest = prm.nkt - nh;
+      const int L2 = L - nh * prm.Hkv;
+      kvh = L2 / rest;
+      u = L2 % rest;
+      for (int k = 0; k < nh; ++k) u += (prm.heavy[k] <= u) ? 1 : 0;  // skip the heavy tiles
+    }
+  }
+  const int b = blockIdx.y;
   const int G = prm.H / prm.Hkv;
   const int j_lo = 2 * u;
   const int j_hi = imin(2 * u + 1, prm.nqb - 1);
@@ -594,7 +612,7 @@ static cudaError_t launch_bwd_impl(const CUtensorMap& tq, const CUtensorMap& tk,
   cudaError_t e =
       cudaFuncSetAttribute(lg_bwd_kernel<D, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (e != cudaSuccess) return e;
-  dim3 grid(prm.nkt, prm.Hkv, B);
+  dim3 grid(prm.nkt * prm.Hkv, B);
   lg_bwd_kernel<D, SPLIT><<<grid, 448, L::ALLOC, stream>>>(tq, tk, tv, tdo, tdk, tdv, prm);
   return cudaGetLastError();
 }

@@ -77,7 +77,9 @@ __global__ void __launch_bounds__(320, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int span = prm.nqt - 1 - (int)blockIdx.x;  // heaviest (latest) spans first
+  // Spans vary fastest in launch order, from the last (heaviest under a causal
+  // mask) to the first; CTAs running together share one head's K/V in L2.
+  const int span = prm.nqt - 1 - (int)blockIdx.x;
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const int kvh = h / (prm.H / prm.Hkv);

@@ -33,6 +33,8 @@ struct BwdParams {
   int nkt;  // ceil(S / 128) KV tiles
   float scale;       // softmax scale
   float scale_log2;  // scale * log2(e)
+  int n_heavy;       // KV tiles scheduled first (for every head), ascending
+  int heavy[128];    // their tile indices; see lg_bwd_kernel's launch order
   int split_lo;      // 1: P and dS also enter dV / dK as bf16 residuals (GQA groups)
   int grad_f32;      // 1: dK / dV written as fp32 straight from the accumulators
   float* dk_f32;     // [B, S, Hkv, D] when grad_f32
