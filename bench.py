@@ -58,6 +58,57 @@ def parse_args(argv=None):
     return ap.parse_args(argv)
 
 
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest value over all ranks (identity without a process group)."""
+    if dist is None:
+        return value
+    import torch
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def pick_peak(peaks, clocks, bound):
+    """Roofline denominator: the measured burst figure, or the sustained one
+    when the power cap throttled the SM clock during the timed region."""
+    if bound == "hbm":
+        return peaks["hbm_gbs"], "copy bandwidth"
+    capped = bool(clocks) and "sw_power_cap" in clocks.get("reasons", [])
+    if capped:
+        return peaks["bf16_tflops_sustained"], "sustained (sw_power_cap active)"
+    return peaks["bf16_tflops"], "burst"
+
+
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "kernel_traffic.json")
+
+
+def sources_sha256(files):
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(part_name):
+    """DRAM bytes per launch of this part from the committed ncu capture, or
+    None when there is none or the kernel's sources changed since."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            table = json.load(f)
+    except Exception:
+        return None
+    e = table.get(part_name)
+    if not e:
+        return None
+    if sources_sha256(e["sources"]) != e["sources_sha256"]:
+        return None
+    return int(e["dram_bytes_per_launch"])
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -343,10 +394,7 @@ def cuda_arm(args, rank, world, dist):
             prev = evs[k][i]
     assert lg.lg_device_status(local) == 0, "a bounded device wait ran out during the timed region"
 
-    if dist is not None:
-        tt = torch.tensor([total_ms], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(total_ms, dist, device)
 
     weights = step.step_weights()
     step_flops = sum(w * p[2] for w, p in zip(weights, step.parts))
@@ -357,6 +405,7 @@ def cuda_arm(args, rank, world, dist):
     value = world * step_flops / (ms_per_step * 1e-3) / 1e12
 
     peaks, peak_src = load_peaks()
+    tensor_peak, tensor_kind = pick_peak(peaks, clk, "tensor")
     rows = {}
     dominant = None
     for i, (name, kind, flops, nbytes, nl) in enumerate(step.parts):
@@ -366,7 +415,7 @@ def cuda_arm(args, rank, world, dist):
             r["gbs"] = round(nbytes / (ms * 1e-3) / 1e9, 1)
             r["frac_hbm"] = round(r["gbs"] / peaks["hbm_gbs"], 4)
         else:
-            r["frac_bf16"] = round(r["useful_tflops"] / peaks["bf16_tflops"], 4)
+            r["frac_bf16"] = round(r["useful_tflops"] / tensor_peak, 4)
         rows[name] = r
         if dominant is None or ms * weights[i] > dominant[1]:
             dominant = (i, ms * weights[i])
@@ -376,13 +425,15 @@ def cuda_arm(args, rank, world, dist):
     if dkind.startswith("decode"):
         achieved = dbytes / (dms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None}
+                "frac": round(achieved / peaks["hbm_gbs"], 4)}
+        roof["peak_source"] = f"{peak_src} (copy bandwidth)"
     else:
         achieved = dflops / (dms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None}
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": round(achieved / tensor_peak, 4)}
+        roof["peak_source"] = f"{peak_src} bf16 dense, {tensor_kind}"
+    roof["traffic"] = recorded_traffic(dname)
     roof["kernel"] = dname
-    roof["peak_source"] = f"{peak_src} (burst)"
 
     # End-to-end through the public API with pinned host buffers.
     e2e = None
@@ -411,11 +462,7 @@ def cuda_arm(args, rank, world, dist):
                 h.copy_(d, non_blocking=True)
         e1.record(step.stream)
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1) / ek
-        if dist is not None:
-            tt = torch.tensor([ems], device=device)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ems = float(tt.item())
+        ems = max_over_ranks(e0.elapsed_time(e1) / ek, dist, device)
         e2e = {"value": round(world * step_flops / (ems * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(ems, 3), "steps": ek}
 

@@ -1,0 +1,98 @@
+"""Host-side logic of bench.py, on CPU: the max-over-ranks timing across two
+gloo ranks, the roofline denominator choice, the recorded ncu traffic lookup,
+and the oracle reference arm (alone and under torchrun with two ranks, where
+only rank 0 works and prints)."""
+
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _rank_main(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        v = bench.max_over_ranks(10.0 + rank * 2.5, dist, "cpu")
+        out[rank] = v
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_two_gloo_ranks():
+    import socket
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_rank_main, args=(2, port, out), nprocs=2, start_method="spawn", join=True)
+    assert dict(out) == {0: 12.5, 1: 12.5}
+    assert bench.max_over_ranks(3.0, None, "cpu") == 3.0
+
+
+def test_peak_choice():
+    peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1650.0, "bf16_tflops_sustained": 1400.0}
+    assert bench.pick_peak(peaks, {"reasons": []}, "tensor") == (1650.0, "burst")
+    assert bench.pick_peak(peaks, {"reasons": ["sw_power_cap"]}, "tensor")[0] == 1400.0
+    assert bench.pick_peak(peaks, None, "tensor")[0] == 1650.0
+    assert bench.pick_peak(peaks, {"reasons": ["sw_power_cap"]}, "hbm")[0] == 6500.0
+
+
+def test_recorded_traffic_is_tied_to_kernel_sources(tmp_path, monkeypatch):
+    assert bench.recorded_traffic("no such part") is None
+    with open(bench.TRAFFIC_FILE) as f:
+        table = json.load(f)
+    for name, e in table.items():
+        assert set(e) >= {"sources", "sources_sha256", "dram_bytes_per_launch", "capture"}
+        # a stale hash reads as "no capture for this kernel"
+        bad = dict(table)
+        bad[name] = dict(e, sources_sha256="0" * 64)
+        p = tmp_path / "t.json"
+        p.write_text(json.dumps(bad))
+        monkeypatch.setattr(bench, "TRAFFIC_FILE", str(p))
+        assert bench.recorded_traffic(name) is None
+        monkeypatch.setattr(bench, "TRAFFIC_FILE", os.path.join(ROOT, "profiles", "kernel_traffic.json"))
+
+
+def test_workloads_and_useful_work():
+    w = bench.workload("step32k")
+    assert w["prefill"]["S"] == 32768 and w["decode"]["L"] == 4160
+    assert bench.pairs_of(bench.SINK_WINDOW, 32768) == 126763008
+    assert bench.pairs_of(bench.FULL, 32768) == 32768 * 32769 // 2
+    assert bench.pairs_of(bench.BLOCK_SPARSE, 131072) == 398032896
+
+
+def _run(cmd, timeout=240):
+    return subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=timeout,
+                          env=dict(os.environ, MASTER_ADDR="127.0.0.1"))
+
+
+def test_reference_arm_prints_one_line():
+    r = _run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "1"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+@pytest.mark.slow
+def test_reference_arm_under_torchrun_two_ranks():
+    r = _run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+              "--master-addr", "127.0.0.1", "--master-port", "29533", "bench.py", "--impl", "reference",
+              "--gpus", "2", "--steps", "1", "--warmup", "0"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip().startswith("{")]
+    assert len(lines) == 1 and json.loads(lines[0])["n_gpus"] == 2
