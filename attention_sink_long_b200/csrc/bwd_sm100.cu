@@ -339,20 +339,26 @@ __global__ void __launch_bounds__(448, 1)
         }
         if (!mbar_wait(&ds_full[bb], use & 1, abort_flag, err, kErrBwdWait)) return false;
         tc_fence_after();
+        // dK and dQ^T are independent accumulations: interleave their k-steps so
+        // the tensor pipe has two chains in flight (one dependent chain of
+        // M=128 MMAs is latency-bound).
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
+        for (int kk = 0; kk < 4; ++kk) {
           tc_mma_ts(tmem + L::T_DK, tb + 96 + 8 * kk, sdesc_sw128(aQ + kk * 2048, 8192, 1024), idesc_g,
                     (m > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) {
+            const int kq = 2 * kk + q2;
+            tc_mma_ss(tb + 32, sdesc_sw128(aK + kq * 2048, 16384, 1024), sdesc_sw128(aDS + kq * 2048, 8192, 1024),
+                      idesc_q, kq > 0 ? 1u : 0u);
+          }
+        }
         if (split) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             tc_mma_ss(tmem + L::T_DK, sdesc_sw128(sbase + L::OFF_DSL + kk * 32, 16, 1024),
                       sdesc_sw128(aQ + kk * 2048, 8192, 1024), idesc_g, 1u);
         }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          tc_mma_ss(tb + 32, sdesc_sw128(aK + kk * 2048, 16384, 1024), sdesc_sw128(aDS + kk * 2048, 8192, 1024),
-                    idesc_q, kk > 0 ? 1u : 0u);
         tc_commit(&dq_full[bb]);
         tc_commit(&dss_free[bb]);
         tc_commit(&q_empty[st]);
@@ -372,20 +378,16 @@ __global__ void __launch_bounds__(448, 1)
         tc_fence_after();
         const uint32_t aQ = sbase + L::OFF_Q + st * L::QB_BYTES;
         const uint32_t aDO = sbase + L::OFF_DO + st * L::QB_BYTES;
+        // S^T and dP^T are independent: interleave their k-steps (two chains in flight).
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ka = (kk >> 2) * 16384 + (kk & 3) * 32;
           const uint32_t kb = (kk >> 2) * 8192 + (kk & 3) * 32;
           tc_mma_ss(tb, sdesc_sw128(aK + ka, 16, 1024), sdesc_sw128(aQ + kb, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&s_full[bb]);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ka = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t kb = (kk >> 2) * 8192 + (kk & 3) * 32;
           tc_mma_ss(tb + 64, sdesc_sw128(aV + ka, 16, 1024), sdesc_sw128(aDO + kb, 16, 1024), idesc_s,
                     kk > 0 ? 1u : 0u);
         }
+        tc_commit(&s_full[bb]);
         tc_commit(&dp_full[bb]);
         if (n >= 1 && !grad(n - 1)) { ok = false; break; }
       }
