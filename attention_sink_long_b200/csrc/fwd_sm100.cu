@@ -52,10 +52,11 @@ struct FwdLayout {
   static constexpr int ALLOC = BYTES + 1024;  // room to align the base to 1024 bytes
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_S = 2 * D;
+  static constexpr int THREADS = 320;
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
     lg_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const FwdParams prm) {
@@ -159,6 +160,15 @@ __global__ void __launch_bounds__(320, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
+      // Operand descriptors are formed once; per MMA only the start-address
+      // field moves (it counts 16-byte units in bits [0, 14), and shared
+      // addresses stay below 2^18, so a plain add never carries out of it).
+      // Keeping the issue path to a few integer adds per MMA matters: one
+      // thread feeds the tensor core, which finishes an M128 N128 K16 MMA in
+      // 64 cycles.
+      const uint64_t dQ0 = sdesc_sw128(sbase + L::OFF_Q, 16, 1024);
+      const uint64_t dK0 = sdesc_sw128(sbase + L::OFF_K, 16, 1024);
+      const uint64_t dV0 = sdesc_sw128(sbase + L::OFF_V, 16384, 1024);
       bool ok = mbar_wait(q_full, 0, abort_flag, err, kErrFwdWait);
       tc_fence_after();
       // S_t(c) = Q_t K(c)^T, N = 64 * nb, into the tile's S columns.
@@ -166,13 +176,14 @@ __global__ void __launch_bounds__(320, 1)
         const int st = c % NS;
         if (t == 0 && !mbar_wait(&k_full[st], (uint32_t)(c / NS) & 1, abort_flag, err, kErrFwdWait)) return false;
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16(128, 64 * nb, false, false);
+        const uint32_t idesc = nb == 2 ? idesc_bf16(128, 128, false, false) : idesc_bf16(128, 64, false, false);
+        const uint64_t a0 = opaque_u64(dQ0 + (uint32_t)((t * L::Q_BYTES) >> 4));
+        const uint64_t b0 = opaque_u64(dK0 + (uint32_t)((st * L::KVC_BYTES) >> 4));
+        const uint32_t d = tmem + L::T_S + 128 * t;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t a = sbase + L::OFF_Q + t * L::Q_BYTES + (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t bb = sbase + L::OFF_K + st * L::KVC_BYTES + (kk >> 2) * 16384 + (kk & 3) * 32;
-          tc_mma_ss(tmem + L::T_S + 128 * t, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 16, 1024), idesc,
-                    kk > 0 ? 1u : 0u);
+          const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+          tc_mma_ss(d, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
         }
         tc_commit(&tile_bars[3 * t + 0]);
         return true;
@@ -183,10 +194,18 @@ __global__ void __launch_bounds__(320, 1)
         if (!mbar_wait(&tile_bars[3 * t + 1], (uint32_t)c & 1, abort_flag, err, kErrFwdWait)) return false;
         if (t == 0 && !mbar_wait(&v_full[st], (uint32_t)(c / NS) & 1, abort_flag, err, kErrFwdWait)) return false;
         tc_fence_after();
-        for (int kk = 0; kk < 4 * nb; ++kk) {
-          const uint32_t bb = sbase + L::OFF_V + st * L::KVC_BYTES + kk * 2048;
-          tc_mma_ts(tmem + (uint32_t)(t * D), tmem + L::T_S + 128 * t + 8 * kk, sdesc_sw128(bb, 16384, 1024),
-                    idesc_pv, (c > 0 || kk > 0) ? 1u : 0u);
+        const uint64_t b0 = opaque_u64(dV0 + (uint32_t)((st * L::KVC_BYTES) >> 4));
+        const uint32_t d = tmem + (uint32_t)(t * D);
+        const uint32_t a = tmem + L::T_S + 128 * t;
+        const uint32_t acc0 = c > 0 ? 1u : 0u;
+        if (nb == 2) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc_mma_ts(d, a + 8 * kk, b0 + (uint32_t)(kk * 2048 >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_ts(d, a + 8 * kk, b0 + (uint32_t)(kk * 2048 >> 4), idesc_pv, kk > 0 ? 1u : acc0);
         }
         tc_commit(&tile_bars[3 * t + 2]);
         return true;
@@ -231,35 +250,40 @@ __global__ void __launch_bounds__(320, 1)
       const int jn = chunks.span(j, &nb);
       if (!__all_sync(0xffffffffu, mbar_wait(s_full, (uint32_t)c & 1, abort_flag, err, kErrFwdWait))) break;
       tc_fence_after();
-      // Pass 1: row max over the chunk, 64 columns at a time straight from TMEM,
-      // masked per 64-column half (blocks outside this row's list, causality
-      // inside the diagonal block). Pass 2 reloads the columns for the
-      // exponentials, which keeps only 64 row values in registers.
+      // One TMEM read of the whole chunk (128 columns, one wait), masked per
+      // 64-column half (blocks outside this row's list, causality inside the
+      // diagonal block); the row max, the exponentials and the packed P then
+      // all come from registers.
       bool vis[2], diag[2];
 #pragma unroll
       for (int hb = 0; hb < 2; ++hb) {
         vis[hb] = hb < nb && row_live && in_list(prm.pat, i, j + hb);
         diag[hb] = (j + hb == i);
       }
-      float mx8[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
+      uint32_t xs[128];
+      tmem_ld128(t_s, xs);
+      // vis and diag are warp-uniform (a warp's rows share a query block). The
+      // register values stay as loaded: masking is applied to the max and to
+      // P, never written back.
+      float mxh[2];
 #pragma unroll
       for (int hb = 0; hb < 2; ++hb) {
-        if (vis[hb]) {  // vis and diag are warp-uniform (a warp's rows share a query block)
-          uint32_t xs[64];
-          tmem_ld64(t_s + 64 * hb, xs);
-          if (diag[hb]) {
+        float m8[8];
 #pragma unroll
-            for (int e = 0; e < 64; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], e > rr ? -INFINITY : __uint_as_float(xs[e]));
-          } else {
+        for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+        if (vis[hb] && !diag[hb]) {
 #pragma unroll
-            for (int e = 0; e < 64; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(xs[e]));
-          }
+          for (int e = 0; e < 64; e += 16)
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              m8[q] = max3f(m8[q], __uint_as_float(xs[64 * hb + e + q]), __uint_as_float(xs[64 * hb + e + 8 + q]));
+        } else if (vis[hb]) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], e > rr ? -INFINITY : __uint_as_float(xs[64 * hb + e]));
         }
+        mxh[hb] = fmaxf(max3f(m8[0], m8[1], m8[2]), fmaxf(max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       }
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float mx = fmaxf(mxh[0], mxh[1]);
       const float m_blk = mx * sl2;
       const bool need = m_blk > m + 8.0f;
       float alpha = 1.f;
@@ -268,32 +292,38 @@ __global__ void __launch_bounds__(320, 1)
         m = m_blk;
       }
       const float m_use = (m == -INFINITY) ? 0.f : m;
-      float rs8[8];
+      // P = 2^(x * scale * log2 e - m), packed to bf16 and written back over the
+      // first half of this tile's S columns (already read). In every group of
+      // eight columns the last pair -- a quarter -- takes the FMA-pipe
+      // polynomial, the rest the special-function unit, so neither pipe alone
+      // sets the pace; scaling, row sums and the polynomial run on paired
+      // fp32 instructions.
+      const float2 sc2 = make_float2(sl2, sl2);
+      const float2 nm2 = make_float2(-m_use, -m_use);
+      float2 rs4[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) rs8[e] = 0.f;
-      // Pass 2: P = 2^(x * scale * log2 e - m), packed to bf16 and written back
-      // over the first half of this tile's S columns. Columns e with
-      // (e & 7) >= 6 -- a quarter -- take the FMA-pipe polynomial, the rest the
-      // special-function unit, so neither pipe alone sets the pace.
+      for (int e = 0; e < 4; ++e) rs4[e] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int hb = 0; hb < 2; ++hb) {
         if (hb < nb) {
           uint32_t pk[32];
-          if (vis[hb]) {
-            uint32_t xs[64];
-            tmem_ld64(t_s + 64 * hb, xs);
-            if (diag[hb]) {
-#pragma unroll
-              for (int e = 0; e < 64; ++e) xs[e] = e > rr ? 0xff800000u : xs[e];  // -inf above the diagonal
-            }
+          if (vis[hb] && !diag[hb]) {
 #pragma unroll
             for (int e = 0; e < 64; e += 2) {
-              const float a0 = fmaf(__uint_as_float(xs[e]), sl2, -m_use);
-              const float a1 = fmaf(__uint_as_float(xs[e + 1]), sl2, -m_use);
-              const float p0 = ((e & 7) >= 6) ? ex2_poly(a0) : ex2_approx(a0);
-              const float p1 = ((e & 7) >= 6) ? ex2_poly(a1) : ex2_approx(a1);
-              rs8[(e >> 1) & 7] += p0 + p1;
-              pk[e >> 1] = pack_bf16x2(p0, p1);
+              const float2 a = fma2(make_float2(__uint_as_float(xs[64 * hb + e]), __uint_as_float(xs[64 * hb + e + 1])),
+                                    sc2, nm2);
+              const float2 pp = ((e & 7) == 6) ? ex2_poly2(a) : make_float2(ex2_approx(a.x), ex2_approx(a.y));
+              rs4[(e >> 1) & 3] = add2(rs4[(e >> 1) & 3], pp);
+              pk[e >> 1] = pack_bf16x2(pp.x, pp.y);
+            }
+          } else if (vis[hb]) {  // the diagonal block: P = 0 above the diagonal
+#pragma unroll
+            for (int e = 0; e < 64; e += 2) {
+              const float2 a = fma2(make_float2(__uint_as_float(xs[64 * hb + e]), __uint_as_float(xs[64 * hb + e + 1])),
+                                    sc2, nm2);
+              const float2 pp = make_float2(e > rr ? 0.f : ex2_approx(a.x), e + 1 > rr ? 0.f : ex2_approx(a.y));
+              rs4[(e >> 1) & 3] = add2(rs4[(e >> 1) & 3], pp);
+              pk[e >> 1] = pack_bf16x2(pp.x, pp.y);
             }
           } else {
 #pragma unroll
@@ -302,8 +332,8 @@ __global__ void __launch_bounds__(320, 1)
           tmem_st32(t_s + 32 * hb, pk);
         }
       }
-      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
-      l = l * alpha + rs;
+      const float2 rs2 = add2(add2(rs4[0], rs4[1]), add2(rs4[2], rs4[3]));
+      l = l * alpha + (rs2.x + rs2.y);
 
       // Lazy rescale of O (warp-uniform: tcgen05.ld/st are warp-collective).
       // PV_t(c-1) completed before S_t(c) did, so O is stable here.
@@ -394,7 +424,7 @@ cudaError_t launch_fwd_impl(const CUtensorMap& tq, const CUtensorMap& tk, const 
   cudaError_t e = cudaFuncSetAttribute(lg_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (e != cudaSuccess) return e;
   dim3 grid(prm.nqt, prm.H, B);
-  lg_fwd_kernel<D><<<grid, 320, L::ALLOC, stream>>>(tq, tk, tv, to, prm);
+  lg_fwd_kernel<D><<<grid, L::THREADS, L::ALLOC, stream>>>(tq, tk, tv, to, prm);
   return cudaGetLastError();
 }
 

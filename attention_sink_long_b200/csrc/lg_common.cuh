@@ -177,6 +177,15 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
+// Returns v unchanged, but opaque to the optimiser: keeps descriptor arithmetic
+// inside the MMA-issue loop instead of hoisting every per-k-step descriptor
+// of every stage into registers for the whole kernel.
+__device__ __forceinline__ uint64_t opaque_u64(uint64_t v) {
+  uint64_t r;
+  asm volatile("mov.b64 %0, %1;" : "=l"(r) : "l"(v));
+  return r;
+}
+
 // kind::f16 instruction descriptor: bf16 A and B, fp32 D, dense.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
@@ -226,6 +235,23 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
       "tcgen05.wait::ld.sync.aligned;\n"
       : LG_R8(0), LG_R8(8), LG_R8(16), LG_R8(24), LG_R8(32), LG_R8(40), LG_R8(48), LG_R8(56)
       : "r"(taddr), "r"(taddr + 32u)
+      : "memory");
+}
+// 128 consecutive columns (four x32 loads, one wait).
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%128];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%129];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
+      "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95}, [%130];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,"
+      "%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%131];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : LG_R8(0), LG_R8(8), LG_R8(16), LG_R8(24), LG_R8(32), LG_R8(40), LG_R8(48), LG_R8(56), LG_R8(64),
+        LG_R8(72), LG_R8(80), LG_R8(88), LG_R8(96), LG_R8(104), LG_R8(112), LG_R8(120)
+      : "r"(taddr), "r"(taddr + 32u), "r"(taddr + 64u), "r"(taddr + 96u)
       : "memory");
 }
 #undef LG_R8
@@ -279,6 +305,47 @@ __device__ __forceinline__ float ex2_poly(float x) {
   p = fmaf(p, f, 0.9999992847442627f);
   const float r = __uint_as_float(__float_as_uint(p) + (__float_as_uint(y) << 23));
   return xc <= -127.0f ? 0.0f : r;
+}
+
+// Paired fp32 arithmetic (one instruction for two lanes' worth of work).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// ex2_poly on a pair, with the range reduction and the Horner steps paired.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  const float2 xc = make_float2(fmaxf(x.x, -127.0f), fmaxf(x.y, -127.0f));
+  const float2 y = add2(xc, make_float2(12582912.0f, 12582912.0f));
+  const float2 n = add2(y, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = add2(xc, make_float2(-n.x, -n.y));
+  float2 p = make_float2(0.009570102207362652f, 0.009570102207362652f);
+  p = fma2(p, f, make_float2(0.05591785907745361f, 0.05591785907745361f));
+  p = fma2(p, f, make_float2(0.240247443318367f, 0.240247443318367f));
+  p = fma2(p, f, make_float2(0.6931217908859253f, 0.6931217908859253f));
+  p = fma2(p, f, make_float2(0.9999992847442627f, 0.9999992847442627f));
+  const float r0 = __uint_as_float(__float_as_uint(p.x) + (__float_as_uint(y.x) << 23));
+  const float r1 = __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(y.y) << 23));
+  return make_float2(xc.x <= -127.0f ? 0.0f : r0, xc.y <= -127.0f ? 0.0f : r1);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -62,13 +62,17 @@ def test_device_exponentials_against_exact():
     xs = torch.cat([xs, torch.tensor([0.0, -0.5, 0.5, -1e-7, 1e-7, -8.0, 8.0])])
     x = xs.cuda()
     exact = torch.exp2(xs.double())
-    for method, bound in ((1, POLY_BOUND), (0, 2.0 ** -21)):
+    ys = {}
+    for method, bound in ((1, POLY_BOUND), (2, POLY_BOUND), (0, 2.0 ** -21)):
         y = torch.empty_like(x)
+        ys[method] = y
         lg.lg_exp2_device(x, y, method)
         torch.cuda.synchronize()
         rel = (y.double().cpu() / exact - 1.0).abs()
         assert rel.max().item() < bound, (method, rel.max().item())
-    for method in (0, 1):
+    # the paired form is the same arithmetic lane by lane
+    assert torch.equal(ys[1], ys[2])
+    for method in (0, 1, 2):
         z = torch.tensor([-float("inf"), -500.0], device="cuda")
         y = torch.empty_like(z)
         lg.lg_exp2_device(z, y, method)
