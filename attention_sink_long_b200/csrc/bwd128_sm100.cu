@@ -1,0 +1,530 @@
+// bwd128_sm100.cu -- LongGen sparse causal attention, training backward for
+// head dim 128 without query-head groups (H == Hkv), on sm_100a.
+//
+// "A Little Goes a Long Way" (LongGen), Abstract insights 1-2 and the
+// atlas.scime.ai summary, "Approach": the sparse layers are trained, so the
+// attention backward runs over the same static block pattern as the forward.
+// Gradients follow from O = softmax(Q K^T * scale) V (FlashAttention-2 style
+// recomputation from the saved row log-sum-exp):
+//   P = exp(S * scale - lse),  dV = P^T dO,  dP = dO V^T,
+//   dS = P o (dP - Delta) with Delta = rowsum(dO o O),
+//   dK = scale * dS^T Q,  dQ = scale * dS K.
+//
+// One CTA owns a 128-row KV tile (two 64-row blocks) of one head and walks
+// the query blocks that see it (QIter) two at a time: a 128-row query step.
+// Every GEMM of a step is then an M = 128, N = 128 tcgen05 MMA -- the shape
+// the tensor core runs at full rate (an N = 64 instruction takes about as
+// long as an N = 128 one):
+//   S^T  = K Q^T       SS, both K-major               -> TMEM region R_s
+//   dP^T = V dO^T      SS, both K-major               -> TMEM region R_d
+//   dV  += P^T dO      TS: P^T (bf16) from TMEM, dO MN-major
+//   dK  += dS^T Q      SS: dS^T (bf16) from shared memory, Q MN-major
+//   dQ^T = K^T dS^T    SS, both MN-major              -> R_d, drained with
+//                      coalesced fp32 reductions into the dQ accumulator.
+// TMEM columns: dV [0,128), dK [128,256), R_s [256,384), R_d [384,512).
+// The P/dS warps read S^T and write P^T (bf16, two per column) over the first
+// half of the columns they read, so no warp overwrites columns another warp
+// still reads. R_d holds dP^T until the warps have read it, then dQ^T.
+//
+// MMA order (one thread; tcgen05 MMAs of one thread execute in order):
+//   S^T(0), dP^T(0), dV(0), S^T(1), then per step n:
+//   [dS(n) ready]  dQ^T(n), dK(n)
+//   [dQ^T(n) drained]  dP^T(n+1)
+//   [P(n+1) ready]  dV(n+1)
+//   [Q(n+2) loaded]  S^T(n+2)        (after dV(n+1), which reads P^T(n+1))
+// so the P/dS warps find S^T of the next step computed while they finish dS,
+// and the tensor pipe has the next GEMMs queued while each wait resolves.
+//
+// Warps: 0-7 P / dS + epilogue (two per TMEM lane quarter: KV rows
+// 32 (w % 4) .. +31, query columns [64 (w / 4), +64) of the step), 8 TMA
+// producer, 9 TMEM owner + MMA issuer, 10-13 dQ drain (one per lane quarter).
+// Shared memory: K, V, two Q / dO stages, dS^T -- seven 32 KB tiles (224 KB)
+// -- plus barriers and the LSE / Delta stages after them.
+#include "lg_common.cuh"
+#include "lg_kernels.h"
+#include "lg_pattern.cuh"
+
+namespace lg {
+
+struct Bwd128Layout {
+  static constexpr int D = 128;
+  static constexpr int QS = 2;                  // Q / dO / LSE / Delta stages
+  static constexpr int TILE = 128 * 128 * 2;    // a 128 x 128 bf16 tile, two 64-column panels
+  static constexpr int PANEL = 128 * 128;       // one 64-column panel of 128 rows (bytes)
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_Q = OFF_V + TILE;          // QS stages
+  static constexpr int OFF_DO = OFF_Q + QS * TILE;    // QS stages
+  static constexpr int OFF_DS = OFF_DO + QS * TILE;   // dS^T, rows = KV, columns = query
+  static constexpr int TILES = OFF_DS + TILE;         // 229376
+  static constexpr int NBAR = 1 + 2 * QS + 8;
+  static constexpr int OFF_BAR = TILES;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_LSE = (OFF_MISC + 16 + 15) / 16 * 16;  // QS x 128 fp32
+  static constexpr int OFF_DEL = OFF_LSE + QS * 512;   // QS x 128 fp32
+  static constexpr int BYTES = OFF_DEL + QS * 512;
+  static constexpr int ALLOC = 232448;                 // the per-block maximum
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t T_DV = 0, T_DK = 128, T_RS = 256, T_RD = 384;
+  static_assert(OFF_LSE % 16 == 0, "bulk copies need 16-byte aligned destinations");
+};
+
+__global__ void __launch_bounds__(448, 1)
+    lg_bwd128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                     const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
+                     const BwdParams prm) {
+  using L = Bwd128Layout;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // The tiles need a 1024-byte aligned base (128-byte swizzle) and the layout
+  // uses nearly the whole per-block allocation, so it only fits when the
+  // dynamic shared memory starts close enough to such a boundary. Checked
+  // uniformly before anything else; a misfit is reported, never run.
+  if ((size_t)(smem - smem_raw) + (size_t)L::BYTES > (size_t)L::ALLOC) {
+    if (threadIdx.x == 0) atomicOr(prm.err, kErrSmemFit);
+    return;
+  }
+  const uint32_t sbase = smem_u32(smem);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* kv_full = bars;
+  uint64_t* q_full = bars + 1;             // [QS] Q, dO, LSE, Delta of a step landed
+  uint64_t* q_empty = bars + 1 + L::QS;    // [QS] the step's stage may be refilled
+  uint64_t* s_full = bars + 1 + 2 * L::QS; // S^T of the next step in R_s
+  uint64_t* dp_full = s_full + 1;          // dP^T in R_d
+  uint64_t* p_full = s_full + 2;           // every P/dS warp wrote its P^T
+  uint64_t* ds_full = s_full + 3;          // dS^T in shared memory, dP^T read
+  uint64_t* dq_full = s_full + 4;          // dQ^T in R_d
+  uint64_t* dq_free = s_full + 5;          // dQ^T read out of R_d
+  uint64_t* dss_free = s_full + 6;         // dQ^T and dK done with the dS^T tile
+  uint64_t* acc_done = s_full + 7;         // every MMA complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+  const float* s_lse = reinterpret_cast<const float*>(smem + L::OFF_LSE);
+  const float* s_del = reinterpret_cast<const float*>(smem + L::OFF_DEL);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // Launch order: first the heavy KV tiles (those a sink or strided block makes
+  // visible to many more queries, listed by the host) of every head, then the
+  // other tiles head by head in ascending order.
+  int u, h;
+  {
+    const int Lx = blockIdx.x;
+    const int nh = prm.n_heavy;
+    if (Lx < nh * prm.Hkv) {
+      u = prm.heavy[Lx / prm.Hkv];
+      h = Lx % prm.Hkv;
+    } else {
+      const int rest = prm.nkt - nh;
+      const int L2 = Lx - nh * prm.Hkv;
+      h = L2 / rest;
+      u = L2 % rest;
+      for (int k = 0; k < nh; ++k) u += (prm.heavy[k] <= u) ? 1 : 0;  // skip the heavy tiles
+    }
+  }
+  const int b = blockIdx.y;
+  const QIter qit(prm.pat, 2 * u, imin(2 * u + 1, prm.nqb - 1), prm.nqb);
+  const int last = qit.last_blk;         // query blocks [first_blk, last] see this KV tile
+  const int N = (qit.count() + 1) / 2;   // 128-row query steps (the last one may hold one block)
+  unsigned int* err = prm.err;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < L::QS; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1 + 256);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, 256);
+    mbar_init(ds_full, 256);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, 128);
+    mbar_init(dss_free, 1);
+    mbar_init(acc_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
+      for (int p = 0; p < 2; ++p) {
+        tma_load_4d(smem + L::OFF_K + p * L::PANEL, &tmK, kv_full, 64 * p, h, 128 * u, b);
+        tma_load_4d(smem + L::OFF_V + p * L::PANEL, &tmV, kv_full, 64 * p, h, 128 * u, b);
+      }
+      int issued = 0;
+      for (int n = 0; n < N; ++n) {
+        const int st = n & 1;
+        const uint32_t use = (uint32_t)(n >> 1);
+        if (use > 0 && !mbar_wait(&q_empty[st], (use - 1) & 1, abort_flag, err, kErrBwdWait)) break;
+        const int i0 = qit.first_blk + 2 * n;
+        // Both 64-row halves always load (rows past the sequence arrive as
+        // zeros), so the stage never holds stale operands; LSE / Delta only
+        // exist for blocks inside the sequence.
+        const int nl = (i0 + 1 < prm.nqb) ? 2 : 1;
+        mbar_arrive_expect_tx(&q_full[st], 2 * L::TILE + nl * 512);
+        for (int hb = 0; hb < 2; ++hb)
+          for (int p = 0; p < 2; ++p) {
+            const int off = st * L::TILE + p * L::PANEL + hb * 8192;
+            tma_load_4d(smem + L::OFF_Q + off, &tmQ, &q_full[st], 64 * p, h, 64 * (i0 + hb), b);
+            tma_load_4d(smem + L::OFF_DO + off, &tmdO, &q_full[st], 64 * p, h, 64 * (i0 + hb), b);
+          }
+        for (int hb = 0; hb < nl; ++hb) {
+          const size_t row = ((size_t)b * prm.H + h) * prm.S + 64 * (size_t)(i0 + hb);
+          bulk_load(smem + L::OFF_LSE + st * 512 + hb * 256, prm.lse + row, 256, &q_full[st]);
+          bulk_load(smem + L::OFF_DEL + st * 512 + hb * 256, prm.delta + row, 256, &q_full[st]);
+        }
+        issued = n + 1;
+      }
+      if (*abort_flag) {
+        // Let copies already in flight land before the CTA's shared memory goes away.
+        const long long t0 = clock64();
+        while (!mbar_try_wait(kv_full, 0) && clock64() - t0 < 20000000LL) {
+        }
+        for (int s = 0; s < L::QS && s < issued; ++s) {
+          const int lastn = issued - 1 - ((issued - 1 - s) & 1);
+          const long long t1 = clock64();
+          while (!mbar_try_wait(&q_full[s], (uint32_t)(lastn >> 1) & 1) && clock64() - t1 < 20000000LL) {
+          }
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_kk = idesc_bf16(128, 128, false, false);   // S^T, dP^T
+      constexpr uint32_t idesc_kmn = idesc_bf16(128, 128, false, true);   // dV (A in TMEM), dK
+      constexpr uint32_t idesc_mnmn = idesc_bf16(128, 128, true, true);   // dQ^T
+      // Descriptor bases (the start field moves by 16-byte units per k-step).
+      // K-major operands advance 32 bytes per k-step inside a 64-column panel
+      // and jump a panel every four; MN-major ones advance 16 rows (2048 bytes)
+      // and reach their second 64-element half through the leading offset.
+      const uint64_t dK_k = sdesc_sw128(sbase + L::OFF_K, 16, 1024);
+      const uint64_t dV_k = sdesc_sw128(sbase + L::OFF_V, 16, 1024);
+      const uint64_t dK_mn = sdesc_sw128(sbase + L::OFF_K, L::PANEL, 1024);
+      const uint64_t dS_k = sdesc_sw128(sbase + L::OFF_DS, 16, 1024);
+      const uint64_t dS_mn = sdesc_sw128(sbase + L::OFF_DS, L::PANEL, 1024);
+      auto kofs = [](int kk) -> uint32_t { return (uint32_t)(((kk >> 2) * L::PANEL + (kk & 3) * 32) >> 4); };
+      auto mofs = [](int kk) -> uint32_t { return (uint32_t)((kk * 2048) >> 4); };
+      auto q_k = [&](int n) { return opaque_u64(sdesc_sw128(sbase + L::OFF_Q + (n & 1) * L::TILE, 16, 1024)); };
+      auto o_k = [&](int n) { return opaque_u64(sdesc_sw128(sbase + L::OFF_DO + (n & 1) * L::TILE, 16, 1024)); };
+      auto q_mn = [&](int n) {
+        return opaque_u64(sdesc_sw128(sbase + L::OFF_Q + (n & 1) * L::TILE, L::PANEL, 1024));
+      };
+      auto o_mn = [&](int n) {
+        return opaque_u64(sdesc_sw128(sbase + L::OFF_DO + (n & 1) * L::TILE, L::PANEL, 1024));
+      };
+      // S^T(n) = K Q(n)^T into R_s.
+      auto issue_s = [&](int n) {
+        const uint64_t q = q_k(n);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_ss(tmem + L::T_RS, dK_k + kofs(kk), q + kofs(kk), idesc_kk, kk > 0 ? 1u : 0u);
+      };
+      // dP^T(n) = V dO(n)^T into R_d.
+      auto issue_dp = [&](int n) {
+        const uint64_t o = o_k(n);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_ss(tmem + L::T_RD, dV_k + kofs(kk), o + kofs(kk), idesc_kk, kk > 0 ? 1u : 0u);
+      };
+      // dV += P^T(n) dO(n); P^T of query columns [64 hf, +64) sits in R_s
+      // columns [64 hf, +32), two bf16 per column.
+      auto issue_dv = [&](int n) {
+        const uint64_t o = o_mn(n);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_ts(tmem + L::T_DV, tmem + L::T_RS + 64 * (kk >> 2) + 8 * (kk & 3), o + mofs(kk), idesc_kmn,
+                    (n > 0 || kk > 0) ? 1u : 0u);
+      };
+      // dQ^T(n) = K^T dS^T(n) into R_d (fresh each step), then dK += dS^T(n) Q(n).
+      auto issue_dq_dk = [&](int n) {
+        const uint64_t q = q_mn(n);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_ss(tmem + L::T_RD, dK_mn + mofs(kk), dS_mn + mofs(kk), idesc_mnmn, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_ss(tmem + L::T_DK, dS_k + kofs(kk), q + mofs(kk), idesc_kmn, (n > 0 || kk > 0) ? 1u : 0u);
+      };
+
+      bool ok = mbar_wait(kv_full, 0, abort_flag, err, kErrBwdWait) &&
+                mbar_wait(&q_full[0], 0, abort_flag, err, kErrBwdWait);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        tc_commit(s_full);
+        issue_dp(0);
+        tc_commit(dp_full);
+        ok = mbar_wait(p_full, 0, abort_flag, err, kErrBwdWait);
+      }
+      if (ok) {
+        tc_fence_after();
+        issue_dv(0);
+        if (N > 1) {
+          ok = mbar_wait(&q_full[1], 0, abort_flag, err, kErrBwdWait);
+          if (ok) {
+            tc_fence_after();
+            issue_s(1);
+            tc_commit(s_full);
+          }
+        }
+      }
+      for (int n = 0; n < N && ok; ++n) {
+        const uint32_t par = (uint32_t)n & 1;
+        if (!mbar_wait(ds_full, par, abort_flag, err, kErrBwdWait)) break;
+        tc_fence_after();
+        issue_dq_dk(n);
+        tc_commit(dq_full);
+        tc_commit(dss_free);
+        tc_commit(&q_empty[n & 1]);
+        if (n + 1 < N) {
+          // R_d takes dP^T(n+1) once the drain warps have read dQ^T(n).
+          if (!mbar_wait(dq_free, par, abort_flag, err, kErrBwdWait)) break;
+          tc_fence_after();
+          issue_dp(n + 1);
+          tc_commit(dp_full);
+          if (!mbar_wait(p_full, par ^ 1u, abort_flag, err, kErrBwdWait)) break;
+          tc_fence_after();
+          issue_dv(n + 1);
+          if (n + 2 < N) {
+            // S^T(n+2) overwrites P^T(n+1), which dV(n+1) -- issued just before --
+            // reads first; its Q stage was refilled after dK(n) completed.
+            if (!mbar_wait(&q_full[n & 1], (uint32_t)((n + 2) >> 1) & 1, abort_flag, err, kErrBwdWait)) break;
+            tc_fence_after();
+            issue_s(n + 2);
+            tc_commit(s_full);
+          }
+        }
+      }
+      tc_commit(acc_done);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ P / dS warps
+    // Warp w owns KV rows 32 (w % 4) .. +31 (its TMEM lane quarter) and query
+    // columns [64 hf, +64) of each step, hf = w / 4 -- one 64 x 64 block pair,
+    // so visibility and the diagonal mask are warp-uniform.
+    const int hf = warp >> 2;
+    const int c0 = 64 * hf;
+    const int r = (warp & 3) * 32 + lane;  // KV row of the tile == TMEM lane
+    const int kvb = 2 * u + (r >> 6);
+    const int rr = r & 63;
+    const bool krow_live = kvb < prm.nqb;
+    const uint32_t t_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const float sl2 = prm.scale_log2;
+    constexpr float kLog2e = 1.4426950408889634f;
+    int n = 0;
+    for (; n < N; ++n) {
+      const int st = n & 1;
+      const uint32_t par = (uint32_t)n & 1;
+      const int i = qit.first_blk + 2 * n + hf;  // this warp's query block
+      const bool vis = krow_live && i <= last && in_list(prm.pat, i, kvb);
+      const bool diag = (i == kvb);
+      if (!__all_sync(0xffffffffu, mbar_wait(&q_full[st], (uint32_t)(n >> 1) & 1, abort_flag, err, kErrBwdWait)))
+        break;
+      if (!__all_sync(0xffffffffu, mbar_wait(s_full, par, abort_flag, err, kErrBwdWait))) break;
+      tc_fence_after();
+      // P^T = exp2(S^T * scale * log2 e - lse * log2 e), 32 columns at a time; the
+      // bf16 pairs go back over the first 32 of this warp's 64 S^T columns
+      // (already read), fp32 copies stay for dS.
+      float pf[64];
+      // LSE and Delta are the same for every thread of the warp: 16-byte
+      // broadcast loads, four columns each.
+      const float4* lse4 = reinterpret_cast<const float4*>(s_lse + st * 128 + c0);
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t sr[32];
+        tmem_ld32(t_lane + L::T_RS + c0 + 32 * ch, sr);
+        if (vis) {
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            const float4 l4 = lse4[8 * ch + g];
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+            for (int e = 4 * g; e < 4 * g + 4; ++e) {
+              const float p = ex2_approx(fmaf(__uint_as_float(sr[e]), sl2, -lv[e - 4 * g] * kLog2e));
+              pf[32 * ch + e] = (diag && 32 * ch + e < rr) ? 0.f : p;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) pf[32 * ch + e] = 0.f;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pf[32 * ch + 2 * e], pf[32 * ch + 2 * e + 1]);
+        tmem_st16(t_lane + L::T_RS + c0 + 16 * ch, pk);
+      }
+      tc_fence_before();
+      mbar_arrive(p_full);
+      if (!__all_sync(0xffffffffu, mbar_wait(dp_full, par, abort_flag, err, kErrBwdWait))) break;
+      // The dS^T tile last fed dQ^T(n-1) and dK(n-1).
+      if (n >= 1 && !__all_sync(0xffffffffu, mbar_wait(dss_free, par ^ 1u, abort_flag, err, kErrBwdWait))) break;
+      tc_fence_after();
+      // dS^T = P^T o (dP^T - Delta), bf16 into the swizzled dS^T tile (rows =
+      // KV, query panel hf). Blocks this row does not see give exact zeros.
+      const float4* del4 = reinterpret_cast<const float4*>(s_del + st * 128 + c0);
+      const uint32_t drow = sbase + L::OFF_DS + hf * L::PANEL;
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t dpr[32];
+        tmem_ld32(t_lane + L::T_RD + c0 + 32 * ch, dpr);
+        // eight columns (one 16-byte chunk of the row) at a time
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[4];
+          if (vis) {
+            const float4 da = del4[8 * ch + 2 * c], db = del4[8 * ch + 2 * c + 1];
+            const float dl[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int k = 32 * ch + 8 * c + 2 * e;
+              const float d0 = pf[k] * (__uint_as_float(dpr[8 * c + 2 * e]) - dl[2 * e]);
+              const float d1 = pf[k + 1] * (__uint_as_float(dpr[8 * c + 2 * e + 1]) - dl[2 * e + 1]);
+              pk[e] = pack_bf16x2(d0, d1);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) pk[e] = 0u;
+          }
+          st_shared_v4(drow + sw128_offset(r, 4 * ch + c), pk[0], pk[1], pk[2], pk[3]);
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+      mbar_arrive(&q_empty[st]);
+    }
+
+    // ------------------------------------------------------------ dK, dV epilogue
+    // Warp (quarter, half) writes rows of its quarter, columns [64 half, +64).
+    bool ok = (n == N) && !*abort_flag;
+    if (ok) ok = mbar_wait(acc_done, 0, abort_flag, err, kErrBwdWait);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok && prm.grad_f32) {
+      // fp32 gradients: each thread stores its part of a KV row straight from TMEM.
+      tc_fence_after();
+      const int krow = 128 * u + r;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tcol = which == 0 ? L::T_DV : L::T_DK;
+        const float mul = which == 0 ? 1.f : prm.scale;
+        float* dst = (which == 0 ? prm.dv_f32 : prm.dk_f32) + (((size_t)b * prm.S + krow) * prm.Hkv + h) * L::D;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int col = c0 + 32 * q;
+          uint32_t o[32];
+          tmem_ld32(t_lane + tcol + col, o);
+          if (krow < prm.S) {
+            float4* d4 = reinterpret_cast<float4*>(dst + col);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              d4[e] = make_float4(__uint_as_float(o[4 * e]) * mul, __uint_as_float(o[4 * e + 1]) * mul,
+                                  __uint_as_float(o[4 * e + 2]) * mul, __uint_as_float(o[4 * e + 3]) * mul);
+          }
+        }
+      }
+    } else if (ok) {
+      // bf16 gradients: stage in the K / V tiles (every MMA is done with them),
+      // then one TMA store per panel.
+      tc_fence_after();
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tcol = which == 0 ? L::T_DV : L::T_DK;
+        const float mul = which == 0 ? 1.f : prm.scale;
+        const uint32_t panel = sbase + (which == 0 ? L::OFF_V : L::OFF_K) + (uint32_t)hf * L::PANEL;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t o[32];
+          tmem_ld32(t_lane + tcol + c0 + 32 * q, o);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const float* f = reinterpret_cast<const float*>(&o[8 * q4]);
+            st_shared_v4(panel + sw128_offset(r, 4 * q + q4), pack_bf16x2(f[0] * mul, f[1] * mul),
+                         pack_bf16x2(f[2] * mul, f[3] * mul), pack_bf16x2(f[4] * mul, f[5] * mul),
+                         pack_bf16x2(f[6] * mul, f[7] * mul));
+          }
+        }
+      }
+    }
+    fence_async_smem();
+    named_bar_sync(1, 256);
+    if (threadIdx.x == 0 && ok && !prm.grad_f32) {
+      for (int p = 0; p < 2; ++p) {
+        tma_store_4d(&tmdV, smem + L::OFF_V + p * L::PANEL, 64 * p, h, 128 * u, b);
+        tma_store_4d(&tmdK, smem + L::OFF_K + p * L::PANEL, 64 * p, h, 128 * u, b);
+      }
+      bulk_commit();
+      bulk_wait_all();
+    }
+  } else {
+    // ------------------------------------------------------------ dQ drain warps 10-13
+    // Thread = dQ^T row d (TMEM lane); a warp's 32 lanes hit 32 consecutive dQ
+    // elements of one query row, so every reduction below is one coalesced
+    // 128-byte request.
+    const int quarter = warp & 3;
+    const int d = quarter * 32 + lane;
+    const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
+    for (int n = 0; n < N; ++n) {
+      const int i0 = qit.first_blk + 2 * n;
+      const bool second = i0 + 1 <= last;  // the step's second query block is in the list range
+      if (!__all_sync(0xffffffffu, mbar_wait(dq_full, (uint32_t)n & 1, abort_flag, err, kErrBwdWait))) break;
+      tc_fence_after();
+      float* dst = prm.dq_acc + (((size_t)b * prm.H + h) * prm.S + 64 * (size_t)i0) * L::D + d;
+      // Read all 128 columns first, so R_d is released before any reduction is
+      // issued (the reductions run at the L2's rate and would otherwise hold
+      // up the next dP^T).
+      uint32_t va[64], vb[64];
+      tmem_ld64(t_lane + L::T_RD, va);
+      tmem_ld64(t_lane + L::T_RD + 64, vb);
+      tc_fence_before();
+      mbar_arrive(dq_free);
+      // Loads before reductions: the Q / dO copies of step n+2 (issued once
+      // dK(n) freed their stage) go through L2 first, then this step's
+      // reductions, so the next S^T is not starved by them.
+      if (n + 2 < N &&
+          !__all_sync(0xffffffffu, mbar_wait(&q_full[n & 1], (uint32_t)((n + 2) >> 1) & 1, abort_flag, err,
+                                             kErrBwdWait)))
+        break;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) red_add_f32(dst + (size_t)c * L::D, __uint_as_float(va[c]));
+      if (second) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) red_add_f32(dst + (size_t)(64 + c) * L::D, __uint_as_float(vb[c]));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+cudaError_t launch_bwd128(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+                          const CUtensorMap& tdk, const CUtensorMap& tdv, const BwdParams& prm, int B,
+                          cudaStream_t stream) {
+  using L = Bwd128Layout;
+  static_assert(L::BYTES <= L::ALLOC, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(lg_bwd128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+  if (e != cudaSuccess) return e;
+  dim3 grid(prm.nkt * prm.Hkv, B);
+  lg_bwd128_kernel<<<grid, 448, L::ALLOC, stream>>>(tq, tk, tv, tdo, tdk, tdv, prm);
+  return cudaGetLastError();
+}
+
+}  // namespace lg

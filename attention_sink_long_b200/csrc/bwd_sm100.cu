@@ -188,9 +188,6 @@ struct BwdLayout {
   static constexpr uint32_t T_DV = 0, T_DK = D, T_BUF = 2 * D;
 };
 
-__device__ __forceinline__ void red_add_f32(float* p, float v) {
-  asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
-}
 
 template <int D, bool SPLIT>
 __global__ void __launch_bounds__(448, 1)
@@ -622,6 +619,7 @@ static cudaError_t launch_bwd_impl(const CUtensorMap& tq, const CUtensorMap& tk,
 cudaError_t launch_bwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv, const BwdParams& prm,
                        int B, cudaStream_t stream) {
+  if (D == 128 && !prm.split_lo) return launch_bwd128(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
   if (prm.split_lo) {
     if (D == 64) return launch_bwd_impl<64, true>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
     return launch_bwd_impl<128, true>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);

@@ -17,7 +17,7 @@
 namespace lg {
 
 // Device error flags (see lg_device_status).
-enum : uint32_t { kErrFwdWait = 1u, kErrBwdWait = 2u, kErrDecode = 4u };
+enum : uint32_t { kErrFwdWait = 1u, kErrBwdWait = 2u, kErrDecode = 4u, kErrSmemFit = 8u };
 
 // A bounded wait gives up after this many SM clock cycles (about 2 s at 1.9 GHz).
 constexpr long long kWaitLimitCycles = 4000000000LL;
@@ -276,6 +276,12 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 #undef LG_W8
+
+// Fire-and-forget fp32 add into global memory (a warp's 32 consecutive
+// addresses coalesce into one reduction request).
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+  asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
 
 // ---------------------------------------------------------------------------
 // Small math helpers (hardware approximations; no library constants)

@@ -47,6 +47,10 @@ cudaError_t launch_bwd_pre(const void* o, int o_f32, const void* dout, float* de
 cudaError_t launch_bwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv, const BwdParams& prm,
                        int B, cudaStream_t stream);
+// Head dim 128, H == Hkv: 128-row query steps, every MMA M = N = 128.
+cudaError_t launch_bwd128(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+                          const CUtensorMap& tdk, const CUtensorMap& tdv, const BwdParams& prm, int B,
+                          cudaStream_t stream);
 cudaError_t launch_bwd_dq(const float* dq_acc, void* dq, int dq_f32, float scale, int B, int S, int H, int D,
                           cudaStream_t stream);
 

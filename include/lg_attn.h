@@ -269,8 +269,10 @@ lg_status_t lg_exp2_device(const float* x, float* y, int64_t n, int32_t method, 
 
 /*
  * Reads and clears the device-side error flags of the given device (bit 0:
- * a forward wait ran out, bit 1: a backward wait ran out, bit 2: decode).
- * SYNCHRONISES that device. *flags == 0 means no bounded wait ran out.
+ * a forward wait ran out, bit 1: a backward wait ran out, bit 2: decode,
+ * bit 3: a kernel found its shared-memory layout would not fit the block's
+ * allocation and did no work). SYNCHRONISES that device. *flags == 0 means
+ * every kernel since the last call ran to completion.
  */
 lg_status_t lg_device_status(int32_t device, uint32_t* flags);
 

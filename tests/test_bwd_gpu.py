@@ -68,6 +68,8 @@ SMALL = [
     (1, 64, 1, 1, 128, lg.Pattern(64, 1, 1, 0), torch.float32),     # a single block
     (1, 2048, 2, 2, 128, lg.Pattern(64, 1, 16, 4), torch.float32),
     (1, 1280, 2, 2, 128, lg.Pattern(64, 0, 1, 0), torch.float32),   # diagonal only
+    (2, 640, 2, 2, 128, lg.Pattern.full(64), torch.float32),        # dense causal, odd 128-row step count
+    (1, 1024, 2, 2, 128, lg.Pattern(64, 1, 4, 0), torch.bfloat16),  # attention sink at head dim 128, bf16 O
 ]
 
 
