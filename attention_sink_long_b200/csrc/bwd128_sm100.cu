@@ -491,15 +491,15 @@ __global__ void __launch_bounds__(448, 1)
       tmem_ld64(t_lane + L::T_RD + 64, vb);
       tc_fence_before();
       mbar_arrive(dq_free);
-      // Loads before reductions: the Q / dO copies of step n+2 (issued once
-      // dK(n) freed their stage) go through L2 first, then this step's
-      // reductions, so the next S^T is not starved by them.
+#pragma unroll
+      for (int c = 0; c < 64; ++c) red_add_f32(dst + (size_t)c * L::D, __uint_as_float(va[c]));
+      // Loads before the second half of the reductions: the Q / dO copies of
+      // step n+2 (issued once dK(n) freed their stage) go through L2 first, so
+      // the next S^T is not starved by this step's reductions.
       if (n + 2 < N &&
           !__all_sync(0xffffffffu, mbar_wait(&q_full[n & 1], (uint32_t)((n + 2) >> 1) & 1, abort_flag, err,
                                              kErrBwdWait)))
         break;
-#pragma unroll
-      for (int c = 0; c < 64; ++c) red_add_f32(dst + (size_t)c * L::D, __uint_as_float(va[c]));
       if (second) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) red_add_f32(dst + (size_t)(64 + c) * L::D, __uint_as_float(vb[c]));
