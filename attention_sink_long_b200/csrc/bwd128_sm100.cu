@@ -28,9 +28,9 @@
 //
 // MMA order (one thread; tcgen05 MMAs of one thread execute in order):
 //   S^T(0), dP^T(0), dV(0), S^T(1), then per step n:
-//   [dS(n) ready]  dQ^T(n), dK(n)
+//   [dS(n) ready]  dK(n), dQ^T(n)    (dK first: Q(n)'s stage refills sooner)
 //   [dQ^T(n) drained]  dP^T(n+1)
-//   [P(n+1) ready]  dV(n+1)
+//   [P(n+1) ready]  dV(n+1)          (dO(n+1)'s stage refills after it)
 //   [Q(n+2) loaded]  S^T(n+2)        (after dV(n+1), which reads P^T(n+1))
 // so the P/dS warps find S^T of the next step computed while they finish dS,
 // and the tensor pipe has the next GEMMs queued while each wait resolves.
@@ -57,7 +57,7 @@ struct Bwd128Layout {
   static constexpr int OFF_DO = OFF_Q + QS * TILE;    // QS stages
   static constexpr int OFF_DS = OFF_DO + QS * TILE;   // dS^T, rows = KV, columns = query
   static constexpr int TILES = OFF_DS + TILE;         // 229376
-  static constexpr int NBAR = 1 + 2 * QS + 8;
+  static constexpr int NBAR = 1 + 4 * QS + 8;
   static constexpr int OFF_BAR = TILES;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_LSE = (OFF_MISC + 16 + 15) / 16 * 16;  // QS x 128 fp32
@@ -89,9 +89,13 @@ __global__ void __launch_bounds__(448, 1)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* kv_full = bars;
-  uint64_t* q_full = bars + 1;             // [QS] Q, dO, LSE, Delta of a step landed
-  uint64_t* q_empty = bars + 1 + L::QS;    // [QS] the step's stage may be refilled
-  uint64_t* s_full = bars + 1 + 2 * L::QS; // S^T of the next step in R_s
+  // Q (+ LSE) and dO (+ Delta) stage separately: dO is done with after
+  // dV, Q only after dK, so each refill starts as soon as its own tile frees.
+  uint64_t* qq_full = bars + 1;               // [QS] Q and LSE of a step landed
+  uint64_t* qq_empty = bars + 1 + L::QS;      // [QS] ... may be refilled
+  uint64_t* qo_full = bars + 1 + 2 * L::QS;   // [QS] dO and Delta of a step landed
+  uint64_t* qo_empty = bars + 1 + 3 * L::QS;  // [QS] ... may be refilled
+  uint64_t* s_full = bars + 1 + 4 * L::QS;    // S^T of the next step in R_s
   uint64_t* dp_full = s_full + 1;          // dP^T in R_d
   uint64_t* p_full = s_full + 2;           // every P/dS warp wrote its P^T
   uint64_t* ds_full = s_full + 3;          // dS^T in shared memory, dP^T read
@@ -133,8 +137,10 @@ __global__ void __launch_bounds__(448, 1)
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     for (int s = 0; s < L::QS; ++s) {
-      mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 1 + 256);
+      mbar_init(&qq_full[s], 1);
+      mbar_init(&qq_empty[s], 1 + 256);
+      mbar_init(&qo_full[s], 1);
+      mbar_init(&qo_empty[s], 1 + 256);
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
@@ -164,39 +170,51 @@ __global__ void __launch_bounds__(448, 1)
         tma_load_4d(smem + L::OFF_K + p * L::PANEL, &tmK, kv_full, 64 * p, h, 128 * u, b);
         tma_load_4d(smem + L::OFF_V + p * L::PANEL, &tmV, kv_full, 64 * p, h, 128 * u, b);
       }
-      int issued = 0;
+      int issued_o = 0, issued_q = 0;  // steps whose dO / Q copies were issued
       for (int n = 0; n < N; ++n) {
         const int st = n & 1;
         const uint32_t use = (uint32_t)(n >> 1);
-        if (use > 0 && !mbar_wait(&q_empty[st], (use - 1) & 1, abort_flag, err, kErrBwdWait)) break;
         const int i0 = qit.first_blk + 2 * n;
         // Both 64-row halves always load (rows past the sequence arrive as
-        // zeros), so the stage never holds stale operands; LSE / Delta only
+        // zeros), so a stage never holds stale operands; LSE / Delta only
         // exist for blocks inside the sequence.
         const int nl = (i0 + 1 < prm.nqb) ? 2 : 1;
-        mbar_arrive_expect_tx(&q_full[st], 2 * L::TILE + nl * 512);
+        if (use > 0 && !mbar_wait(&qo_empty[st], (use - 1) & 1, abort_flag, err, kErrBwdWait)) break;
+        mbar_arrive_expect_tx(&qo_full[st], L::TILE + nl * 256);
+        issued_o = n + 1;
         for (int hb = 0; hb < 2; ++hb)
-          for (int p = 0; p < 2; ++p) {
-            const int off = st * L::TILE + p * L::PANEL + hb * 8192;
-            tma_load_4d(smem + L::OFF_Q + off, &tmQ, &q_full[st], 64 * p, h, 64 * (i0 + hb), b);
-            tma_load_4d(smem + L::OFF_DO + off, &tmdO, &q_full[st], 64 * p, h, 64 * (i0 + hb), b);
-          }
+          for (int p = 0; p < 2; ++p)
+            tma_load_4d(smem + L::OFF_DO + st * L::TILE + p * L::PANEL + hb * 8192, &tmdO, &qo_full[st], 64 * p, h,
+                        64 * (i0 + hb), b);
         for (int hb = 0; hb < nl; ++hb) {
           const size_t row = ((size_t)b * prm.H + h) * prm.S + 64 * (size_t)(i0 + hb);
-          bulk_load(smem + L::OFF_LSE + st * 512 + hb * 256, prm.lse + row, 256, &q_full[st]);
-          bulk_load(smem + L::OFF_DEL + st * 512 + hb * 256, prm.delta + row, 256, &q_full[st]);
+          bulk_load(smem + L::OFF_DEL + st * 512 + hb * 256, prm.delta + row, 256, &qo_full[st]);
         }
-        issued = n + 1;
+        if (use > 0 && !mbar_wait(&qq_empty[st], (use - 1) & 1, abort_flag, err, kErrBwdWait)) break;
+        mbar_arrive_expect_tx(&qq_full[st], L::TILE + nl * 256);
+        issued_q = n + 1;
+        for (int hb = 0; hb < 2; ++hb)
+          for (int p = 0; p < 2; ++p)
+            tma_load_4d(smem + L::OFF_Q + st * L::TILE + p * L::PANEL + hb * 8192, &tmQ, &qq_full[st], 64 * p, h,
+                        64 * (i0 + hb), b);
+        for (int hb = 0; hb < nl; ++hb) {
+          const size_t row = ((size_t)b * prm.H + h) * prm.S + 64 * (size_t)(i0 + hb);
+          bulk_load(smem + L::OFF_LSE + st * 512 + hb * 256, prm.lse + row, 256, &qq_full[st]);
+        }
       }
       if (*abort_flag) {
         // Let copies already in flight land before the CTA's shared memory goes away.
         const long long t0 = clock64();
         while (!mbar_try_wait(kv_full, 0) && clock64() - t0 < 20000000LL) {
         }
-        for (int s = 0; s < L::QS && s < issued; ++s) {
-          const int lastn = issued - 1 - ((issued - 1 - s) & 1);
+        for (int s = 0; s < 2 * L::QS; ++s) {
+          const int issued = s < L::QS ? issued_o : issued_q;
+          const int stg = s % L::QS;
+          if (stg >= issued) continue;
+          const int lastn = issued - 1 - ((issued - 1 - stg) & 1);
+          uint64_t* bar = s < L::QS ? &qo_full[stg] : &qq_full[stg];
           const long long t1 = clock64();
-          while (!mbar_try_wait(&q_full[s], (uint32_t)(lastn >> 1) & 1) && clock64() - t1 < 20000000LL) {
+          while (!mbar_try_wait(bar, (uint32_t)(lastn >> 1) & 1) && clock64() - t1 < 20000000LL) {
           }
         }
       }
@@ -249,23 +267,31 @@ __global__ void __launch_bounds__(448, 1)
           tc_mma_ts(tmem + L::T_DV, tmem + L::T_RS + 64 * (kk >> 2) + 8 * (kk & 3), o + mofs(kk), idesc_kmn,
                     (n > 0 || kk > 0) ? 1u : 0u);
       };
-      // dQ^T(n) = K^T dS^T(n) into R_d (fresh each step), then dK += dS^T(n) Q(n).
-      auto issue_dq_dk = [&](int n) {
+      // dK += dS^T(n) Q(n).
+      auto issue_dk = [&](int n) {
         const uint64_t q = q_mn(n);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          tc_mma_ss(tmem + L::T_RD, dK_mn + mofs(kk), dS_mn + mofs(kk), idesc_mnmn, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           tc_mma_ss(tmem + L::T_DK, dS_k + kofs(kk), q + mofs(kk), idesc_kmn, (n > 0 || kk > 0) ? 1u : 0u);
       };
+      // dQ^T(n) = K^T dS^T(n) into R_d (fresh each step).
+      auto issue_dq = [&](int n) {
+        (void)n;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_ss(tmem + L::T_RD, dK_mn + mofs(kk), dS_mn + mofs(kk), idesc_mnmn, kk > 0 ? 1u : 0u);
+      };
 
       bool ok = mbar_wait(kv_full, 0, abort_flag, err, kErrBwdWait) &&
-                mbar_wait(&q_full[0], 0, abort_flag, err, kErrBwdWait);
+                mbar_wait(&qq_full[0], 0, abort_flag, err, kErrBwdWait);
       if (ok) {
         tc_fence_after();
         issue_s(0);
         tc_commit(s_full);
+        ok = mbar_wait(&qo_full[0], 0, abort_flag, err, kErrBwdWait);
+      }
+      if (ok) {
+        tc_fence_after();
         issue_dp(0);
         tc_commit(dp_full);
         ok = mbar_wait(p_full, 0, abort_flag, err, kErrBwdWait);
@@ -273,8 +299,9 @@ __global__ void __launch_bounds__(448, 1)
       if (ok) {
         tc_fence_after();
         issue_dv(0);
+        tc_commit(&qo_empty[0]);
         if (N > 1) {
-          ok = mbar_wait(&q_full[1], 0, abort_flag, err, kErrBwdWait);
+          ok = mbar_wait(&qq_full[1], 0, abort_flag, err, kErrBwdWait);
           if (ok) {
             tc_fence_after();
             issue_s(1);
@@ -286,23 +313,28 @@ __global__ void __launch_bounds__(448, 1)
         const uint32_t par = (uint32_t)n & 1;
         if (!mbar_wait(ds_full, par, abort_flag, err, kErrBwdWait)) break;
         tc_fence_after();
-        issue_dq_dk(n);
+        // dK first: it is Q(n)'s last use, so the refill of that stage with
+        // Q(n+2) -- which S^T(n+2) waits for -- starts one GEMM earlier.
+        issue_dk(n);
+        tc_commit(&qq_empty[n & 1]);
+        issue_dq(n);
         tc_commit(dq_full);
         tc_commit(dss_free);
-        tc_commit(&q_empty[n & 1]);
         if (n + 1 < N) {
           // R_d takes dP^T(n+1) once the drain warps have read dQ^T(n).
           if (!mbar_wait(dq_free, par, abort_flag, err, kErrBwdWait)) break;
+          if (!mbar_wait(&qo_full[(n + 1) & 1], (uint32_t)((n + 1) >> 1) & 1, abort_flag, err, kErrBwdWait)) break;
           tc_fence_after();
           issue_dp(n + 1);
           tc_commit(dp_full);
           if (!mbar_wait(p_full, par ^ 1u, abort_flag, err, kErrBwdWait)) break;
           tc_fence_after();
           issue_dv(n + 1);
+          tc_commit(&qo_empty[(n + 1) & 1]);
           if (n + 2 < N) {
             // S^T(n+2) overwrites P^T(n+1), which dV(n+1) -- issued just before --
             // reads first; its Q stage was refilled after dK(n) completed.
-            if (!mbar_wait(&q_full[n & 1], (uint32_t)((n + 2) >> 1) & 1, abort_flag, err, kErrBwdWait)) break;
+            if (!mbar_wait(&qq_full[n & 1], (uint32_t)((n + 2) >> 1) & 1, abort_flag, err, kErrBwdWait)) break;
             tc_fence_after();
             issue_s(n + 2);
             tc_commit(s_full);
@@ -332,7 +364,7 @@ __global__ void __launch_bounds__(448, 1)
       const int i = qit.first_blk + 2 * n + hf;  // this warp's query block
       const bool vis = krow_live && i <= last && in_list(prm.pat, i, kvb);
       const bool diag = (i == kvb);
-      if (!__all_sync(0xffffffffu, mbar_wait(&q_full[st], (uint32_t)(n >> 1) & 1, abort_flag, err, kErrBwdWait)))
+      if (!__all_sync(0xffffffffu, mbar_wait(&qq_full[st], (uint32_t)(n >> 1) & 1, abort_flag, err, kErrBwdWait)))
         break;
       if (!__all_sync(0xffffffffu, mbar_wait(s_full, par, abort_flag, err, kErrBwdWait))) break;
       tc_fence_after();
@@ -369,6 +401,9 @@ __global__ void __launch_bounds__(448, 1)
       }
       tc_fence_before();
       mbar_arrive(p_full);
+      mbar_arrive(&qq_empty[st]);  // done with this step's LSE
+      if (!__all_sync(0xffffffffu, mbar_wait(&qo_full[st], (uint32_t)(n >> 1) & 1, abort_flag, err, kErrBwdWait)))
+        break;
       if (!__all_sync(0xffffffffu, mbar_wait(dp_full, par, abort_flag, err, kErrBwdWait))) break;
       // The dS^T tile last fed dQ^T(n-1) and dK(n-1).
       if (n >= 1 && !__all_sync(0xffffffffu, mbar_wait(dss_free, par ^ 1u, abort_flag, err, kErrBwdWait))) break;
@@ -405,7 +440,7 @@ __global__ void __launch_bounds__(448, 1)
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(ds_full);
-      mbar_arrive(&q_empty[st]);
+      mbar_arrive(&qo_empty[st]);  // done with this step's Delta
     }
 
     // ------------------------------------------------------------ dK, dV epilogue
@@ -497,7 +532,7 @@ __global__ void __launch_bounds__(448, 1)
       // step n+2 (issued once dK(n) freed their stage) go through L2 first, so
       // the next S^T is not starved by this step's reductions.
       if (n + 2 < N &&
-          !__all_sync(0xffffffffu, mbar_wait(&q_full[n & 1], (uint32_t)((n + 2) >> 1) & 1, abort_flag, err,
+          !__all_sync(0xffffffffu, mbar_wait(&qq_full[n & 1], (uint32_t)((n + 2) >> 1) & 1, abort_flag, err,
                                              kErrBwdWait)))
         break;
       if (second) {
