@@ -46,7 +46,7 @@ struct FwdLayout {
   static constexpr int OFF_K = OFF_Q + NT * Q_BYTES;
   static constexpr int OFF_V = OFF_K + NS * KVC_BYTES;
   static constexpr int OFF_BAR = OFF_V + NS * KVC_BYTES;
-  static constexpr int NBAR = 1 + 3 * NS + NT * 3;
+  static constexpr int NBAR = 1 + 3 * NS + NT * 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;  // room to align the base to 1024 bytes
@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
   uint64_t* k_full = bars + 1;
   uint64_t* v_full = bars + 1 + NS;
   uint64_t* kv_empty = bars + 1 + 2 * NS;
-  uint64_t* tile_bars = bars + 1 + 3 * NS;  // per tile: s_full, p_full, pv_done
+  uint64_t* tile_bars = bars + 1 + 3 * NS;  // per tile: s_full, p_full, pv_done, p_half
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -95,9 +95,10 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
       mbar_init(&kv_empty[s], 1);
     }
     for (int t = 0; t < NT; ++t) {
-      mbar_init(&tile_bars[3 * t + 0], 1);    // s_full
-      mbar_init(&tile_bars[3 * t + 1], 128);  // p_full
-      mbar_init(&tile_bars[3 * t + 2], 1);    // pv_done
+      mbar_init(&tile_bars[4 * t + 0], 1);    // s_full
+      mbar_init(&tile_bars[4 * t + 1], 128);  // p_full: all of P written (and the row state updated)
+      mbar_init(&tile_bars[4 * t + 2], 1);    // pv_done
+      mbar_init(&tile_bars[4 * t + 3], 128);  // p_half: O rescaled and P of the first 64 columns written
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -185,29 +186,33 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
           const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
           tc_mma_ss(d, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&tile_bars[3 * t + 0]);
+        tc_commit(&tile_bars[4 * t + 0]);
         return true;
       };
-      // O_t += P_t(c) V(c), K = 64 * nb, P from TMEM.
+      // O_t += P_t(c) V(c), K = 64 * nb, P from TMEM. The first 64 KV rows go
+      // as soon as the softmax has written their P (p_half), the second 64
+      // once the whole chunk is done (p_full), so half of PV overlaps the
+      // softmax's second half.
       auto issue_pv = [&](int c, int nb, int t) -> bool {
         const int st = c % NS;
-        if (!mbar_wait(&tile_bars[3 * t + 1], (uint32_t)c & 1, abort_flag, err, kErrFwdWait)) return false;
+        if (!mbar_wait(&tile_bars[4 * t + 3], (uint32_t)c & 1, abort_flag, err, kErrFwdWait)) return false;
         if (t == 0 && !mbar_wait(&v_full[st], (uint32_t)(c / NS) & 1, abort_flag, err, kErrFwdWait)) return false;
         tc_fence_after();
         const uint64_t b0 = opaque_u64(dV0 + (uint32_t)((st * L::KVC_BYTES) >> 4));
         const uint32_t d = tmem + (uint32_t)(t * D);
         const uint32_t a = tmem + L::T_S + 128 * t;
         const uint32_t acc0 = c > 0 ? 1u : 0u;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma_ts(d, a + 8 * kk, b0 + (uint32_t)(kk * 2048 >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+        if (!mbar_wait(&tile_bars[4 * t + 1], (uint32_t)c & 1, abort_flag, err, kErrFwdWait)) return false;
+        tc_fence_after();
         if (nb == 2) {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            tc_mma_ts(d, a + 8 * kk, b0 + (uint32_t)(kk * 2048 >> 4), idesc_pv, kk > 0 ? 1u : acc0);
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            tc_mma_ts(d, a + 8 * kk, b0 + (uint32_t)(kk * 2048 >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+          for (int kk = 4; kk < 8; ++kk)
+            tc_mma_ts(d, a + 8 * kk, b0 + (uint32_t)(kk * 2048 >> 4), idesc_pv, 1u);
         }
-        tc_commit(&tile_bars[3 * t + 2]);
+        tc_commit(&tile_bars[4 * t + 2]);
         return true;
       };
       int nb = 1;
@@ -235,9 +240,10 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
     const int i = 4 * span + 2 * t + (r >> 6);
     const int rr = r & 63;
     const bool row_live = i < prm.nqb;
-    uint64_t* s_full = &tile_bars[3 * t + 0];
-    uint64_t* p_full = &tile_bars[3 * t + 1];
-    uint64_t* pv_done = &tile_bars[3 * t + 2];
+    uint64_t* s_full = &tile_bars[4 * t + 0];
+    uint64_t* p_full = &tile_bars[4 * t + 1];
+    uint64_t* pv_done = &tile_bars[4 * t + 2];
+    uint64_t* p_half = &tile_bars[4 * t + 3];
     const uint32_t t_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t t_o = t_lane + (uint32_t)(t * D);
     const uint32_t t_s = t_lane + L::T_S + (uint32_t)(128 * t);
@@ -292,6 +298,19 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
         m = m_blk;
       }
       const float m_use = (m == -INFINITY) ? 0.f : m;
+      // Lazy rescale of O (warp-uniform: tcgen05.ld/st are warp-collective),
+      // before any P of this chunk is handed to the tensor core. PV_t(c-1)
+      // completed before S_t(c) did, so O is stable here.
+      if (__any_sync(0xffffffffu, need && c > 0)) {
+#pragma unroll 1
+        for (int ch = 0; ch < D / 16; ++ch) {  // 16 columns at a time: the chunk's S is live
+          uint32_t o[16];
+          tmem_ld16(t_o + (uint32_t)(16 * ch), o);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st16(t_o + (uint32_t)(16 * ch), o);
+        }
+      }
       // P = 2^(x * scale * log2 e - m), packed to bf16 and written back over the
       // first half of this tile's S columns (already read). In every group of
       // eight columns the last pair -- a quarter -- takes the FMA-pipe
@@ -331,22 +350,14 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
           }
           tmem_st32(t_s + 32 * hb, pk);
         }
+        if (hb == 0) {
+          tc_fence_before();
+          mbar_arrive(p_half);
+        }
       }
       const float2 rs2 = add2(add2(rs4[0], rs4[1]), add2(rs4[2], rs4[3]));
       l = l * alpha + (rs2.x + rs2.y);
 
-      // Lazy rescale of O (warp-uniform: tcgen05.ld/st are warp-collective).
-      // PV_t(c-1) completed before S_t(c) did, so O is stable here.
-      if (__any_sync(0xffffffffu, need && c > 0)) {
-#pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t o[32];
-          tmem_ld32(t_o + (uint32_t)(32 * ch), o);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(t_o + (uint32_t)(32 * ch), o);
-        }
-      }
       tc_fence_before();
       mbar_arrive(p_full);
       j = jn;
