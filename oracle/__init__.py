@@ -40,5 +40,7 @@ from .attention import (  # noqa: F401
     attention_backward_rows,
     attention_backward_kv_rows,
     decode,
+    reduced_cache_rows,
+    reduced_cache,
     merge_partials,
 )

@@ -320,6 +320,25 @@ def decode(q, k_cache, v_cache, cache_lens, scale: float):
     return o, lse
 
 
+def reduced_cache_rows(T: int, p: Pattern) -> np.ndarray:
+    """Prompt rows the reduced KV cache of a sparse layer holds when decoding
+    the token at position T: every key token kj < T that query T may attend
+    (Abstract: "GPU-friendly KV cache reduction"; the cache keeps only what
+    the static pattern can still reach), ascending. int64 row indices."""
+    kj = np.arange(T, dtype=np.int64)
+    return kj[allowed(T, kj, p)]
+
+
+def reduced_cache(k, v, T: int, p: Pattern):
+    """Gather the reduced cache from prompt K/V [B, >=T, Hkv, D]: returns
+    (k_cache [B, n, Hkv, D], v_cache [B, n, Hkv, D], rows [n]) with the rows of
+    ``reduced_cache_rows`` in that order (values copied, not converted)."""
+    rows = reduced_cache_rows(T, p)
+    k = np.asarray(k)
+    v = np.asarray(v)
+    return k[:, rows], v[:, rows], rows
+
+
 def merge_partials(o_parts, lse_parts):
     """Combine attention over disjoint key subsets: lse = log sum exp(lse_s),
     o = sum_s exp(lse_s - lse) o_s. Empty parts carry lse_s = -inf."""

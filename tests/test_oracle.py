@@ -317,6 +317,45 @@ def test_decode_over_gathered_cache_equals_prefill_row():
         assert abs(lse[0, 0] - l2[0]) < 1e-12
 
 
+GOLDEN_CACHE = os.path.join(os.path.dirname(__file__), "golden", "reduced_cache_rows.txt")
+
+
+def load_cache_golden():
+    rows = {}
+    with open(GOLDEN_CACHE) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            name, T, b, sink, local, stride, n = line.split()
+            rows[name] = (int(T), Pattern(int(b), int(sink), int(local), int(stride)), int(n))
+    return rows
+
+
+@pytest.mark.parametrize("name", sorted(load_cache_golden()))
+def test_reduced_cache_rows_match_hand_counts(name):
+    T, p, n = load_cache_golden()[name]
+    rows = oracle.reduced_cache_rows(T, p)
+    assert len(rows) == n
+    assert np.all(np.diff(rows) > 0) and (n == 0 or rows[-1] < T)
+
+
+@pytest.mark.parametrize("p", [Pattern(16, 1, 3, 4), Pattern(16, 2, 2, 0), Pattern(16, 0, 1, 0), Pattern.full(16)])
+def test_decode_over_reduced_cache_plus_own_row_equals_prefill_row(p):
+    # The hand-off identity: decoding token T over the reduced cache of the
+    # prompt [0, T) plus its own K/V row gives prefill attention row T.
+    S, D, scale = 16 * 12, 8, 0.3
+    q, k, v = rnd((S, D), 60), rnd((S, D), 61), rnd((S, D), 62)
+    for T in (16, 80, 176):
+        kc, vc, rows = oracle.reduced_cache(k[None, :, None], v[None, :, None], T, p)
+        kc = np.concatenate([kc, k[None, T:T + 1, None]], axis=1)
+        vc = np.concatenate([vc, v[None, T:T + 1, None]], axis=1)
+        o, lse = oracle.decode(q[T][None, None], kc, vc, [kc.shape[1]], scale)
+        o2, l2 = oracle.attention_rows(q, k, v, [T], p, scale)
+        np.testing.assert_allclose(o[0, 0], o2[0], atol=1e-13)
+        assert abs(lse[0, 0] - l2[0]) < 1e-12
+
+
 @pytest.mark.parametrize("nsplit", [1, 2, 5, 17])
 def test_merge_of_any_partition_equals_unsplit(nsplit):
     L, D = 97, 8
