@@ -28,15 +28,16 @@ __all__ = [
     "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd",
     "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd",
     "lg_sparse_decode_splits", "lg_sparse_decode_workspace", "lg_sparse_decode",
-    "lg_sparse_decode_noalloc", "lg_exp2_device", "lg_device_status", "EXPORTED_SYMBOLS",
+    "lg_sparse_decode_noalloc", "lg_kv_compact_rows", "lg_kv_compact", "lg_exp2_device", "lg_device_status",
+    "EXPORTED_SYMBOLS",
 ]
 
 EXPORTED_SYMBOLS = (
     "lg_strerror", "lg_version", "lg_pattern_expand", "lg_pattern_expand_t", "lg_pattern_pairs",
     "lg_pattern_iterate_device", "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd",
     "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd", "lg_sparse_decode_splits",
-    "lg_sparse_decode_workspace", "lg_sparse_decode", "lg_sparse_decode_noalloc", "lg_exp2_device",
-    "lg_device_status",
+    "lg_sparse_decode_workspace", "lg_sparse_decode", "lg_sparse_decode_noalloc", "lg_kv_compact_rows",
+    "lg_kv_compact", "lg_exp2_device", "lg_device_status",
 )
 
 
@@ -83,6 +84,8 @@ _SIGS = {
     "lg_sparse_decode_workspace": (_c_i32, [_c_i32] * 6 + [_P(_c_sz)]),
     "lg_sparse_decode": (_c_i32, [_c_vp] * 6 + [_c_i32] * 6 + [_c_f, _c_vp, _c_sz, _c_vp]),
     "lg_sparse_decode_noalloc": (_c_i32, [_c_vp] * 6 + [_c_i32] * 6 + [_c_f, _c_vp]),
+    "lg_kv_compact_rows": (_c_i32, [_P(_lg_pattern_t), _c_i32, _P(_c_i32)]),
+    "lg_kv_compact": (_c_i32, [_P(_lg_pattern_t), _c_vp, _c_vp] + [_c_i32] * 4 + [_c_vp, _c_vp, _c_i32, _c_vp, _c_vp]),
     "lg_exp2_device": (_c_i32, [_c_vp, _c_vp, _c_i64, _c_i32, _c_vp]),
     "lg_device_status": (_c_i32, [_c_i32, _P(ctypes.c_uint32)]),
 }
@@ -301,6 +304,30 @@ def lg_sparse_decode(q, k_cache, v_cache, cache_lens, o, lse, scale: float, num_
     _check(lib().lg_sparse_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), cache_lens.data_ptr(),
                                   o.data_ptr(), _ptr(lse), B, H, Hkv, D, Lmax, int(num_splits), float(scale),
                                   _ptr(workspace), ws, _stream(stream)), "lg_sparse_decode")
+
+
+def lg_kv_compact_rows(pattern, S) -> int:
+    """Rows of the reduced cache lg_kv_compact writes for a prompt of S tokens."""
+    n = _c_i32(0)
+    _check(lib().lg_kv_compact_rows(ctypes.byref(_pat(pattern)), int(S), ctypes.byref(n)), "lg_kv_compact_rows")
+    return n.value
+
+
+def lg_kv_compact(pattern, k, v, k_cache, v_cache, cache_lens, stream=None):
+    """k, v [B,S,Hkv,D] bf16 (prompt); k_cache, v_cache [B,Lmax,Hkv,D] bf16 and
+    cache_lens [B] int32 (written): the reduced cache for decoding token S."""
+    import torch
+
+    B, S, Hkv, D = k.shape
+    Lmax = k_cache.shape[1]
+    _expect(k, "k", torch.bfloat16, (B, S, Hkv, D))
+    _expect(v, "v", torch.bfloat16, (B, S, Hkv, D), k.device)
+    _expect(k_cache, "k_cache", torch.bfloat16, (B, Lmax, Hkv, D), k.device)
+    _expect(v_cache, "v_cache", torch.bfloat16, (B, Lmax, Hkv, D), k.device)
+    _expect(cache_lens, "cache_lens", torch.int32, (B,), k.device)
+    _check(lib().lg_kv_compact(ctypes.byref(_pat(pattern)), k.data_ptr(), v.data_ptr(), B, S, Hkv, D,
+                               k_cache.data_ptr(), v_cache.data_ptr(), Lmax, cache_lens.data_ptr(), _stream(stream)),
+           "lg_kv_compact")
 
 
 def lg_sparse_decode_noalloc(q, k_cache, v_cache, cache_lens, o, lse, scale: float, num_splits: int = 0,

@@ -333,6 +333,36 @@ lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* p, const void* q, const void*
   return cuda_status(lg::launch_bwd_dq(dq_acc, dq, grad_f32, scale, B, S, H, D, s));
 }
 
+// ---------------------------------------------------------------- prefill -> decode hand-off
+lg_status_t lg_kv_compact_rows(const lg_pattern_t* p, int32_t S, int32_t* rows) {
+  lg_status_t st = check_pattern(p);
+  if (st != LG_OK) return st;
+  if (rows == nullptr || S <= 0) return LG_ERR_INVALID_ARG;
+  if (p->block_size != 64 || S % 64 != 0) return LG_ERR_UNSUPPORTED;
+  *rows = 64 * lg::compact_blocks(*p, S);
+  return LG_OK;
+}
+
+lg_status_t lg_kv_compact(const lg_pattern_t* p, const void* k, const void* v, int32_t B, int32_t S, int32_t Hkv,
+                          int32_t D, void* k_cache, void* v_cache, int32_t Lmax, int32_t* cache_lens,
+                          lg_stream_t stream) {
+  int32_t rows = 0;
+  lg_status_t st = lg_kv_compact_rows(p, S, &rows);
+  if (st != LG_OK) return st;
+  if (!k || !v || !k_cache || !v_cache || !cache_lens) return LG_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || D <= 0 || Lmax <= 0) return LG_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return LG_ERR_UNSUPPORTED;
+  if (B > 65535) return LG_ERR_UNSUPPORTED;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache)) return LG_ERR_UNSUPPORTED;
+  if (Lmax < rows) return LG_ERR_CAPACITY;
+  lg::CompactParams prm;
+  prm.pat = *p;
+  prm.S = S;
+  prm.Lmax = Lmax;
+  prm.row_chunks = (long long)Hkv * D / 8;
+  return cuda_status(lg::launch_compact(k, v, k_cache, v_cache, cache_lens, prm, B, static_cast<cudaStream_t>(stream)));
+}
+
 // ---------------------------------------------------------------- decode
 lg_status_t lg_sparse_decode_splits(int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax, int32_t num_splits,
                                     int32_t* splits) {

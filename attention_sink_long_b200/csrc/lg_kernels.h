@@ -54,6 +54,17 @@ cudaError_t launch_bwd128(const CUtensorMap& tq, const CUtensorMap& tk, const CU
 cudaError_t launch_bwd_dq(const float* dq_acc, void* dq, int dq_f32, float scale, int B, int S, int H, int D,
                           cudaStream_t stream);
 
+// Prefill -> decode hand-off (compact.cu).
+struct CompactParams {
+  lg_pattern_t pat;
+  int S;                // prompt length (multiple of 64)
+  int Lmax;             // cache rows per batch row
+  long long row_chunks; // 16-byte chunks per token row of all KV heads (Hkv * D / 8)
+};
+int compact_blocks(const lg_pattern_t& pat, int S);
+cudaError_t launch_compact(const void* k, const void* v, void* kc, void* vc, int32_t* lens, const CompactParams& prm,
+                           int B, cudaStream_t stream);
+
 struct DecodeParams {
   const void* q;        // [B, H, D] bf16
   const void* k_cache;  // [B, Lmax, Hkv, D] bf16

@@ -65,6 +65,20 @@ struct KvIter {
     if (stride > 0) n += ceil_div_nonneg(lo, stride) - ceil_div_nonneg(a, stride);
     return n + (hi - lo + 1);
   }
+  // The n-th listed block (0 <= n < count()) in closed form: the sink blocks
+  // below the window, then the strided blocks below it, then the window.
+  LG_HD int nth(int n) const {
+    const int a = imin(imax(sink, 0), lo);
+    if (n < a) return n;
+    n -= a;
+    if (stride > 0) {
+      const int s0 = ceil_div_nonneg(a, stride);
+      const int ns = ceil_div_nonneg(lo, stride) - s0;
+      if (n < ns) return (s0 + n) * stride;
+      n -= ns;
+    }
+    return lo + n;
+  }
 };
 
 // The KvIter sequence grouped into chunks of one listed block, or two when the

@@ -51,7 +51,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
-    ap.add_argument("--workload", choices=["step32k", "fwd128k", "bwd128k", "decode"], default="step32k")
+    ap.add_argument("--workload", choices=["step32k", "fwd128k", "bwd128k", "decode", "handoff"], default="step32k")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
@@ -145,6 +145,11 @@ def workload(name):
         return {"workload": "32-layer hybrid decode step: 21 sparse layers (4160 rows) + 11 full layers (131072 rows)",
                 "prefill": None, "fwd": [], "bwd": [],
                 "decode": {"B": 32, "H": 32, "Hkv": 32, "D": D, "L": 4160, "L_full": 131072}}
+    if name == "handoff":
+        return {"workload": "prefill->decode hand-off: reduced sink+window KV cache of 32K-token prompts, "
+                            "B32 Hkv32 D128",
+                "prefill": None, "fwd": [], "bwd": [], "decode": None,
+                "handoff": {"B": 32, "S": 32768, "Hkv": 32, "D": D, "pattern": SINK_WINDOW}}
     raise ValueError(name)
 
 
@@ -270,6 +275,17 @@ class CudaStep:
                                        device=device)
                 fbytes = 2 * B * Lf * Hkv * D * 2 + 2 * B * H * D * 2
                 self.parts.append(("decode full layer", "decode_full", 4 * D * Lf * B * H, fbytes, 1))
+        ho = wl.get("handoff")
+        if ho is not None:
+            B, S, Hkv, D = ho["B"], ho["S"], ho["Hkv"], ho["D"]
+            self.hk = si.device_normal((B, S, Hkv, D), si.SEED_BASE + 1, device)
+            self.hv = si.device_normal((B, S, Hkv, D), si.SEED_BASE + 2, device)
+            rows = lg.lg_kv_compact_rows(ho["pattern"], S)
+            self.hkc = torch.empty(B, rows + 64, Hkv, D, dtype=torch.bfloat16, device=device)
+            self.hvc = torch.empty_like(self.hkc)
+            self.hlens = torch.empty(B, dtype=torch.int32, device=device)
+            nbytes = 2 * 2 * B * rows * Hkv * D * 2  # K and V, each row read once and written once
+            self.parts.append(("handoff sink+window", "copy", 0, nbytes, 1))
 
     def _bwd_available(self, pf, pattern):
         """One tiny backward call: False when the library reports it unsupported."""
@@ -315,6 +331,11 @@ class CudaStep:
                 if events is not None:
                     events[i].record(self.stream)
                 i += 1
+        if wl.get("handoff") is not None:
+            lg.lg_kv_compact(wl["handoff"]["pattern"], self.hk, self.hv, self.hkc, self.hvc, self.hlens)
+            if events is not None:
+                events[i].record(self.stream)
+            i += 1
 
     def scale_dec(self):
         return 1.0 / math.sqrt(self.wl["decode"]["D"])
@@ -334,14 +355,14 @@ def host_buffers(step):
     torch = step.torch
     pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu())  # noqa: E731
     ins, outs = [], []
-    for name in ("q", "k", "v", "do", "dq_in", "kc", "vc", "lens"):
+    for name in ("q", "k", "v", "do", "dq_in", "kc", "vc", "lens", "hk", "hv"):
         if hasattr(step, name):
             ins.append((getattr(step, name), pin(getattr(step, name))))
     for d in ("o", "lse"):
         if hasattr(step, d):
             for t in getattr(step, d).values():
                 outs.append((t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)))
-    for name in ("dq", "dk", "dv", "do_out", "dlse"):
+    for name in ("dq", "dk", "dv", "do_out", "dlse", "hkc", "hvc", "hlens"):
         if hasattr(step, name):
             t = getattr(step, name)
             outs.append((t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)))
@@ -402,7 +423,12 @@ def cuda_arm(args, rank, world, dist):
     if wl["workload"].startswith("32-layer"):
         # Reported decode step: 21 sparse-layer + 11 full-layer calls, from the per-call times.
         ms_per_step = sum(w * statistics.mean(per_part_ms[i]) for i, w in enumerate(weights))
-    value = world * step_flops / (ms_per_step * 1e-3) / 1e12
+    # A workload without FLOPs (the hand-off copy) reports bytes moved per second.
+    step_bytes = sum(w * (p[3] or 0) for w, p in zip(weights, step.parts))
+    by_bytes = step_flops == 0
+    unit = "GB/s" if by_bytes else "TFLOP/s"
+    value = world * (step_bytes / (ms_per_step * 1e-3) / 1e9 if by_bytes else
+                     step_flops / (ms_per_step * 1e-3) / 1e12)
 
     peaks, peak_src = load_peaks()
     tensor_peak, tensor_kind = pick_peak(peaks, clk, "tensor")
@@ -411,7 +437,7 @@ def cuda_arm(args, rank, world, dist):
     for i, (name, kind, flops, nbytes, nl) in enumerate(step.parts):
         ms = statistics.mean(per_part_ms[i])
         r = {"ms": round(ms, 4), "useful_tflops": round(flops / (ms * 1e-3) / 1e12, 2)}
-        if kind.startswith("decode"):
+        if kind.startswith("decode") or kind == "copy":
             r["gbs"] = round(nbytes / (ms * 1e-3) / 1e9, 1)
             r["frac_hbm"] = round(r["gbs"] / peaks["hbm_gbs"], 4)
         else:
@@ -422,7 +448,7 @@ def cuda_arm(args, rank, world, dist):
     di = dominant[0]
     dname, dkind, dflops, dbytes, _ = step.parts[di]
     dms = statistics.mean(per_part_ms[di])
-    if dkind.startswith("decode"):
+    if dkind.startswith("decode") or dkind == "copy":
         achieved = dbytes / (dms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4)}
@@ -463,7 +489,8 @@ def cuda_arm(args, rank, world, dist):
         e1.record(step.stream)
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1) / ek, dist, device)
-        e2e = {"value": round(world * step_flops / (ems * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        e2e_v = step_bytes / (ems * 1e-3) / 1e9 if by_bytes else step_flops / (ems * 1e-3) / 1e12
+        e2e = {"value": round(world * e2e_v, 3), "unit": unit,
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(ems, 3), "steps": ek}
 
     cpu = None
@@ -478,8 +505,10 @@ def cuda_arm(args, rank, world, dist):
         config.update({"prefill_shape": pf, "patterns": {n: list(p) for n, p in wl["fwd"] + wl["bwd"]}})
     if wl["decode"]:
         config["decode_shape"] = wl["decode"]
+    if wl.get("handoff"):
+        config["handoff_shape"] = {k: (list(v) if k == "pattern" else v) for k, v in wl["handoff"].items()}
     line = {
-        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16; no dataset, no weights)",
         "config": config, "roofline": roof, "rows": rows, "cpu_baseline": cpu, "e2e": e2e,
@@ -521,6 +550,12 @@ def oracle_sample(wl, budget_s, seed=11):
             jobs.append(("bwd " + n, "bwd", p))
     if wl["decode"]:
         jobs.append(("decode", "decode", None))
+    ho = wl.get("handoff")
+    if ho:
+        # One KV head of one prompt, drawn on the host with the same seed as head 0.
+        _, hk, hv = si.prefill_inputs(1, ho["S"], 1, 1, ho["D"])
+        hk, hv = hk.double().numpy(), hv.double().numpy()
+        jobs.append(("handoff", "handoff", oracle.Pattern(*ho["pattern"])))
     per_job = budget_s / max(1, len(jobs))
     for name, kind, p in jobs:
         t_start = time.perf_counter()
@@ -538,6 +573,9 @@ def oracle_sample(wl, budget_s, seed=11):
                 else:
                     oracle.attention_backward_rows(qh, kh, vh, doh, rows, op, scale)
                     job_flops += 6 * D * pairs  # S, dP and dQ for these rows
+            elif kind == "handoff":
+                kc, vc, rws = oracle.reduced_cache(hk, hv, ho["S"], p)
+                job_flops += 2 * 2 * len(rws) * ho["D"] * 2  # bytes: K and V rows read and written (bf16)
             else:
                 dc = wl["decode"]
                 L, D2 = dc["L"], dc["D"]
@@ -548,8 +586,15 @@ def oracle_sample(wl, budget_s, seed=11):
         dt = time.perf_counter() - t_start
         flops += job_flops
         t_used += dt
-        desc.append(f"{name}: {n_done} {'query blocks of one head' if kind != 'decode' else '(b,h) rows'}")
+        what = {"decode": "(b,h) rows", "handoff": "one-head prompt compactions"}.get(kind, "query blocks of one head")
+        desc.append(f"{name}: {n_done} {what}")
     return flops, t_used, "; ".join(desc)
+
+
+def work_unit(wl):
+    """(unit, scale) of oracle_sample's work count: FLOPs, or bytes for the hand-off alone."""
+    only_copy = wl.get("handoff") and not (wl["prefill"] or wl["decode"])
+    return ("GB/s", 1e9) if only_copy else ("TFLOP/s", 1e12)
 
 
 def cpu_cores():
@@ -564,9 +609,10 @@ def cpu_baseline(wl, budget_s):
 
     with threadpool_limits(limits=cpu_cores()):
         flops, secs, desc = oracle_sample(wl, budget_s)
-    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+    unit, sc = work_unit(wl)
+    return {"value": round(flops / secs / sc, 6), "unit": unit, "cores": cpu_cores(), "kind": "oracle",
             "sample": f"fp64 numpy oracle, {secs:.1f} s: {desc}; useful FLOPs credited 4D/pair fwd, "
-                      f"6D/pair bwd dQ rows, 4D/row decode"}
+                      f"6D/pair bwd dQ rows, 4D/row decode; hand-off credited its bf16 bytes"}
 
 
 def reference_arm(args, rank, world):
@@ -581,16 +627,17 @@ def reference_arm(args, rank, world):
         f, s, desc = oracle_sample(wl, per_step)
         tot_f += f
         tot_s += s
-    value = tot_f / tot_s / 1e12
+    unit, sc = work_unit(wl)
+    value = tot_f / tot_s / sc
     line = {
-        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) bf16 upcast to f64)",
         "config": {"workload": wl["workload"], "sample": "bounded oracle sample per step (see cpu_baseline)"},
-        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+        "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cpu_cores(), "kind": "oracle",
                          "sample": desc},
-        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 

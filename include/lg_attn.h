@@ -166,8 +166,9 @@ lg_status_t lg_sparse_attn_bwd_workspace(const lg_pattern_t* pattern, int32_t B,
  * Device pointers: q, k, v, dout bf16; o as written by the forward, of
  * element type o_dtype; lse as written by the forward; dq [B,S,H,D], dk/dv
  * [B,S,Hkv,D] (written; dk/dv sum over the query heads of a KV group) of
- * element type grad_dtype. P enters the dV product as a bf16 hi + lo pair
- * (dV is exact to fp32 accumulation); dS enters dK and dQ as bf16.
+ * element type grad_dtype. P and dS enter the tensor-core products as bf16;
+ * with query-head groups (H > Hkv) they also enter dV / dK as a bf16 hi + lo
+ * pair (exact to fp32 accumulation), since those sums grow with the group.
  * workspace (device, 256-byte aligned) of at least the queried size; its
  * contents on entry do not matter.
  */
@@ -175,6 +176,41 @@ lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* pattern, const void* q, const
                                const void* o, int32_t o_dtype, const void* dout, const float* lse, void* dq,
                                void* dk, void* dv, int32_t grad_dtype, int32_t B, int32_t S, int32_t H, int32_t Hkv,
                                int32_t D, float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Prefill -> decode hand-off: the reduced KV cache                         */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Rows of the reduced cache lg_kv_compact writes for a prompt of S tokens
+ * (S a multiple of block_size = 64): 64 x the number of whole blocks kb < S/64
+ * with kb < sink_blocks, or S/64 - kb < local_blocks, or (stride > 0 and
+ * kb % stride == 0). Written to *rows. Host only; errors: LG_ERR_INVALID_ARG
+ * (bad pattern, S <= 0, rows NULL), LG_ERR_UNSUPPORTED (block_size != 64,
+ * S % 64 != 0).
+ */
+lg_status_t lg_kv_compact_rows(const lg_pattern_t* pattern, int32_t S, int32_t* rows);
+
+/*
+ * Prefill -> decode hand-off for a sparse layer (Abstract: the static patterns
+ * allow a "GPU-friendly KV cache reduction"; summary, "Key results": 69.2 ->
+ * 26.5 GB of KV cache at 128K). After the prefill of S tokens, the next token
+ * (position S) may attend exactly the whole earlier blocks counted by
+ * lg_kv_compact_rows; this call copies those 64-row blocks of k and v, in
+ * ascending block order, to rows [0, rows) of k_cache / v_cache and writes
+ * cache_lens[b] = rows for every batch row. Decoding token S over rows
+ * [0, rows) plus its own K/V row (appended by the caller at row `rows`)
+ * equals prefill attention row S. Values are copied bit for bit.
+ * Device pointers, 16-byte aligned: k, v [B,S,Hkv,D] bf16 (read);
+ * k_cache, v_cache [B,Lmax,Hkv,D] bf16 (rows [0, rows) written, the rest
+ * untouched; must not overlap k / v); cache_lens [B] int32 (written).
+ * Errors: LG_ERR_INVALID_ARG (NULL pointer, non-positive sizes, bad pattern),
+ * LG_ERR_UNSUPPORTED (block_size != 64, S % 64 != 0, D not 64 or 128,
+ * misaligned pointer), LG_ERR_CAPACITY (Lmax < rows), LG_ERR_CUDA (launch).
+ */
+lg_status_t lg_kv_compact(const lg_pattern_t* pattern, const void* k, const void* v, int32_t B, int32_t S,
+                          int32_t Hkv, int32_t D, void* k_cache, void* v_cache, int32_t Lmax, int32_t* cache_lens,
+                          lg_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Decode over the reduced KV cache                                         */

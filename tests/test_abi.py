@@ -153,3 +153,34 @@ def test_workspace_queries():
     ns = lg.lg_sparse_decode_splits(32, 32, 32, 128, 131072)
     assert lg.lg_sparse_decode_workspace(32, 32, 32, 128, 131072) >= 32 * 32 * ns * 129 * 4
     assert lg.lg_sparse_decode_splits(2, 8, 8, 128, 100, 7) == 7
+
+
+# ---------------------------------------------------------------- prefill -> decode hand-off (host side)
+
+@pytest.mark.parametrize("p", [(64, 1, 64, 0), (64, 1, 16, 32), (64, 0, 2**31 - 1, 0), (64, 0, 1, 0), (64, 1, 4, 0),
+                               (64, 4, 8, 0), (64, 0, 2, 3), (64, 2, 3, 5), (64, 7, 1, 2), (64, 100, 1, 0)])
+@pytest.mark.parametrize("S", [64, 128, 1024, 4096, 8192])
+def test_compact_rows_match_oracle(p, S):
+    """Host row count of the reduced cache equals the oracle's row list length, bit for bit."""
+    assert lg.lg_kv_compact_rows(p, S) == len(oracle.reduced_cache_rows(S, oracle.Pattern(*p)))
+
+
+def test_compact_argument_errors():
+    L = lg.lib()
+    p = lg._lg_pattern_t(64, 1, 64, 0)
+    n = ctypes.c_int32(0)
+    assert L.lg_kv_compact_rows(ctypes.byref(p), 1000, ctypes.byref(n)) == 2            # S % 64
+    assert L.lg_kv_compact_rows(ctypes.byref(p), 0, ctypes.byref(n)) == 1
+    assert L.lg_kv_compact_rows(ctypes.byref(p), 4096, None) == 1
+    assert L.lg_kv_compact_rows(None, 4096, ctypes.byref(n)) == 1
+
+    def compact(k=0x10000, v=0x20000, kc=0x30000, vc=0x40000, lens=0x50000, B=2, S=32768, Hkv=8, D=128, Lmax=4160):
+        return L.lg_kv_compact(ctypes.byref(p), k, v, B, S, Hkv, D, kc, vc, Lmax, lens, None)
+
+    assert compact(Lmax=4095) == 6          # 4096 rows do not fit
+    assert compact(k=None) == 1
+    assert compact(lens=None) == 1
+    assert compact(B=0) == 1
+    assert compact(D=96) == 2
+    assert compact(S=1000) == 2
+    assert compact(kc=0x30008) == 2         # misaligned
