@@ -8,8 +8,9 @@
 // blocks, computes S = Q K^T and O += P V on the tcgen05 tensor cores with the
 // accumulators in TMEM, and keeps an online softmax per row.
 //
-// KV blocks are consumed in chunks of one block, or two adjacent listed blocks
-// (KvChunks), so most MMAs run with N = 128 (S) and K = 128 (PV).
+// KV blocks are consumed in chunks of two consecutive listed blocks (KvChunks;
+// adjacent or not, each 64-row half loaded by its own TMA copy), so the MMAs
+// run with N = 128 (S) and K = 128 (PV) on every pattern term.
 //
 // CTA = 10 warps, two 128-row query tiles that share every K/V chunk:
 //   warps 0-3 / 4-7  softmax + epilogue of tile 0 / tile 1; thread r of a group
@@ -129,7 +130,8 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
       int c = 0;
       int nb = 1;
       for (int j = chunks.first(); j >= 0; ++c) {
-        const int jn = chunks.span(j, &nb);
+        int j2 = -1;
+        const int jn = chunks.span(j, &nb, &j2);
         const int st = c % NS;
         const uint32_t use = (uint32_t)(c / NS);
         if (use > 0 && !mbar_wait(&kv_empty[st], (use - 1) & 1, abort_flag, err, kErrFwdWait)) break;
@@ -137,12 +139,12 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
         for (int hb = 0; hb < nb; ++hb)
           for (int p = 0; p < L::DP; ++p)
             tma_load_4d(smem + L::OFF_K + st * L::KVC_BYTES + p * 16384 + hb * 8192, &tmK, &k_full[st], 64 * p, kvh,
-                        64 * (j + hb), b);
+                        64 * (hb == 0 ? j : j2), b);
         mbar_arrive_expect_tx(&v_full[st], nb * 64 * D * 2);
         for (int hb = 0; hb < nb; ++hb)
           for (int p = 0; p < L::DP; ++p)
             tma_load_4d(smem + L::OFF_V + st * L::KVC_BYTES + p * 16384 + hb * 8192, &tmV, &v_full[st], 64 * p, kvh,
-                        64 * (j + hb), b);
+                        64 * (hb == 0 ? j : j2), b);
         j = jn;
       }
       if (*abort_flag) {
@@ -217,11 +219,12 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
       };
       int nb = 1;
       int j = chunks.first();
-      int jn = j >= 0 ? chunks.span(j, &nb) : -1;
+      int jx = -1;
+      int jn = j >= 0 ? chunks.span(j, &nb, &jx) : -1;
       for (int t = 0; t < NT && ok && j >= 0; ++t) ok = issue_s(0, nb, t);
       for (int c = 0; j >= 0 && ok; ++c) {
         int nb_next = 1;
-        const int jnn = jn >= 0 ? chunks.span(jn, &nb_next) : -1;
+        const int jnn = jn >= 0 ? chunks.span(jn, &nb_next, &jx) : -1;
         for (int t = 0; t < NT && ok; ++t) {
           ok = issue_pv(c, nb, t);
           if (ok && jn >= 0) ok = issue_s(c + 1, nb_next, t);
@@ -253,7 +256,8 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
     int c = 0;
     int nb = 1;
     for (int j = chunks.first(); j >= 0; ++c) {
-      const int jn = chunks.span(j, &nb);
+      int j2 = -1;
+      const int jn = chunks.span(j, &nb, &j2);
       if (!__all_sync(0xffffffffu, mbar_wait(s_full, (uint32_t)c & 1, abort_flag, err, kErrFwdWait))) break;
       tc_fence_after();
       // One TMEM read of the whole chunk (128 columns, one wait), masked per
@@ -263,8 +267,9 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
       bool vis[2], diag[2];
 #pragma unroll
       for (int hb = 0; hb < 2; ++hb) {
-        vis[hb] = hb < nb && row_live && in_list(prm.pat, i, j + hb);
-        diag[hb] = (j + hb == i);
+        const int kb = hb == 0 ? j : j2;
+        vis[hb] = hb < nb && row_live && in_list(prm.pat, i, kb);
+        diag[hb] = (kb == i);
       }
       uint32_t xs[128];
       tmem_ld128(t_s, xs);

@@ -81,22 +81,26 @@ struct KvIter {
   }
 };
 
-// The KvIter sequence grouped into chunks of one listed block, or two when the
-// next listed block is adjacent (window and sink runs pair up, isolated strided
-// blocks stay single). span(j, &nb) takes a chunk start j, sets nb to its
-// block count and returns the next chunk start (or -1).
+// The KvIter sequence grouped into chunks of two consecutive listed blocks
+// (adjacent or not: a sink block pairs with the first window block, isolated
+// strided blocks pair with each other), the last chunk holding one block when
+// the list is odd. span(j, &nb, &j2) takes a chunk start j, sets nb to its
+// block count and j2 to its second block (-1 when nb == 1) and returns the
+// next chunk start (or -1).
 struct KvChunks {
   KvIter it;
   LG_HD KvChunks(const lg_pattern_t& p, int i_lo, int i_hi) : it(p, i_lo, i_hi) {}
   LG_HD int first() const { return it.first(); }
-  LG_HD int span(int j, int* nb) const {
-    const int j2 = it.next(j);
-    if (j2 == j + 1) {
+  LG_HD int span(int j, int* nb, int* j2) const {
+    const int n2 = it.next(j);
+    if (n2 >= 0) {
       *nb = 2;
-      return it.next(j2);
+      *j2 = n2;
+      return it.next(n2);
     }
     *nb = 1;
-    return j2;
+    *j2 = -1;
+    return -1;
   }
 };
 

@@ -51,7 +51,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
-    ap.add_argument("--workload", choices=["step32k", "fwd128k", "bwd128k", "decode", "handoff"], default="step32k")
+    ap.add_argument("--workload", choices=["step32k", "fwd128k", "bwd128k", "decode", "handoff", "blocksparse128k"], default="step32k")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
@@ -145,6 +145,13 @@ def workload(name):
         return {"workload": "32-layer hybrid decode step: 21 sparse layers (4160 rows) + 11 full layers (131072 rows)",
                 "prefill": None, "fwd": [], "bwd": [],
                 "decode": {"B": 32, "H": 32, "Hkv": 32, "D": D, "L": 4160, "L_full": 131072}}
+    if name == "blocksparse128k":
+        # 5056 = the block-sparse reduced cache of a 128K prompt (lg_kv_compact_rows).
+        return {"workload": "128K block-sparse {64,1,16,32}: prefill forward + training backward + "
+                            "decode over the reduced cache (5056 rows, B32)",
+                "prefill": {"B": 1, "S": 131072, "H": 32, "Hkv": 32, "D": D},
+                "fwd": [("block-sparse", BLOCK_SPARSE)], "bwd": [("block-sparse", BLOCK_SPARSE)],
+                "decode": {"B": 32, "H": 32, "Hkv": 32, "D": D, "L": 5056}}
     if name == "handoff":
         return {"workload": "prefill->decode hand-off: reduced sink+window KV cache of 32K-token prompts, "
                             "B32 Hkv32 D128",

@@ -71,6 +71,12 @@ def test_workloads_and_useful_work():
     assert bench.pairs_of(bench.SINK_WINDOW, 32768) == 126763008
     assert bench.pairs_of(bench.FULL, 32768) == 32768 * 32769 // 2
     assert bench.pairs_of(bench.BLOCK_SPARSE, 131072) == 398032896
+    import attention_sink_long_b200 as lg
+
+    bs = bench.workload("blocksparse128k")
+    assert bs["decode"]["L"] == lg.lg_kv_compact_rows(bench.BLOCK_SPARSE, bs["prefill"]["S"])
+    ho = bench.workload("handoff")["handoff"]
+    assert lg.lg_kv_compact_rows(ho["pattern"], ho["S"]) == 4096
 
 
 def _run(cmd, timeout=240):

@@ -7,14 +7,14 @@ Parity is checked on the fp32 gradient outputs (the accumulators before any
 output rounding), at max |err| <= 1e-2 and mean |err| <= 1e-3; the bf16
 outputs are checked to be those fp32 values rounded to nearest even (within
 one bf16 ulp, since the order of the dQ reduce-adds varies between runs).
-The benchmark workloads (1K attention-sink, 128K sink+window) run the
-training configuration: bf16 O from the forward. The other shapes take the
+The benchmark workloads (1K attention-sink, 128K sink+window and 128K
+block-sparse) run the training configuration: bf16 O from the forward. The other shapes take the
 forward's fp32 O, which makes Delta = rowsum(dO * O) exact to fp32: with a
 bf16 O, Delta alone carries ~1e-3 relative error, which reaches the 1e-2
 bound on dQ / dK for shapes with large gradients (GQA groups).
-Small shapes are compared in full; the 128K sink+window training workload on
-sampled query blocks (dQ) and KV blocks (dK, dV -- the sink block gathers
-every query of the sequence).
+Small shapes are compared in full; the 128K training workloads on sampled
+query blocks (dQ) and KV blocks (dK, dV -- the sink block gathers every query
+of the sequence; with the strided pattern, block nqb/2 is a strided block).
 """
 
 import math
@@ -89,9 +89,10 @@ def test_bwd_matches_oracle_small(B, S, H, Hkv, D, pat, odt):
     assert_bf16_rounding_of("dV", bv, dv)
 
 
-def test_bwd_128k_sink_window_sampled():
+@pytest.mark.parametrize("pat", [lg.Pattern(64, 1, 64, 0), lg.Pattern(64, 1, 16, 32)],
+                         ids=["sink_window", "block_sparse"])
+def test_bwd_128k_sampled(pat):
     B, S, H, D = 1, 131072, 32, 128
-    pat = lg.Pattern(64, 1, 64, 0)
     op = oracle.Pattern(*pat)
     dev = torch.device("cuda")
     q, k, v, do = si.prefill_inputs_device(B, S, H, H, D, dev, with_dout=True)
