@@ -16,6 +16,7 @@ __device__ unsigned int g_lg_error_word;
 
 namespace {
 
+using lg::imax;
 using lg::imin;
 
 constexpr int kMaxDevices = 64;
@@ -282,15 +283,20 @@ lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* p, const void* q, const void*
   float* dq_acc = static_cast<float*>(workspace);
   float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + round256((size_t)B * H * S * D * 4));
 
+  // Head dim 128 without query-head groups runs the 128-row-step kernel, whose
+  // KV tiles are two separately placed 64-row blocks (BlockPairing); the other
+  // kernel's tiles are 128 consecutive rows.
+  const bool paired = (D == 128 && H == Hkv);
+  const int kv_box = paired ? 64 : 128;
   CUtensorMap tq, tk, tv, tdo, tdk, tdv;
   if ((st = make_map(&tq, q, B, S, H, D, 64)) != LG_OK) return st;
-  if ((st = make_map(&tk, k, B, S, Hkv, D, 128)) != LG_OK) return st;
-  if ((st = make_map(&tv, v, B, S, Hkv, D, 128)) != LG_OK) return st;
+  if ((st = make_map(&tk, k, B, S, Hkv, D, kv_box)) != LG_OK) return st;
+  if ((st = make_map(&tv, v, B, S, Hkv, D, kv_box)) != LG_OK) return st;
   if ((st = make_map(&tdo, dout, B, S, H, D, 64)) != LG_OK) return st;
   // With fp32 gradients the kernel stores dK / dV directly; the bf16 maps are
   // then built over K / V only to have valid (unused) descriptors.
-  if ((st = make_map(&tdk, grad_f32 ? k : dk, B, S, Hkv, D, 128)) != LG_OK) return st;
-  if ((st = make_map(&tdv, grad_f32 ? v : dv, B, S, Hkv, D, 128)) != LG_OK) return st;
+  if ((st = make_map(&tdk, grad_f32 ? k : dk, B, S, Hkv, D, kv_box)) != LG_OK) return st;
+  if ((st = make_map(&tdv, grad_f32 ? v : dv, B, S, Hkv, D, kv_box)) != LG_OK) return st;
 
   st = cuda_status(lg::launch_bwd_pre(o, o_dtype == LG_F32, dout, delta, dq_acc, B, S, H, D, s));
   if (st != LG_OK) return st;
@@ -311,8 +317,18 @@ lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* p, const void* q, const void*
   // tile, seen by every query). Scheduled first; at most 128 of them.
   {
     std::vector<int> counts(prm.nkt);
-    for (int t = 0; t < prm.nkt; ++t)
-      counts[t] = lg::QIter(*p, 2 * t, imin(2 * t + 1, prm.nqb - 1), prm.nqb).count();
+    const lg::BlockPairing bp(*p, prm.nqb);
+    for (int t = 0; t < prm.nkt; ++t) {
+      if (paired) {
+        int x, y;
+        bp.pair(t, &x, &y);
+        const int first = y >= 0 ? imin(x, y) : x;
+        const int last = y >= 0 ? imax(bp.reach(x), bp.reach(y)) : bp.reach(x);
+        counts[t] = last - first + 1;
+      } else {
+        counts[t] = lg::QIter(*p, 2 * t, imin(2 * t + 1, prm.nqb - 1), prm.nqb).count();
+      }
+    }
     std::vector<int> sorted_counts(counts);
     std::nth_element(sorted_counts.begin(), sorted_counts.begin() + prm.nkt / 2, sorted_counts.end());
     const int median = sorted_counts[prm.nkt / 2];

@@ -10,8 +10,11 @@
 //   dS = P o (dP - Delta) with Delta = rowsum(dO o O),
 //   dK = scale * dS^T Q,  dQ = scale * dS K.
 //
-// One CTA owns a 128-row KV tile (two 64-row blocks) of one head and walks
-// the query blocks that see it (QIter) two at a time: a 128-row query step.
+// One CTA owns a 128-row KV tile of one head -- two 64-row KV blocks paired
+// by BlockPairing (blocks every later query sees pair with each other, then
+// the window-only blocks pair in order), so both halves of the tile see nearly
+// the same query blocks -- and walks those query blocks two at a time: a
+// 128-row query step.
 // Every GEMM of a step is then an M = 128, N = 128 tcgen05 MMA -- the shape
 // the tensor core runs at full rate (an N = 64 instruction takes about as
 // long as an N = 128 one):
@@ -129,9 +132,16 @@ __global__ void __launch_bounds__(448, 1)
     }
   }
   const int b = blockIdx.y;
-  const QIter qit(prm.pat, 2 * u, imin(2 * u + 1, prm.nqb - 1), prm.nqb);
-  const int last = qit.last_blk;         // query blocks [first_blk, last] see this KV tile
-  const int N = (qit.count() + 1) / 2;   // 128-row query steps (the last one may hold one block)
+  // The tile's two KV blocks (ky = -1: the tile holds one block; its rows
+  // 64..127 load past the sequence end, i.e. as zeros, and stay masked).
+  const BlockPairing bp(prm.pat, prm.nqb);
+  int kx, ky;
+  bp.pair(u, &kx, &ky);
+  const int kload[2] = {kx, ky >= 0 ? ky : prm.nqb};
+  // Query blocks [q_first, last] see the tile (the union of both blocks' lists).
+  const int q_first = ky >= 0 ? imin(kx, ky) : kx;
+  const int last = ky >= 0 ? imax(bp.reach(kx), bp.reach(ky)) : bp.reach(kx);
+  const int N = (last - q_first + 2) / 2;  // 128-row query steps (the last one may hold one block)
   unsigned int* err = prm.err;
 
   if (threadIdx.x == 0) {
@@ -166,15 +176,16 @@ __global__ void __launch_bounds__(448, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
-      for (int p = 0; p < 2; ++p) {
-        tma_load_4d(smem + L::OFF_K + p * L::PANEL, &tmK, kv_full, 64 * p, h, 128 * u, b);
-        tma_load_4d(smem + L::OFF_V + p * L::PANEL, &tmV, kv_full, 64 * p, h, 128 * u, b);
-      }
+      for (int hb = 0; hb < 2; ++hb)
+        for (int p = 0; p < 2; ++p) {
+          tma_load_4d(smem + L::OFF_K + p * L::PANEL + hb * 8192, &tmK, kv_full, 64 * p, h, 64 * kload[hb], b);
+          tma_load_4d(smem + L::OFF_V + p * L::PANEL + hb * 8192, &tmV, kv_full, 64 * p, h, 64 * kload[hb], b);
+        }
       int issued_o = 0, issued_q = 0;  // steps whose dO / Q copies were issued
       for (int n = 0; n < N; ++n) {
         const int st = n & 1;
         const uint32_t use = (uint32_t)(n >> 1);
-        const int i0 = qit.first_blk + 2 * n;
+        const int i0 = q_first + 2 * n;
         // Both 64-row halves always load (rows past the sequence arrive as
         // zeros), so a stage never holds stale operands; LSE / Delta only
         // exist for blocks inside the sequence.
@@ -351,9 +362,9 @@ __global__ void __launch_bounds__(448, 1)
     const int hf = warp >> 2;
     const int c0 = 64 * hf;
     const int r = (warp & 3) * 32 + lane;  // KV row of the tile == TMEM lane
-    const int kvb = 2 * u + (r >> 6);
+    const int kvb = (r >> 6) ? ky : kx;  // this thread's KV block (-1: none)
     const int rr = r & 63;
-    const bool krow_live = kvb < prm.nqb;
+    const bool krow_live = kvb >= 0;
     const uint32_t t_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const float sl2 = prm.scale_log2;
     constexpr float kLog2e = 1.4426950408889634f;
@@ -361,7 +372,7 @@ __global__ void __launch_bounds__(448, 1)
     for (; n < N; ++n) {
       const int st = n & 1;
       const uint32_t par = (uint32_t)n & 1;
-      const int i = qit.first_blk + 2 * n + hf;  // this warp's query block
+      const int i = q_first + 2 * n + hf;  // this warp's query block
       const bool vis = krow_live && i <= last && in_list(prm.pat, i, kvb);
       const bool diag = (i == kvb);
       if (!__all_sync(0xffffffffu, mbar_wait(&qq_full[st], (uint32_t)(n >> 1) & 1, abort_flag, err, kErrBwdWait)))
@@ -451,7 +462,7 @@ __global__ void __launch_bounds__(448, 1)
     if (ok && prm.grad_f32) {
       // fp32 gradients: each thread stores its part of a KV row straight from TMEM.
       tc_fence_after();
-      const int krow = 128 * u + r;
+      const int krow = kvb >= 0 ? 64 * kvb + (r & 63) : 0;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t tcol = which == 0 ? L::T_DV : L::T_DK;
@@ -462,7 +473,7 @@ __global__ void __launch_bounds__(448, 1)
           const int col = c0 + 32 * q;
           uint32_t o[32];
           tmem_ld32(t_lane + tcol + col, o);
-          if (krow < prm.S) {
+          if (kvb >= 0) {
             float4* d4 = reinterpret_cast<float4*>(dst + col);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
@@ -497,10 +508,11 @@ __global__ void __launch_bounds__(448, 1)
     fence_async_smem();
     named_bar_sync(1, 256);
     if (threadIdx.x == 0 && ok && !prm.grad_f32) {
-      for (int p = 0; p < 2; ++p) {
-        tma_store_4d(&tmdV, smem + L::OFF_V + p * L::PANEL, 64 * p, h, 128 * u, b);
-        tma_store_4d(&tmdK, smem + L::OFF_K + p * L::PANEL, 64 * p, h, 128 * u, b);
-      }
+      for (int hb = 0; hb < (ky >= 0 ? 2 : 1); ++hb)
+        for (int p = 0; p < 2; ++p) {
+          tma_store_4d(&tmdV, smem + L::OFF_V + p * L::PANEL + hb * 8192, 64 * p, h, 64 * kload[hb], b);
+          tma_store_4d(&tmdK, smem + L::OFF_K + p * L::PANEL + hb * 8192, 64 * p, h, 64 * kload[hb], b);
+        }
       bulk_commit();
       bulk_wait_all();
     }
@@ -513,7 +525,7 @@ __global__ void __launch_bounds__(448, 1)
     const int d = quarter * 32 + lane;
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
     for (int n = 0; n < N; ++n) {
-      const int i0 = qit.first_blk + 2 * n;
+      const int i0 = q_first + 2 * n;
       const bool second = i0 + 1 <= last;  // the step's second query block is in the list range
       if (!__all_sync(0xffffffffu, mbar_wait(dq_full, (uint32_t)n & 1, abort_flag, err, kErrBwdWait))) break;
       tc_fence_after();

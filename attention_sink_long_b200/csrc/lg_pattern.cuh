@@ -104,6 +104,54 @@ struct KvChunks {
   }
 };
 
+// The backward's pairing of KV blocks into 128-row tiles. Blocks that every
+// later query sees ("global": sink blocks and strided blocks) come first in
+// ascending order, then the window-only ("local") blocks in ascending order;
+// tile t holds elements 2t and 2t+1 of that sequence. Two global blocks, or two
+// nearby local blocks, share nearly the same query range, so few rows of a
+// tile are masked while the CTA walks it (pairing block 32a with 32a+1 instead
+// would mask half the tile for most queries of a strided pattern).
+struct BlockPairing {
+  int nqb, sink, stride, local;
+  int nG;  // global blocks below nqb
+  LG_HD BlockPairing(const lg_pattern_t& p, int nqb_) : nqb(nqb_), sink(p.sink_blocks), stride(p.stride),
+                                                        local(p.local_blocks) {
+    const int s = imin(imax(sink, 0), nqb);
+    nG = s;
+    if (stride > 0 && s < nqb) nG += ceil_div_nonneg(nqb, stride) - ceil_div_nonneg(s, stride);
+  }
+  LG_HD bool is_global(int kb) const { return kb < sink || (stride > 0 && kb % stride == 0); }
+  LG_HD int tiles() const { return (nqb + 1) / 2; }
+  // n-th global block (n < nG).
+  LG_HD int global_nth(int n) const {
+    const int s = imin(imax(sink, 0), nqb);
+    if (n < s) return n;
+    return (ceil_div_nonneg(s, stride) + (n - s)) * stride;
+  }
+  // n-th local block (n < nqb - nG): blocks >= sink that are not multiples of stride.
+  LG_HD int local_nth(int n) const {
+    const int s = imin(imax(sink, 0), nqb);
+    if (stride <= 0) return s + n;
+    const int m0 = ceil_div_nonneg(s, stride) * stride;  // first multiple >= s
+    if (n < m0 - s) return s + n;
+    n -= m0 - s;
+    // after m0, each period of `stride` blocks holds stride - 1 local blocks
+    return m0 + (n / (stride - 1)) * stride + 1 + n % (stride - 1);
+  }
+  LG_HD int seq(int n) const { return n < nG ? global_nth(n) : local_nth(n - nG); }
+  // Blocks of tile t: *x always, *y = -1 when the tile holds one block.
+  LG_HD void pair(int t, int* x, int* y) const {
+    *x = seq(2 * t);
+    *y = 2 * t + 1 < nqb ? seq(2 * t + 1) : -1;
+  }
+  // Last query block that sees KV block kb.
+  LG_HD int reach(int kb) const {
+    if (is_global(kb)) return nqb - 1;
+    const long long r = (long long)kb + local - 1;
+    return (int)(r < nqb - 1 ? r : nqb - 1);
+  }
+};
+
 // Union of the query-block lists (transpose) of the consecutive KV blocks
 // [j_lo, j_hi], given nqb query blocks. A sink or strided KV block is seen by
 // every later query block; any other by the local_blocks query blocks starting
