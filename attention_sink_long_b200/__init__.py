@@ -356,7 +356,7 @@ def lg_sparse_decode_noalloc(q, k_cache, v_cache, cache_lens, o, lse, scale: flo
 
 # ---------------------------------------------------------------- numerics
 def lg_exp2_device(x, y, method: int, stream=None):
-    """y = 2^x on the device with the softmax's exponential (0: ex2.approx, 1: polynomial)."""
+    """y = 2^x on the device with the softmax's exponential (method 0: ex2.approx)."""
     import torch
 
     _expect(x, "x", torch.float32, tuple(x.shape))

@@ -464,7 +464,7 @@ lg_status_t lg_sparse_decode(const void* q, const void* k_cache, const void* v_c
 // ---------------------------------------------------------------- numerics
 lg_status_t lg_exp2_device(const float* x, float* y, int64_t n, int32_t method, lg_stream_t stream) {
   if (x == nullptr || y == nullptr || n < 0) return LG_ERR_INVALID_ARG;
-  if (method < 0 || method > 2) return LG_ERR_INVALID_ARG;
+  if (method != 0) return LG_ERR_INVALID_ARG;
   if (n == 0) return LG_OK;
   if (n > (int64_t)1 << 40) return LG_ERR_UNSUPPORTED;
   return cuda_status(lg::launch_exp2(x, y, (long long)n, method, static_cast<cudaStream_t>(stream)));

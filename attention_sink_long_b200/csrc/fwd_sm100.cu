@@ -317,11 +317,11 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
         }
       }
       // P = 2^(x * scale * log2 e - m), packed to bf16 and written back over the
-      // first half of this tile's S columns (already read). In every group of
-      // eight columns the last pair -- a quarter -- takes the FMA-pipe
-      // polynomial, the rest the special-function unit, so neither pipe alone
-      // sets the pace; scaling, row sums and the polynomial run on paired
-      // fp32 instructions.
+      // first half of this tile's S columns (already read). All exponentials
+      // run on the special-function unit (measured: moving a share of them to
+      // an FMA-pipe polynomial made this kernel slower -- the softmax is bound
+      // by instruction issue and latency, not by the special-function unit);
+      // scaling and row sums run on paired fp32 instructions.
       const float2 sc2 = make_float2(sl2, sl2);
       const float2 nm2 = make_float2(-m_use, -m_use);
       float2 rs4[4];
@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
             for (int e = 0; e < 64; e += 2) {
               const float2 a = fma2(make_float2(__uint_as_float(xs[64 * hb + e]), __uint_as_float(xs[64 * hb + e + 1])),
                                     sc2, nm2);
-              const float2 pp = ((e & 7) == 6) ? ex2_poly2(a) : make_float2(ex2_approx(a.x), ex2_approx(a.y));
+              const float2 pp = make_float2(ex2_approx(a.x), ex2_approx(a.y));
               rs4[(e >> 1) & 3] = add2(rs4[(e >> 1) & 3], pp);
               pk[e >> 1] = pack_bf16x2(pp.x, pp.y);
             }

@@ -302,27 +302,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for the share of the softmax exponentials that is kept
-// off the special-function unit. Cody-Waite additive range reduction x = n + f
-// with n = round(x) (adding and subtracting 1.5 * 2^23 rounds to an integer)
-// and f in [-1/2, 1/2]; 2^f by a degree-4 polynomial, the Remez minimax fit
-// of the relative error on [-1/2, 1/2] made by csrc/exp2_poly_fit.py (max
-// relative error 2.7e-6 over [-126, 64]); 2^n enters through the exponent
-// bits. Exactly 0 for x <= -127 (masked entries arrive as -inf).
-__device__ __forceinline__ float ex2_poly(float x) {
-  const float xc = fmaxf(x, -127.0f);
-  const float y = xc + 12582912.0f;
-  const float n = y - 12582912.0f;
-  const float f = xc - n;
-  float p = 0.009570102207362652f;
-  p = fmaf(p, f, 0.05591785907745361f);
-  p = fmaf(p, f, 0.240247443318367f);
-  p = fmaf(p, f, 0.6931217908859253f);
-  p = fmaf(p, f, 0.9999992847442627f);
-  const float r = __uint_as_float(__float_as_uint(p) + (__float_as_uint(y) << 23));
-  return xc <= -127.0f ? 0.0f : r;
-}
-
 // Paired fp32 arithmetic (one instruction for two lanes' worth of work).
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
   float2 d;
@@ -346,22 +325,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
-}
-
-// ex2_poly on a pair, with the range reduction and the Horner steps paired.
-__device__ __forceinline__ float2 ex2_poly2(float2 x) {
-  const float2 xc = make_float2(fmaxf(x.x, -127.0f), fmaxf(x.y, -127.0f));
-  const float2 y = add2(xc, make_float2(12582912.0f, 12582912.0f));
-  const float2 n = add2(y, make_float2(-12582912.0f, -12582912.0f));
-  const float2 f = add2(xc, make_float2(-n.x, -n.y));
-  float2 p = make_float2(0.009570102207362652f, 0.009570102207362652f);
-  p = fma2(p, f, make_float2(0.05591785907745361f, 0.05591785907745361f));
-  p = fma2(p, f, make_float2(0.240247443318367f, 0.240247443318367f));
-  p = fma2(p, f, make_float2(0.6931217908859253f, 0.6931217908859253f));
-  p = fma2(p, f, make_float2(0.9999992847442627f, 0.9999992847442627f));
-  const float r0 = __uint_as_float(__float_as_uint(p.x) + (__float_as_uint(y.x) << 23));
-  const float r1 = __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(y.y) << 23));
-  return make_float2(xc.x <= -127.0f ? 0.0f : r0, xc.y <= -127.0f ? 0.0f : r1);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -289,13 +289,10 @@ lg_status_t lg_sparse_decode_noalloc(const void* q, const void* k_cache, const v
 
 /*
  * y[k] = 2^x[k] for k < n, evaluated on the device exactly as the softmax
- * kernels evaluate their exponentials: method 0 is the special-function unit
- * (ex2.approx), method 1 the FMA-pipe polynomial that takes a fixed share of
- * the forward's exponentials (Cody-Waite range reduction + degree-4 Remez
- * minimax polynomial), method 2 the same polynomial in the paired-fp32 form
- * the forward softmax issues (must equal method 1 bit for bit); any other
- * method is LG_ERR_INVALID_ARG. Device pointers x, y of n fp32. For tests of the
- * softmax arithmetic; not on the attention path itself.
+ * kernels evaluate their exponentials: the special-function unit's
+ * ex2.approx (method 0; any other method is LG_ERR_INVALID_ARG). Device
+ * pointers x, y of n fp32. For tests of the softmax arithmetic; not on the
+ * attention path itself.
  */
 lg_status_t lg_exp2_device(const float* x, float* y, int64_t n, int32_t method, lg_stream_t stream);
 
