@@ -255,7 +255,7 @@ lg_status_t lg_sparse_attn_bwd_workspace(const lg_pattern_t* p, int32_t B, int32
   lg_status_t st = check_prefill_shape(p, B, S, H, Hkv, D);
   if (st != LG_OK) return st;
   if (bytes == nullptr) return LG_ERR_INVALID_ARG;
-  *bytes = round256((size_t)B * H * S * D * sizeof(float)) + round256((size_t)B * H * S * sizeof(float));
+  *bytes = round256((size_t)B * H * S * D * sizeof(float)) + 2 * round256((size_t)B * H * S * sizeof(float));
   return LG_OK;
 }
 
@@ -282,6 +282,7 @@ lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* p, const void* q, const void*
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* dq_acc = static_cast<float*>(workspace);
   float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + round256((size_t)B * H * S * D * 4));
+  float* lse2 = reinterpret_cast<float*>(reinterpret_cast<char*>(delta) + round256((size_t)B * H * S * 4));
 
   // Head dim 128 without query-head groups runs the 128-row-step kernel, whose
   // KV tiles are two separately placed 64-row blocks (BlockPairing); the other
@@ -298,12 +299,13 @@ lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* p, const void* q, const void*
   if ((st = make_map(&tdk, grad_f32 ? k : dk, B, S, Hkv, D, kv_box)) != LG_OK) return st;
   if ((st = make_map(&tdv, grad_f32 ? v : dv, B, S, Hkv, D, kv_box)) != LG_OK) return st;
 
-  st = cuda_status(lg::launch_bwd_pre(o, o_dtype == LG_F32, dout, delta, dq_acc, B, S, H, D, s));
+  st = cuda_status(lg::launch_bwd_pre(o, o_dtype == LG_F32, dout, delta, dq_acc, lse, lse2, B, S, H, D, s));
   if (st != LG_OK) return st;
   lg::BwdParams prm;
   prm.pat = *p;
   prm.lse = lse;
   prm.delta = delta;
+  prm.lse2 = lse2;
   prm.dq_acc = dq_acc;
   prm.S = S;
   prm.H = H;

@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(448, 1)
                         64 * (i0 + hb), b);
         for (int hb = 0; hb < nl; ++hb) {
           const size_t row = ((size_t)b * prm.H + h) * prm.S + 64 * (size_t)(i0 + hb);
-          bulk_load(smem + L::OFF_LSE + st * 512 + hb * 256, prm.lse + row, 256, &qq_full[st]);
+          bulk_load(smem + L::OFF_LSE + st * 512 + hb * 256, prm.lse2 + row, 256, &qq_full[st]);
         }
       }
       if (*abort_flag) {
@@ -367,7 +367,6 @@ __global__ void __launch_bounds__(448, 1)
     const bool krow_live = kvb >= 0;
     const uint32_t t_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const float sl2 = prm.scale_log2;
-    constexpr float kLog2e = 1.4426950408889634f;
     int n = 0;
     for (; n < N; ++n) {
       const int st = n & 1;
@@ -391,15 +390,19 @@ __global__ void __launch_bounds__(448, 1)
         uint32_t sr[32];
         tmem_ld32(t_lane + L::T_RS + c0 + 32 * ch, sr);
         if (vis) {
+          // the stage holds LSE in log2 units (preprocess), so one paired FMA
+          // gives the exponent of two columns
+          const float2 sc2 = make_float2(sl2, sl2);
 #pragma unroll
           for (int g = 0; g < 8; ++g) {
             const float4 l4 = lse4[8 * ch + g];
-            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+            const float2 a0 = fma2(make_float2(__uint_as_float(sr[4 * g]), __uint_as_float(sr[4 * g + 1])), sc2,
+                                   make_float2(-l4.x, -l4.y));
+            const float2 a1 = fma2(make_float2(__uint_as_float(sr[4 * g + 2]), __uint_as_float(sr[4 * g + 3])), sc2,
+                                   make_float2(-l4.z, -l4.w));
+            const float pv[4] = {ex2_approx(a0.x), ex2_approx(a0.y), ex2_approx(a1.x), ex2_approx(a1.y)};
 #pragma unroll
-            for (int e = 4 * g; e < 4 * g + 4; ++e) {
-              const float p = ex2_approx(fmaf(__uint_as_float(sr[e]), sl2, -lv[e - 4 * g] * kLog2e));
-              pf[32 * ch + e] = (diag && 32 * ch + e < rr) ? 0.f : p;
-            }
+            for (int e = 4 * g; e < 4 * g + 4; ++e) pf[32 * ch + e] = (diag && 32 * ch + e < rr) ? 0.f : pv[e - 4 * g];
           }
         } else {
 #pragma unroll
@@ -437,9 +440,11 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int k = 32 * ch + 8 * c + 2 * e;
-              const float d0 = pf[k] * (__uint_as_float(dpr[8 * c + 2 * e]) - dl[2 * e]);
-              const float d1 = pf[k + 1] * (__uint_as_float(dpr[8 * c + 2 * e + 1]) - dl[2 * e + 1]);
-              pk[e] = pack_bf16x2(d0, d1);
+              const float2 d = mul2(make_float2(pf[k], pf[k + 1]),
+                                    sub2(make_float2(__uint_as_float(dpr[8 * c + 2 * e]),
+                                                     __uint_as_float(dpr[8 * c + 2 * e + 1])),
+                                         make_float2(dl[2 * e], dl[2 * e + 1])));
+              pk[e] = pack_bf16x2(d.x, d.y);
             }
           } else {
 #pragma unroll

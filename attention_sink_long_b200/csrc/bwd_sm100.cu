@@ -21,6 +21,7 @@ template <int D, bool OF32>
 __global__ void __launch_bounds__(256) lg_bwd_pre_kernel(const void* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dout,
                                                          float* __restrict__ delta, float* __restrict__ dq_acc,
+                                                         const float* __restrict__ lse, float* __restrict__ lse2,
                                                          int B, int S, int H) {
   constexpr int TPR = D / 8;
   const long long rows = (long long)B * S * H;
@@ -61,23 +62,25 @@ __global__ void __launch_bounds__(256) lg_bwd_pre_kernel(const void* __restrict_
     const int b = (int)(bs / S);
     const long long drow = ((long long)b * H + h) * S + s;
     if (c == 0) delta[drow] = acc;
+    if (c == 1) lse2[drow] = lse[drow] * 1.4426950408889634f;  // log2 units, for exp2 in the backward
     float4* z = reinterpret_cast<float4*>(dq_acc + drow * D + 8 * c);
     z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
-cudaError_t launch_bwd_pre(const void* o, int o_f32, const void* dout, float* delta, float* dq_acc, int B, int S,
+cudaError_t launch_bwd_pre(const void* o, int o_f32, const void* dout, float* delta, float* dq_acc, const float* lse,
+                           float* lse2, int B, int S,
                            int H, int D, cudaStream_t stream) {
   const long long threads = (long long)B * S * H * (D / 8);
   const unsigned int blocks = (unsigned int)((threads + 255) / 256);
   const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(dout);
   if (D == 64) {
-    if (o_f32) lg_bwd_pre_kernel<64, true><<<blocks, 256, 0, stream>>>(o, g, delta, dq_acc, B, S, H);
-    else lg_bwd_pre_kernel<64, false><<<blocks, 256, 0, stream>>>(o, g, delta, dq_acc, B, S, H);
+    if (o_f32) lg_bwd_pre_kernel<64, true><<<blocks, 256, 0, stream>>>(o, g, delta, dq_acc, lse, lse2, B, S, H);
+    else lg_bwd_pre_kernel<64, false><<<blocks, 256, 0, stream>>>(o, g, delta, dq_acc, lse, lse2, B, S, H);
   } else {
-    if (o_f32) lg_bwd_pre_kernel<128, true><<<blocks, 256, 0, stream>>>(o, g, delta, dq_acc, B, S, H);
-    else lg_bwd_pre_kernel<128, false><<<blocks, 256, 0, stream>>>(o, g, delta, dq_acc, B, S, H);
+    if (o_f32) lg_bwd_pre_kernel<128, true><<<blocks, 256, 0, stream>>>(o, g, delta, dq_acc, lse, lse2, B, S, H);
+    else lg_bwd_pre_kernel<128, false><<<blocks, 256, 0, stream>>>(o, g, delta, dq_acc, lse, lse2, B, S, H);
   }
   return cudaGetLastError();
 }

@@ -27,6 +27,7 @@ struct BwdParams {
   lg_pattern_t pat;
   const float* lse;      // [B, H, S]
   const float* delta;    // [B, H, S] (workspace, written by the preprocess kernel)
+  const float* lse2;     // [B, H, S] lse * log2(e) (workspace, written by the preprocess kernel)
   float* dq_acc;         // [B, H, S, D] fp32 (workspace)
   int S, H, Hkv, D;
   int nqb;  // S / 64
@@ -42,7 +43,8 @@ struct BwdParams {
   unsigned int* err;
 };
 
-cudaError_t launch_bwd_pre(const void* o, int o_f32, const void* dout, float* delta, float* dq_acc, int B, int S,
+cudaError_t launch_bwd_pre(const void* o, int o_f32, const void* dout, float* delta, float* dq_acc, const float* lse,
+                           float* lse2, int B, int S,
                            int H, int D, cudaStream_t stream);
 cudaError_t launch_bwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv, const BwdParams& prm,

@@ -154,7 +154,7 @@ lg_status_t lg_sparse_attn_fwd(const lg_pattern_t* pattern, const void* q, const
 /* Training backward                                                        */
 /* ------------------------------------------------------------------------ */
 
-/* Workspace bytes for lg_sparse_attn_bwd: fp32 dQ accumulator [B,H,S,D] plus Delta [B,H,S]. */
+/* Workspace bytes for lg_sparse_attn_bwd: fp32 dQ accumulator [B,H,S,D] plus Delta and LSE * log2(e) [B,H,S]. */
 lg_status_t lg_sparse_attn_bwd_workspace(const lg_pattern_t* pattern, int32_t B, int32_t S, int32_t H,
                                          int32_t Hkv, int32_t D, size_t* bytes);
 
