@@ -25,7 +25,7 @@ INT32_MAX = 2**31 - 1
 __all__ = [
     "LgError", "Pattern", "lib", "lg_strerror", "lg_version",
     "lg_pattern_expand", "lg_pattern_expand_t", "lg_pattern_pairs", "lg_pattern_iterate_device",
-    "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd",
+    "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd", "lg_sparse_attn_fwd_varlen",
     "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd",
     "lg_sparse_decode_splits", "lg_sparse_decode_workspace", "lg_sparse_decode",
     "lg_sparse_decode_noalloc", "lg_kv_compact_rows", "lg_kv_compact", "lg_exp2_device", "lg_device_status",
@@ -34,7 +34,7 @@ __all__ = [
 
 EXPORTED_SYMBOLS = (
     "lg_strerror", "lg_version", "lg_pattern_expand", "lg_pattern_expand_t", "lg_pattern_pairs",
-    "lg_pattern_iterate_device", "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd",
+    "lg_pattern_iterate_device", "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd", "lg_sparse_attn_fwd_varlen",
     "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd", "lg_sparse_decode_splits",
     "lg_sparse_decode_workspace", "lg_sparse_decode", "lg_sparse_decode_noalloc", "lg_kv_compact_rows",
     "lg_kv_compact", "lg_exp2_device", "lg_device_status",
@@ -77,6 +77,8 @@ _SIGS = {
     "lg_sparse_attn_fwd_workspace": (_c_i32, [_P(_lg_pattern_t)] + [_c_i32] * 5 + [_P(_c_sz)]),
     "lg_sparse_attn_fwd": (_c_i32, [_P(_lg_pattern_t), _c_vp, _c_vp, _c_vp, _c_vp, _c_i32, _c_vp] + [_c_i32] * 5
                            + [_c_f, _c_vp, _c_sz, _c_vp]),
+    "lg_sparse_attn_fwd_varlen": (_c_i32, [_P(_lg_pattern_t), _c_vp, _c_vp, _c_vp, _c_vp, _c_i32, _c_vp, _c_vp]
+                                  + [_c_i32] * 6 + [_c_f, _c_vp]),
     "lg_sparse_attn_bwd_workspace": (_c_i32, [_P(_lg_pattern_t)] + [_c_i32] * 5 + [_P(_c_sz)]),
     "lg_sparse_attn_bwd": (_c_i32, [_P(_lg_pattern_t)] + [_c_vp] * 4 + [_c_i32] + [_c_vp] * 5 + [_c_i32] * 6
                            + [_c_f, _c_vp, _c_sz, _c_vp]),
@@ -236,6 +238,29 @@ def lg_sparse_attn_fwd(pattern, q, k, v, o, lse, scale: float, workspace=None, s
     _check(lib().lg_sparse_attn_fwd(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), odt,
                                     _ptr(lse), B, S, H, Hkv, D, float(scale), _ptr(workspace), ws, _stream(stream)),
            "lg_sparse_attn_fwd")
+
+
+def lg_sparse_attn_fwd_varlen(pattern, q, k, v, o, lse, cu_seqlens, max_seqlen: int, scale: float, stream=None):
+    """Packed sequences: q [total,H,D], k/v [total,Hkv,D] bf16; o [total,H,D] bf16
+    or fp32 (written); lse [H,total] fp32 or None; cu_seqlens [B+1] int32 on the
+    device; max_seqlen the longest sequence (a multiple of 64)."""
+    import torch
+
+    total, H, D = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    _expect(q, "q", torch.bfloat16, (total, H, D))
+    _expect(k, "k", torch.bfloat16, (total, Hkv, D), q.device)
+    _expect(v, "v", torch.bfloat16, (total, Hkv, D), q.device)
+    odt = _dtype_code(o, "o")
+    _expect(o, "o", o.dtype, (total, H, D), q.device)
+    if lse is not None:
+        _expect(lse, "lse", torch.float32, (H, total), q.device)
+    _expect(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,), q.device)
+    _check(lib().lg_sparse_attn_fwd_varlen(ctypes.byref(_pat(pattern)), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                           o.data_ptr(), odt, _ptr(lse), cu_seqlens.data_ptr(), B, total,
+                                           int(max_seqlen), H, Hkv, D, float(scale), _stream(stream)),
+           "lg_sparse_attn_fwd_varlen")
 
 
 # ---------------------------------------------------------------- backward

@@ -234,7 +234,7 @@ lg_status_t lg_sparse_attn_fwd(const lg_pattern_t* p, const void* q, const void*
   if ((st = make_map(&tv, v, B, S, Hkv, D, 64)) != LG_OK) return st;
   // With an fp32 O the kernel stores rows directly; the bf16 map is then built
   // over q only to have a valid (unused) descriptor.
-  if ((st = make_map(&to, o_dtype == LG_F32 ? q : o, B, S, H, D, 128)) != LG_OK) return st;
+  if ((st = make_map(&to, o_dtype == LG_F32 ? q : o, B, S, H, D, 64)) != LG_OK) return st;
   lg::FwdParams prm;
   prm.pat = *p;
   prm.lse = lse;
@@ -244,6 +244,49 @@ lg_status_t lg_sparse_attn_fwd(const lg_pattern_t* p, const void* q, const void*
   prm.Hkv = Hkv;
   prm.nqb = S / 64;
   prm.nqt = (S + 255) / 256;  // 256-row query spans (two 128-row tiles per CTA)
+  prm.cu_seqlens = nullptr;
+  prm.max_len = S;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.err = err;
+  return cuda_status(lg::launch_fwd(D, tq, tk, tv, to, prm, B, static_cast<cudaStream_t>(stream)));
+}
+
+lg_status_t lg_sparse_attn_fwd_varlen(const lg_pattern_t* p, const void* q, const void* k, const void* v, void* o,
+                                      int32_t o_dtype, float* lse, const int32_t* cu_seqlens, int32_t B,
+                                      int32_t total, int32_t max_seqlen, int32_t H, int32_t Hkv, int32_t D,
+                                      float scale, lg_stream_t stream) {
+  lg_status_t st = check_pattern(p);
+  if (st != LG_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || cu_seqlens == nullptr)
+    return LG_ERR_INVALID_ARG;
+  if (B <= 0 || total <= 0 || max_seqlen <= 0 || H <= 0 || Hkv <= 0 || D <= 0 || H % Hkv != 0)
+    return LG_ERR_INVALID_ARG;
+  if (o_dtype != LG_BF16 && o_dtype != LG_F32) return LG_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return LG_ERR_INVALID_ARG;
+  if (p->block_size != 64 || max_seqlen % 64 != 0 || (D != 64 && D != 128)) return LG_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535 || max_seqlen > total) return LG_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0)
+    return LG_ERR_UNSUPPORTED;
+  unsigned int* err = error_word(&st);
+  if (st != LG_OK) return st;
+  // Packed tensors are one batch of `total` rows to the tensor maps.
+  CUtensorMap tq, tk, tv, to;
+  if ((st = make_map(&tq, q, 1, total, H, D, 128)) != LG_OK) return st;
+  if ((st = make_map(&tk, k, 1, total, Hkv, D, 64)) != LG_OK) return st;
+  if ((st = make_map(&tv, v, 1, total, Hkv, D, 64)) != LG_OK) return st;
+  if ((st = make_map(&to, o_dtype == LG_F32 ? q : o, 1, total, H, D, 64)) != LG_OK) return st;
+  lg::FwdParams prm;
+  prm.pat = *p;
+  prm.lse = lse;
+  prm.o_f32 = o_dtype == LG_F32 ? static_cast<float*>(o) : nullptr;
+  prm.S = total;
+  prm.H = H;
+  prm.Hkv = Hkv;
+  prm.nqb = total / 64;
+  prm.nqt = (max_seqlen + 255) / 256;
+  prm.cu_seqlens = cu_seqlens;
+  prm.max_len = max_seqlen;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.err = err;
   return cuda_status(lg::launch_fwd(D, tq, tk, tv, to, prm, B, static_cast<cudaStream_t>(stream)));

@@ -85,7 +85,26 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const int kvh = h / (prm.H / prm.Hkv);
-  const KvChunks chunks(prm.pat, 4 * span, imin(4 * span + 3, prm.nqb - 1));
+  // Sequence b occupies rows [base, base + len) at tensor-map batch coordinate
+  // bc: the (B, S) layout, or the packed variable-length layout (one batch of
+  // all rows) whose offsets come from cu_seqlens and are checked here; a bad
+  // list is reported and its sequence skipped, never read out of bounds.
+  int len = prm.S, base = 0, bc = b;
+  long long lin0 = (long long)b * prm.S;  // linear row of the sequence's first row
+  if (prm.cu_seqlens != nullptr) {
+    const int s0 = prm.cu_seqlens[b], s1 = prm.cu_seqlens[b + 1];
+    if (s0 < 0 || s1 < s0 || ((s1 - s0) & 63) != 0 || s1 > prm.S || s1 - s0 > prm.max_len) {
+      if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) atomicOr(prm.err, kErrVarlen);
+      return;
+    }
+    len = s1 - s0;
+    base = s0;
+    bc = 0;
+    lin0 = s0;
+  }
+  const int nqb = len / 64;
+  if (span >= (len + 255) / 256) return;  // this span lies past a shorter sequence's end (uniform exit)
+  const KvChunks chunks(prm.pat, 4 * span, imin(4 * span + 3, nqb - 1));
   unsigned int* err = prm.err;
 
   if (threadIdx.x == 0) {
@@ -125,8 +144,8 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
       mbar_arrive_expect_tx(q_full, NT * L::Q_BYTES);
       for (int t = 0; t < NT; ++t)
         for (int p = 0; p < L::DP; ++p)
-          tma_load_4d(smem + L::OFF_Q + t * L::Q_BYTES + p * 16384, &tmQ, q_full, 64 * p, h, 256 * span + 128 * t,
-                      b);
+          tma_load_4d(smem + L::OFF_Q + t * L::Q_BYTES + p * 16384, &tmQ, q_full, 64 * p, h,
+                      base + 256 * span + 128 * t, bc);
       int c = 0;
       int nb = 1;
       for (int j = chunks.first(); j >= 0; ++c) {
@@ -139,12 +158,12 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
         for (int hb = 0; hb < nb; ++hb)
           for (int p = 0; p < L::DP; ++p)
             tma_load_4d(smem + L::OFF_K + st * L::KVC_BYTES + p * 16384 + hb * 8192, &tmK, &k_full[st], 64 * p, kvh,
-                        64 * (hb == 0 ? j : j2), b);
+                        base + 64 * (hb == 0 ? j : j2), bc);
         mbar_arrive_expect_tx(&v_full[st], nb * 64 * D * 2);
         for (int hb = 0; hb < nb; ++hb)
           for (int p = 0; p < L::DP; ++p)
             tma_load_4d(smem + L::OFF_V + st * L::KVC_BYTES + p * 16384 + hb * 8192, &tmV, &v_full[st], 64 * p, kvh,
-                        64 * (hb == 0 ? j : j2), b);
+                        base + 64 * (hb == 0 ? j : j2), bc);
         j = jn;
       }
       if (*abort_flag) {
@@ -242,7 +261,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
     const int r = threadIdx.x & 127;  // tile row == TMEM lane
     const int i = 4 * span + 2 * t + (r >> 6);
     const int rr = r & 63;
-    const bool row_live = i < prm.nqb;
+    const bool row_live = i < nqb;
     uint64_t* s_full = &tile_bars[4 * t + 0];
     uint64_t* p_full = &tile_bars[4 * t + 1];
     uint64_t* pv_done = &tile_bars[4 * t + 2];
@@ -379,12 +398,12 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
     if (ok && prm.o_f32 != nullptr) {
       // fp32 output: each thread stores its row straight from TMEM.
       tc_fence_after();
-      float* dst = prm.o_f32 + (((size_t)b * prm.S + srow) * prm.H + h) * D;
+      float* dst = prm.o_f32 + ((size_t)(lin0 + srow) * prm.H + h) * D;
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t o[32];
         tmem_ld32(t_o + (uint32_t)(32 * ch), o);
-        if (row_live && srow < prm.S) {
+        if (row_live && srow < len) {
           float4* d4 = reinterpret_cast<float4*>(dst + 32 * ch);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
@@ -410,15 +429,21 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
         }
       }
     }
-    if (ok && prm.lse != nullptr && row_live && srow < prm.S) {
+    if (ok && prm.lse != nullptr && row_live && srow < len) {
       const float lse = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-      prm.lse[((size_t)b * prm.H + h) * prm.S + srow] = lse;
+      const size_t li = prm.cu_seqlens != nullptr ? (size_t)h * prm.S + (size_t)(base + srow)
+                                                  : ((size_t)b * prm.H + h) * prm.S + srow;
+      prm.lse[li] = lse;
     }
     fence_async_smem();
     named_bar_sync(1 + t, 128);
-    if (r == 0 && !*abort_flag && prm.o_f32 == nullptr && row0 < prm.S) {
-      for (int p = 0; p < L::DP; ++p)
-        tma_store_4d(&tmO, smem + L::OFF_Q + t * L::Q_BYTES + p * 16384, 64 * p, h, row0, b);
+    if (r == 0 && !*abort_flag && prm.o_f32 == nullptr && row0 < len) {
+      // One 64-row box per block inside the sequence: a box never reaches into
+      // the next sequence of a packed batch.
+      for (int hb = 0; hb < 2 && row0 + 64 * hb < len; ++hb)
+        for (int p = 0; p < L::DP; ++p)
+          tma_store_4d(&tmO, smem + L::OFF_Q + t * L::Q_BYTES + p * 16384 + hb * 8192, 64 * p, h,
+                       base + row0 + 64 * hb, bc);
       bulk_commit();
       bulk_wait_all();
     }

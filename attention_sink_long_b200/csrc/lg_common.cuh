@@ -17,7 +17,7 @@
 namespace lg {
 
 // Device error flags (see lg_device_status).
-enum : uint32_t { kErrFwdWait = 1u, kErrBwdWait = 2u, kErrDecode = 4u, kErrSmemFit = 8u };
+enum : uint32_t { kErrFwdWait = 1u, kErrBwdWait = 2u, kErrDecode = 4u, kErrSmemFit = 8u, kErrVarlen = 16u };
 
 // A bounded wait gives up after this many SM clock cycles (about 2 s at 1.9 GHz).
 constexpr long long kWaitLimitCycles = 4000000000LL;

@@ -11,11 +11,13 @@ namespace lg {
 
 struct FwdParams {
   lg_pattern_t pat;
-  float* lse;    // [B, H, S] or nullptr
+  float* lse;    // [B, H, S] (or [H, total] with cu_seqlens) or nullptr
   float* o_f32;  // [B, S, H, D] fp32 output, or nullptr for the bf16 TMA-stored output
-  int S, H, Hkv;
+  int S, H, Hkv;  // S: rows per sequence; with cu_seqlens the total row count
   int nqb;  // S / 64
-  int nqt;  // ceil(S / 256): CTAs along the sequence
+  int nqt;  // CTAs along the sequence: ceil(S / 256), or ceil(max_len / 256) with cu_seqlens
+  const int32_t* cu_seqlens;  // device [B + 1] sequence offsets (packed layout), or nullptr
+  int max_len;                // with cu_seqlens: the longest sequence the grid covers
   float scale_log2;  // scale * log2(e)
   unsigned int* err;
 };

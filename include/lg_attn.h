@@ -150,6 +150,26 @@ lg_status_t lg_sparse_attn_fwd(const lg_pattern_t* pattern, const void* q, const
                                void* o, int32_t o_dtype, float* lse, int32_t B, int32_t S, int32_t H, int32_t Hkv,
                                int32_t D, float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream);
 
+/*
+ * The forward above for a batch of sequences of different lengths, packed
+ * one after another (the prefill of several prompts; Abstract and summary,
+ * "Key results": 1.67x prefill). Sequence b is rows [cu_seqlens[b],
+ * cu_seqlens[b+1]) of the packed tensors and the pattern applies to positions
+ * inside it (its first row is position 0); no sequence sees another's rows.
+ * Device pointers: q [total,H,D] bf16, k/v [total,Hkv,D] bf16, o [total,H,D]
+ * (written) of element type o_dtype, lse [H,total] fp32 (written; may be
+ * NULL), cu_seqlens [B+1] int32 (read on the device): non-decreasing, starting
+ * at >= 0, ending at <= total, every length a multiple of 64 and at most
+ * max_seqlen (a multiple of 64 that sizes the grid). Rows of o outside every
+ * sequence are not written. A cu_seqlens entry that breaks these rules is
+ * found on the device: that sequence is skipped (its o rows unwritten) and
+ * lg_device_status reports bit 4.
+ */
+lg_status_t lg_sparse_attn_fwd_varlen(const lg_pattern_t* pattern, const void* q, const void* k, const void* v,
+                                      void* o, int32_t o_dtype, float* lse, const int32_t* cu_seqlens, int32_t B,
+                                      int32_t total, int32_t max_seqlen, int32_t H, int32_t Hkv, int32_t D,
+                                      float scale, lg_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Training backward                                                        */
 /* ------------------------------------------------------------------------ */
@@ -304,7 +324,8 @@ lg_status_t lg_exp2_device(const float* x, float* y, int64_t n, int32_t method, 
  * Reads and clears the device-side error flags of the given device (bit 0:
  * a forward wait ran out, bit 1: a backward wait ran out, bit 2: decode,
  * bit 3: a kernel found its shared-memory layout would not fit the block's
- * allocation and did no work). SYNCHRONISES that device. *flags == 0 means
+ * allocation and did no work, bit 4: a variable-length call skipped a
+ * sequence whose offsets broke the rules). SYNCHRONISES that device. *flags == 0 means
  * every kernel since the last call ran to completion.
  */
 lg_status_t lg_device_status(int32_t device, uint32_t* flags);

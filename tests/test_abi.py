@@ -184,3 +184,24 @@ def test_compact_argument_errors():
     assert compact(D=96) == 2
     assert compact(S=1000) == 2
     assert compact(kc=0x30008) == 2         # misaligned
+
+
+def test_fwd_varlen_argument_errors():
+    L = lg.lib()
+    p = lg._lg_pattern_t(64, 1, 4, 0)
+
+    def call(q=0x10000, cu=0x60000, B=2, total=1024, mx=512, H=4, Hkv=4, D=128, odt=0, scale=0.125):
+        return L.lg_sparse_attn_fwd_varlen(ctypes.byref(p), q, 0x20000, 0x30000, 0x40000, odt, 0x50000, cu, B,
+                                           total, mx, H, Hkv, D, scale, None)
+
+    assert call(q=None) == 1
+    assert call(cu=None) == 1
+    assert call(B=0) == 1
+    assert call(H=4, Hkv=3) == 1
+    assert call(odt=3) == 1
+    assert call(scale=-1.0) == 1
+    assert call(mx=500) == 2          # max_seqlen not a multiple of 64
+    assert call(mx=2048) == 2         # longer than the packed tensor
+    assert call(D=96) == 2
+    assert call(q=0x10008) == 2       # misaligned
+    assert call(cu=0x60002) == 2      # misaligned offsets

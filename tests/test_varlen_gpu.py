@@ -1,0 +1,108 @@
+"""Variable-length prefill forward (lg_sparse_attn_fwd_varlen) through the
+C-ABI vs the fp64 oracle, one sequence at a time (the pattern applies inside
+each sequence, positions counted from its first row).
+
+Also: equal-length sequences give bit-for-bit the fixed-length call's O and
+LSE (the same kernel arithmetic); rows outside every sequence are left as
+they were; an offset list that breaks the rules is reported through
+lg_device_status (bit 4) while the valid sequences are still computed.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import attention_sink_long_b200 as lg
+import synthetic_inputs as si
+from parity import assert_close, LSE_TOL
+
+pytestmark = pytest.mark.gpu
+
+SENTINEL = -12345
+
+
+def packed_inputs(lens, H, Hkv, D, seed=0):
+    total = int(sum(lens))
+    q, k, v = si.prefill_inputs(1, total, H, Hkv, D, seed=si.SEED_BASE + 100 + seed)
+    return q[0], k[0], v[0]
+
+
+def run_varlen(pat, q, k, v, cu, max_len, scale, odt=torch.bfloat16):
+    total, H, D = q.shape
+    o = torch.full((total, H, D), SENTINEL, dtype=torch.int16, device="cuda")
+    o = o.view(torch.bfloat16) if odt == torch.bfloat16 else torch.full((total, H, D), float("nan"), device="cuda")
+    lse = torch.full((H, total), float("nan"), dtype=torch.float32, device="cuda")
+    cu_d = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    lg.lg_sparse_attn_fwd_varlen(pat, q.cuda(), k.cuda(), v.cuda(), o, lse, cu_d, max_len, scale)
+    torch.cuda.synchronize()
+    return o, lse
+
+
+CASES = [
+    # lens, H, Hkv, D, pattern, O dtype
+    ([192, 64, 512, 1024, 320], 4, 2, 128, (64, 1, 4, 0), torch.float32),
+    ([256, 640, 128], 2, 2, 128, (64, 1, 2, 4), torch.float32),
+    ([384, 64, 448], 2, 1, 64, (64, 0, 2**31 - 1, 0), torch.float32),
+    ([1024, 512], 4, 4, 128, (64, 1, 4, 0), torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("lens,H,Hkv,D,pat,odt", CASES)
+def test_varlen_matches_oracle_per_sequence(lens, H, Hkv, D, pat, odt):
+    q, k, v = packed_inputs(lens, H, Hkv, D)
+    cu = [0] + list(np.cumsum(lens))
+    scale = 1.0 / math.sqrt(D)
+    o, lse = run_varlen(pat, q, k, v, cu, max(lens), scale, odt)
+    assert lg.lg_device_status(0) == 0
+    p = oracle.Pattern(*pat)
+    for b, n in enumerate(lens):
+        s0, s1 = cu[b], cu[b + 1]
+        ro, rl = oracle.attention_forward(q[None, s0:s1], k[None, s0:s1], v[None, s0:s1], p, scale)
+        assert_close(f"O seq{b}", o[s0:s1].float().cpu().numpy(), ro[0])
+        got_l = lse[:, s0:s1].cpu().numpy()
+        assert np.max(np.abs(got_l - rl[0])) <= LSE_TOL, (b, np.max(np.abs(got_l - rl[0])))
+
+
+def test_equal_lengths_match_the_fixed_length_call_bitwise():
+    B, S, H, Hkv, D = 3, 768, 4, 2, 128
+    pat = (64, 1, 4, 0)
+    scale = 1.0 / math.sqrt(D)
+    q, k, v = si.prefill_inputs(B, S, H, Hkv, D)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o = torch.empty(B, S, H, D, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, H, S, dtype=torch.float32, device="cuda")
+    lg.lg_sparse_attn_fwd(pat, qd, kd, vd, o, lse, scale)
+    ov, lv = run_varlen(pat, q.reshape(B * S, H, D), k.reshape(B * S, Hkv, D), v.reshape(B * S, Hkv, D),
+                        [b * S for b in range(B + 1)], S, scale)
+    assert torch.equal(ov.view(B, S, H, D).view(torch.int16), o.view(torch.int16))
+    assert torch.equal(lv.view(H, B, S).permute(1, 0, 2), lse)
+
+
+def test_rows_outside_every_sequence_are_not_written():
+    lens, H, Hkv, D = [128, 256], 2, 2, 128
+    q, k, v = packed_inputs([64] + lens + [64], H, Hkv, D, seed=1)
+    cu = [64, 64 + 128, 64 + 128 + 256]  # rows [0, 64) and the last 64 rows belong to no sequence
+    o, lse = run_varlen((64, 1, 2, 0), q, k, v, cu, 256, 0.125)
+    assert lg.lg_device_status(0) == 0
+    total = q.shape[0]
+    assert torch.all(o[:64].view(torch.int16) == SENTINEL)
+    assert torch.all(o[total - 64:].view(torch.int16) == SENTINEL)
+    assert torch.all(torch.isnan(lse[:, :64])) and torch.all(torch.isnan(lse[:, total - 64:]))
+    assert not torch.any(o[64:total - 64].view(torch.int16) == SENTINEL)
+
+
+def test_bad_offsets_are_reported_and_skipped():
+    lens, H, Hkv, D = [128, 192, 256], 2, 2, 128
+    q, k, v = packed_inputs(lens, H, Hkv, D, seed=2)
+    cu = [0, 128, 128 + 100, 128 + 192 + 256]  # sequence 1 has 100 rows: not a multiple of 64
+    scale = 0.125
+    o, lse = run_varlen((64, 1, 2, 0), q, k, v, cu, 448, scale)
+    assert lg.lg_device_status(0) & 16
+    assert lg.lg_device_status(0) == 0  # read and cleared
+    p = oracle.Pattern(64, 1, 2, 0)
+    ro, _ = oracle.attention_forward(q[None, :128], k[None, :128], v[None, :128], p, scale)
+    assert_close("O seq0", o[:128].float().cpu().numpy(), ro[0])
+    assert torch.all(o[128:228].view(torch.int16) == SENTINEL)  # the skipped sequence
