@@ -51,7 +51,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
-    ap.add_argument("--workload", choices=["step32k", "fwd128k", "bwd128k", "decode", "handoff", "blocksparse128k"], default="step32k")
+    ap.add_argument("--workload", choices=["step32k", "fwd128k", "bwd128k", "decode", "handoff", "blocksparse128k", "varlen"], default="step32k")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
@@ -152,6 +152,12 @@ def workload(name):
                 "prefill": {"B": 1, "S": 131072, "H": 32, "Hkv": 32, "D": D},
                 "fwd": [("block-sparse", BLOCK_SPARSE)], "bwd": [("block-sparse", BLOCK_SPARSE)],
                 "decode": {"B": 32, "H": 32, "Hkv": 32, "D": D, "L": 5056}}
+    if name == "varlen":
+        return {"workload": "variable-length prefill forward: 8 packed sink+window prompts of 32K..512 tokens "
+                            "(64K rows), H32 D128",
+                "prefill": None, "fwd": [], "bwd": [], "decode": None,
+                "varlen": {"lens": [32768, 16384, 8192, 4096, 2048, 1024, 512, 512], "H": 32, "Hkv": 32, "D": D,
+                           "pattern": SINK_WINDOW}}
     if name == "handoff":
         return {"workload": "prefill->decode hand-off: reduced sink+window KV cache of 32K-token prompts, "
                             "B32 Hkv32 D128",
@@ -282,6 +288,22 @@ class CudaStep:
                                        device=device)
                 fbytes = 2 * B * Lf * Hkv * D * 2 + 2 * B * H * D * 2
                 self.parts.append(("decode full layer", "decode_full", 4 * D * Lf * B * H, fbytes, 1))
+        vl = wl.get("varlen")
+        if vl is not None:
+            lens, H, Hkv, D = vl["lens"], vl["H"], vl["Hkv"], vl["D"]
+            total = sum(lens)
+            self.scale = 1.0 / math.sqrt(D)
+            self.vq = si.device_normal((total, H, D), si.SEED_BASE + 0, device)
+            self.vk = si.device_normal((total, Hkv, D), si.SEED_BASE + 1, device)
+            self.vv = si.device_normal((total, Hkv, D), si.SEED_BASE + 2, device)
+            self.vo = torch.empty_like(self.vq)
+            self.vlse = torch.empty(H, total, dtype=torch.float32, device=device)
+            cu = [0]
+            for n in lens:
+                cu.append(cu[-1] + n)
+            self.vcu = torch.tensor(cu, dtype=torch.int32, device=device)
+            flops = sum(4 * D * pairs_of(vl["pattern"], n) * H for n in lens)
+            self.parts.append(("fwd varlen sink+window", "fwd", flops, None, 1))
         ho = wl.get("handoff")
         if ho is not None:
             B, S, Hkv, D = ho["B"], ho["S"], ho["Hkv"], ho["D"]
@@ -338,6 +360,13 @@ class CudaStep:
                 if events is not None:
                     events[i].record(self.stream)
                 i += 1
+        if wl.get("varlen") is not None:
+            vl = wl["varlen"]
+            lg.lg_sparse_attn_fwd_varlen(vl["pattern"], self.vq, self.vk, self.vv, self.vo, self.vlse, self.vcu,
+                                         max(vl["lens"]), self.scale)
+            if events is not None:
+                events[i].record(self.stream)
+            i += 1
         if wl.get("handoff") is not None:
             lg.lg_kv_compact(wl["handoff"]["pattern"], self.hk, self.hv, self.hkc, self.hvc, self.hlens)
             if events is not None:
@@ -362,14 +391,14 @@ def host_buffers(step):
     torch = step.torch
     pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu())  # noqa: E731
     ins, outs = [], []
-    for name in ("q", "k", "v", "do", "dq_in", "kc", "vc", "lens", "hk", "hv"):
+    for name in ("q", "k", "v", "do", "dq_in", "kc", "vc", "lens", "hk", "hv", "vq", "vk", "vv"):
         if hasattr(step, name):
             ins.append((getattr(step, name), pin(getattr(step, name))))
     for d in ("o", "lse"):
         if hasattr(step, d):
             for t in getattr(step, d).values():
                 outs.append((t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)))
-    for name in ("dq", "dk", "dv", "do_out", "dlse", "hkc", "hvc", "hlens"):
+    for name in ("dq", "dk", "dv", "do_out", "dlse", "hkc", "hvc", "hlens", "vo", "vlse"):
         if hasattr(step, name):
             t = getattr(step, name)
             outs.append((t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)))
@@ -512,6 +541,8 @@ def cuda_arm(args, rank, world, dist):
         config.update({"prefill_shape": pf, "patterns": {n: list(p) for n, p in wl["fwd"] + wl["bwd"]}})
     if wl["decode"]:
         config["decode_shape"] = wl["decode"]
+    if wl.get("varlen"):
+        config["varlen_shape"] = {k: (list(v) if k == "pattern" else v) for k, v in wl["varlen"].items()}
     if wl.get("handoff"):
         config["handoff_shape"] = {k: (list(v) if k == "pattern" else v) for k, v in wl["handoff"].items()}
     line = {
@@ -557,6 +588,15 @@ def oracle_sample(wl, budget_s, seed=11):
             jobs.append(("bwd " + n, "bwd", p))
     if wl["decode"]:
         jobs.append(("decode", "decode", None))
+    vl = wl.get("varlen")
+    if vl:
+        # Forward rows of the longest sequence (the pattern acts inside each sequence alone).
+        S, D = max(vl["lens"]), vl["D"]
+        nqb = S // 64
+        q, k, v = si.prefill_inputs(1, S, 1, 1, D)
+        qh, kh, vh = (t[0, :, 0].double().numpy() for t in (q, k, v))
+        scale = 1.0 / math.sqrt(D)
+        jobs.append(("fwd varlen", "fwd", vl["pattern"]))
     ho = wl.get("handoff")
     if ho:
         # One KV head of one prompt, drawn on the host with the same seed as head 0.
