@@ -28,8 +28,8 @@ __all__ = [
     "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd", "lg_sparse_attn_fwd_varlen",
     "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd",
     "lg_sparse_decode_splits", "lg_sparse_decode_workspace", "lg_sparse_decode",
-    "lg_sparse_decode_noalloc", "lg_kv_compact_rows", "lg_kv_compact", "lg_exp2_device", "lg_device_status",
-    "EXPORTED_SYMBOLS",
+    "lg_sparse_decode_noalloc", "lg_kv_compact_rows", "lg_kv_compact", "lg_exp2_device", "lg_wait_selftest",
+    "lg_device_status", "EXPORTED_SYMBOLS",
 ]
 
 EXPORTED_SYMBOLS = (
@@ -37,7 +37,7 @@ EXPORTED_SYMBOLS = (
     "lg_pattern_iterate_device", "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd", "lg_sparse_attn_fwd_varlen",
     "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd", "lg_sparse_decode_splits",
     "lg_sparse_decode_workspace", "lg_sparse_decode", "lg_sparse_decode_noalloc", "lg_kv_compact_rows",
-    "lg_kv_compact", "lg_exp2_device", "lg_device_status",
+    "lg_kv_compact", "lg_exp2_device", "lg_wait_selftest", "lg_device_status",
 )
 
 
@@ -89,6 +89,7 @@ _SIGS = {
     "lg_kv_compact_rows": (_c_i32, [_P(_lg_pattern_t), _c_i32, _P(_c_i32)]),
     "lg_kv_compact": (_c_i32, [_P(_lg_pattern_t), _c_vp, _c_vp] + [_c_i32] * 4 + [_c_vp, _c_vp, _c_i32, _c_vp, _c_vp]),
     "lg_exp2_device": (_c_i32, [_c_vp, _c_vp, _c_i64, _c_i32, _c_vp]),
+    "lg_wait_selftest": (_c_i32, [_c_i64, _c_vp]),
     "lg_device_status": (_c_i32, [_c_i32, _P(ctypes.c_uint32)]),
 }
 
@@ -391,6 +392,10 @@ def lg_exp2_device(x, y, method: int, stream=None):
 
 
 # ---------------------------------------------------------------- diagnostics
+def lg_wait_selftest(limit_cycles: int, stream=None):
+    """Run the bounded-wait failure path once (sets device error bit 5)."""
+    _check(lib().lg_wait_selftest(int(limit_cycles), _stream(stream)), "lg_wait_selftest")
+
 def lg_device_status(device: int = 0) -> int:
     """Reads and clears the device error flags (synchronises the device)."""
     f = ctypes.c_uint32(0)

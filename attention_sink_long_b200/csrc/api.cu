@@ -507,6 +507,14 @@ lg_status_t lg_sparse_decode(const void* q, const void* k_cache, const void* v_c
 }
 
 // ---------------------------------------------------------------- numerics
+lg_status_t lg_wait_selftest(int64_t limit_cycles, lg_stream_t stream) {
+  if (limit_cycles <= 0 || limit_cycles > 4000000000LL) return LG_ERR_INVALID_ARG;
+  lg_status_t st = LG_OK;
+  unsigned int* err = error_word(&st);
+  if (st != LG_OK) return st;
+  return cuda_status(lg::launch_wait_selftest((long long)limit_cycles, err, static_cast<cudaStream_t>(stream)));
+}
+
 lg_status_t lg_exp2_device(const float* x, float* y, int64_t n, int32_t method, lg_stream_t stream) {
   if (x == nullptr || y == nullptr || n < 0) return LG_ERR_INVALID_ARG;
   if (method != 0) return LG_ERR_INVALID_ARG;

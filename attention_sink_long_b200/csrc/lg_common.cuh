@@ -17,7 +17,14 @@
 namespace lg {
 
 // Device error flags (see lg_device_status).
-enum : uint32_t { kErrFwdWait = 1u, kErrBwdWait = 2u, kErrDecode = 4u, kErrSmemFit = 8u, kErrVarlen = 16u };
+enum : uint32_t {
+  kErrFwdWait = 1u,
+  kErrBwdWait = 2u,
+  kErrDecode = 4u,
+  kErrSmemFit = 8u,
+  kErrVarlen = 16u,
+  kErrSelfTest = 32u
+};
 
 // A bounded wait gives up after this many SM clock cycles (about 2 s at 1.9 GHz).
 constexpr long long kWaitLimitCycles = 4000000000LL;
@@ -57,6 +64,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
+}
+
+// mbar_wait with an explicit limit in cycles (the self-test of the wait path).
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, long long limit) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > limit) return false;
+  }
+  return true;
 }
 
 // Waits for the phase with the given parity to complete. Gives up when another

@@ -86,6 +86,7 @@ struct DecodeParams {
 
 cudaError_t launch_decode(int D, int G, const DecodeParams& prm, cudaStream_t stream);
 
+cudaError_t launch_wait_selftest(long long limit, unsigned int* err, cudaStream_t stream);
 cudaError_t launch_exp2(const float* x, float* y, long long n, int method, cudaStream_t stream);
 
 cudaError_t launch_pattern_iterate(const lg_pattern_t& p, int seqlen, int tile_blocks, int transpose, int32_t* out,

@@ -19,4 +19,21 @@ cudaError_t launch_exp2(const float* x, float* y, long long n, int method, cudaS
   return cudaGetLastError();
 }
 
+// The bounded-wait failure path, end to end: one thread waits on an mbarrier
+// that nothing ever arrives on, gives up after `limit` cycles and records
+// kErrSelfTest in the device error word; the context stays usable.
+__global__ void lg_wait_selftest_kernel(long long limit, unsigned int* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    if (!mbar_wait_limit(&bar, 0, limit)) atomicOr(err, kErrSelfTest);
+  }
+}
+
+cudaError_t launch_wait_selftest(long long limit, unsigned int* err, cudaStream_t stream) {
+  lg_wait_selftest_kernel<<<1, 32, 0, stream>>>(limit, err);
+  return cudaGetLastError();
+}
+
 }  // namespace lg

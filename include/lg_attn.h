@@ -321,11 +321,22 @@ lg_status_t lg_exp2_device(const float* x, float* y, int64_t n, int32_t method, 
 /* ------------------------------------------------------------------------ */
 
 /*
+ * Self-test of the bounded-wait failure path every kernel uses (no passage of
+ * the pages; this is the library's own failure detection): launches one
+ * thread that waits on a barrier nothing arrives on, gives up after
+ * limit_cycles SM cycles (1 .. 4e9) and sets bit 5 of the device error word
+ * (read it with lg_device_status). The device stays usable afterwards.
+ * Errors: LG_ERR_INVALID_ARG (limit out of range), LG_ERR_CUDA.
+ */
+lg_status_t lg_wait_selftest(int64_t limit_cycles, lg_stream_t stream);
+
+/*
  * Reads and clears the device-side error flags of the given device (bit 0:
  * a forward wait ran out, bit 1: a backward wait ran out, bit 2: decode,
  * bit 3: a kernel found its shared-memory layout would not fit the block's
  * allocation and did no work, bit 4: a variable-length call skipped a
- * sequence whose offsets broke the rules). SYNCHRONISES that device. *flags == 0 means
+ * sequence whose offsets broke the rules, bit 5: lg_wait_selftest's wait ran
+ * out, as it should). SYNCHRONISES that device. *flags == 0 means
  * every kernel since the last call ran to completion.
  */
 lg_status_t lg_device_status(int32_t device, uint32_t* flags);

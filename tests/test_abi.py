@@ -205,3 +205,9 @@ def test_fwd_varlen_argument_errors():
     assert call(D=96) == 2
     assert call(q=0x10008) == 2       # misaligned
     assert call(cu=0x60002) == 2      # misaligned offsets
+
+
+def test_wait_selftest_argument_errors():
+    L = lg.lib()
+    assert L.lg_wait_selftest(0, None) == 1
+    assert L.lg_wait_selftest(5_000_000_000, None) == 1
