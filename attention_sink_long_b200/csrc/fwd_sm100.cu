@@ -180,7 +180,10 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp walks the schedule (uniform control flow); one elected
+    // lane issues each MMA and commit.
+    {
+      const uint32_t leader = elect_one();
       constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
       // Operand descriptors are formed once; per MMA only the start-address
       // field moves (it counts 16-byte units in bits [0, 14), and shared
@@ -199,15 +202,15 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
         if (t == 0 && !mbar_wait(&k_full[st], (uint32_t)(c / NS) & 1, abort_flag, err, kErrFwdWait)) return false;
         tc_fence_after();
         const uint32_t idesc = nb == 2 ? idesc_bf16(128, 128, false, false) : idesc_bf16(128, 64, false, false);
-        const uint64_t a0 = opaque_u64(dQ0 + (uint32_t)((t * L::Q_BYTES) >> 4));
-        const uint64_t b0 = opaque_u64(dK0 + (uint32_t)((st * L::KVC_BYTES) >> 4));
+        const uint64_t a0 = dQ0 + (uint32_t)((t * L::Q_BYTES) >> 4);
+        const uint64_t b0 = dK0 + (uint32_t)((st * L::KVC_BYTES) >> 4);
         const uint32_t d = tmem + L::T_S + 128 * t;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-          tc_mma_ss(d, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
+          tc_mma_ss_if(leader, d, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&tile_bars[4 * t + 0]);
+        tc_commit_if(leader, &tile_bars[4 * t + 0]);
         return true;
       };
       // O_t += P_t(c) V(c), K = 64 * nb, P from TMEM. The first 64 KV rows go
@@ -219,21 +222,21 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
         if (!mbar_wait(&tile_bars[4 * t + 3], (uint32_t)c & 1, abort_flag, err, kErrFwdWait)) return false;
         if (t == 0 && !mbar_wait(&v_full[st], (uint32_t)(c / NS) & 1, abort_flag, err, kErrFwdWait)) return false;
         tc_fence_after();
-        const uint64_t b0 = opaque_u64(dV0 + (uint32_t)((st * L::KVC_BYTES) >> 4));
+        const uint64_t b0 = dV0 + (uint32_t)((st * L::KVC_BYTES) >> 4);
         const uint32_t d = tmem + (uint32_t)(t * D);
         const uint32_t a = tmem + L::T_S + 128 * t;
         const uint32_t acc0 = c > 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          tc_mma_ts(d, a + 8 * kk, b0 + (uint32_t)(kk * 2048 >> 4), idesc_pv, kk > 0 ? 1u : acc0);
+          tc_mma_ts_if(leader, d, a + 8 * kk, b0 + (uint32_t)(kk * 2048 >> 4), idesc_pv, kk > 0 ? 1u : acc0);
         if (!mbar_wait(&tile_bars[4 * t + 1], (uint32_t)c & 1, abort_flag, err, kErrFwdWait)) return false;
         tc_fence_after();
         if (nb == 2) {
 #pragma unroll
           for (int kk = 4; kk < 8; ++kk)
-            tc_mma_ts(d, a + 8 * kk, b0 + (uint32_t)(kk * 2048 >> 4), idesc_pv, 1u);
+            tc_mma_ts_if(leader, d, a + 8 * kk, b0 + (uint32_t)(kk * 2048 >> 4), idesc_pv, 1u);
         }
-        tc_commit(&tile_bars[4 * t + 2]);
+        tc_commit_if(leader, &tile_bars[4 * t + 2]);
         return true;
       };
       int nb = 1;
@@ -249,7 +252,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
           if (ok && jn >= 0) ok = issue_s(c + 1, nb_next, t);
         }
         if (!ok) break;
-        tc_commit(&kv_empty[c % NS]);
+        tc_commit_if(leader, &kv_empty[c % NS]);
         j = jn;
         jn = jnn;
         nb = nb_next;
