@@ -232,7 +232,10 @@ __global__ void __launch_bounds__(448, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp walks the schedule (uniform control flow); one elected
+    // lane issues each MMA and commit.
+    {
+      const uint32_t leader = elect_one();
       constexpr uint32_t idesc_kk = idesc_bf16(128, 128, false, false);   // S^T, dP^T
       constexpr uint32_t idesc_kmn = idesc_bf16(128, 128, false, true);   // dV (A in TMEM), dK
       constexpr uint32_t idesc_mnmn = idesc_bf16(128, 128, true, true);   // dQ^T
@@ -247,27 +250,27 @@ __global__ void __launch_bounds__(448, 1)
       const uint64_t dS_mn = sdesc_sw128(sbase + L::OFF_DS, L::PANEL, 1024);
       auto kofs = [](int kk) -> uint32_t { return (uint32_t)(((kk >> 2) * L::PANEL + (kk & 3) * 32) >> 4); };
       auto mofs = [](int kk) -> uint32_t { return (uint32_t)((kk * 2048) >> 4); };
-      auto q_k = [&](int n) { return opaque_u64(sdesc_sw128(sbase + L::OFF_Q + (n & 1) * L::TILE, 16, 1024)); };
-      auto o_k = [&](int n) { return opaque_u64(sdesc_sw128(sbase + L::OFF_DO + (n & 1) * L::TILE, 16, 1024)); };
+      auto q_k = [&](int n) { return sdesc_sw128(sbase + L::OFF_Q + (n & 1) * L::TILE, 16, 1024); };
+      auto o_k = [&](int n) { return sdesc_sw128(sbase + L::OFF_DO + (n & 1) * L::TILE, 16, 1024); };
       auto q_mn = [&](int n) {
-        return opaque_u64(sdesc_sw128(sbase + L::OFF_Q + (n & 1) * L::TILE, L::PANEL, 1024));
+        return sdesc_sw128(sbase + L::OFF_Q + (n & 1) * L::TILE, L::PANEL, 1024);
       };
       auto o_mn = [&](int n) {
-        return opaque_u64(sdesc_sw128(sbase + L::OFF_DO + (n & 1) * L::TILE, L::PANEL, 1024));
+        return sdesc_sw128(sbase + L::OFF_DO + (n & 1) * L::TILE, L::PANEL, 1024);
       };
       // S^T(n) = K Q(n)^T into R_s.
       auto issue_s = [&](int n) {
         const uint64_t q = q_k(n);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          tc_mma_ss(tmem + L::T_RS, dK_k + kofs(kk), q + kofs(kk), idesc_kk, kk > 0 ? 1u : 0u);
+          tc_mma_ss_if(leader, tmem + L::T_RS, dK_k + kofs(kk), q + kofs(kk), idesc_kk, kk > 0 ? 1u : 0u);
       };
       // dP^T(n) = V dO(n)^T into R_d.
       auto issue_dp = [&](int n) {
         const uint64_t o = o_k(n);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          tc_mma_ss(tmem + L::T_RD, dV_k + kofs(kk), o + kofs(kk), idesc_kk, kk > 0 ? 1u : 0u);
+          tc_mma_ss_if(leader, tmem + L::T_RD, dV_k + kofs(kk), o + kofs(kk), idesc_kk, kk > 0 ? 1u : 0u);
       };
       // dV += P^T(n) dO(n); P^T of query columns [64 hf, +64) sits in R_s
       // columns [64 hf, +32), two bf16 per column.
@@ -275,7 +278,7 @@ __global__ void __launch_bounds__(448, 1)
         const uint64_t o = o_mn(n);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          tc_mma_ts(tmem + L::T_DV, tmem + L::T_RS + 64 * (kk >> 2) + 8 * (kk & 3), o + mofs(kk), idesc_kmn,
+          tc_mma_ts_if(leader, tmem + L::T_DV, tmem + L::T_RS + 64 * (kk >> 2) + 8 * (kk & 3), o + mofs(kk), idesc_kmn,
                     (n > 0 || kk > 0) ? 1u : 0u);
       };
       // dK += dS^T(n) Q(n).
@@ -283,14 +286,14 @@ __global__ void __launch_bounds__(448, 1)
         const uint64_t q = q_mn(n);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          tc_mma_ss(tmem + L::T_DK, dS_k + kofs(kk), q + mofs(kk), idesc_kmn, (n > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ss_if(leader, tmem + L::T_DK, dS_k + kofs(kk), q + mofs(kk), idesc_kmn, (n > 0 || kk > 0) ? 1u : 0u);
       };
       // dQ^T(n) = K^T dS^T(n) into R_d (fresh each step).
       auto issue_dq = [&](int n) {
         (void)n;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          tc_mma_ss(tmem + L::T_RD, dK_mn + mofs(kk), dS_mn + mofs(kk), idesc_mnmn, kk > 0 ? 1u : 0u);
+          tc_mma_ss_if(leader, tmem + L::T_RD, dK_mn + mofs(kk), dS_mn + mofs(kk), idesc_mnmn, kk > 0 ? 1u : 0u);
       };
 
       bool ok = mbar_wait(kv_full, 0, abort_flag, err, kErrBwdWait) &&
@@ -298,25 +301,25 @@ __global__ void __launch_bounds__(448, 1)
       if (ok) {
         tc_fence_after();
         issue_s(0);
-        tc_commit(s_full);
+        tc_commit_if(leader, s_full);
         ok = mbar_wait(&qo_full[0], 0, abort_flag, err, kErrBwdWait);
       }
       if (ok) {
         tc_fence_after();
         issue_dp(0);
-        tc_commit(dp_full);
+        tc_commit_if(leader, dp_full);
         ok = mbar_wait(p_full, 0, abort_flag, err, kErrBwdWait);
       }
       if (ok) {
         tc_fence_after();
         issue_dv(0);
-        tc_commit(&qo_empty[0]);
+        tc_commit_if(leader, &qo_empty[0]);
         if (N > 1) {
           ok = mbar_wait(&qq_full[1], 0, abort_flag, err, kErrBwdWait);
           if (ok) {
             tc_fence_after();
             issue_s(1);
-            tc_commit(s_full);
+            tc_commit_if(leader, s_full);
           }
         }
       }
@@ -327,32 +330,32 @@ __global__ void __launch_bounds__(448, 1)
         // dK first: it is Q(n)'s last use, so the refill of that stage with
         // Q(n+2) -- which S^T(n+2) waits for -- starts one GEMM earlier.
         issue_dk(n);
-        tc_commit(&qq_empty[n & 1]);
+        tc_commit_if(leader, &qq_empty[n & 1]);
         issue_dq(n);
-        tc_commit(dq_full);
-        tc_commit(dss_free);
+        tc_commit_if(leader, dq_full);
+        tc_commit_if(leader, dss_free);
         if (n + 1 < N) {
           // R_d takes dP^T(n+1) once the drain warps have read dQ^T(n).
           if (!mbar_wait(dq_free, par, abort_flag, err, kErrBwdWait)) break;
           if (!mbar_wait(&qo_full[(n + 1) & 1], (uint32_t)((n + 1) >> 1) & 1, abort_flag, err, kErrBwdWait)) break;
           tc_fence_after();
           issue_dp(n + 1);
-          tc_commit(dp_full);
+          tc_commit_if(leader, dp_full);
           if (!mbar_wait(p_full, par ^ 1u, abort_flag, err, kErrBwdWait)) break;
           tc_fence_after();
           issue_dv(n + 1);
-          tc_commit(&qo_empty[(n + 1) & 1]);
+          tc_commit_if(leader, &qo_empty[(n + 1) & 1]);
           if (n + 2 < N) {
             // S^T(n+2) overwrites P^T(n+1), which dV(n+1) -- issued just before --
             // reads first; its Q stage was refilled after dK(n) completed.
             if (!mbar_wait(&qq_full[n & 1], (uint32_t)((n + 2) >> 1) & 1, abort_flag, err, kErrBwdWait)) break;
             tc_fence_after();
             issue_s(n + 2);
-            tc_commit(s_full);
+            tc_commit_if(leader, s_full);
           }
         }
       }
-      tc_commit(acc_done);
+      tc_commit_if(leader, acc_done);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ P / dS warps
