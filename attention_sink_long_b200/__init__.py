@@ -28,8 +28,8 @@ __all__ = [
     "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd", "lg_sparse_attn_fwd_varlen",
     "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd",
     "lg_sparse_decode_splits", "lg_sparse_decode_workspace", "lg_sparse_decode",
-    "lg_sparse_decode_noalloc", "lg_kv_compact_rows", "lg_kv_compact", "lg_exp2_device", "lg_wait_selftest",
-    "lg_device_status", "EXPORTED_SYMBOLS",
+    "lg_sparse_decode_noalloc", "lg_kv_compact_rows", "lg_kv_compact", "lg_kv_compact_paged", "lg_kv_append_paged",
+    "lg_sparse_decode_paged", "lg_exp2_device", "lg_wait_selftest", "lg_device_status", "EXPORTED_SYMBOLS",
 ]
 
 EXPORTED_SYMBOLS = (
@@ -37,7 +37,8 @@ EXPORTED_SYMBOLS = (
     "lg_pattern_iterate_device", "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd", "lg_sparse_attn_fwd_varlen",
     "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd", "lg_sparse_decode_splits",
     "lg_sparse_decode_workspace", "lg_sparse_decode", "lg_sparse_decode_noalloc", "lg_kv_compact_rows",
-    "lg_kv_compact", "lg_exp2_device", "lg_wait_selftest", "lg_device_status",
+    "lg_kv_compact", "lg_kv_compact_paged", "lg_kv_append_paged", "lg_sparse_decode_paged", "lg_exp2_device",
+    "lg_wait_selftest", "lg_device_status",
 )
 
 
@@ -88,6 +89,12 @@ _SIGS = {
     "lg_sparse_decode_noalloc": (_c_i32, [_c_vp] * 6 + [_c_i32] * 6 + [_c_f, _c_vp]),
     "lg_kv_compact_rows": (_c_i32, [_P(_lg_pattern_t), _c_i32, _P(_c_i32)]),
     "lg_kv_compact": (_c_i32, [_P(_lg_pattern_t), _c_vp, _c_vp] + [_c_i32] * 4 + [_c_vp, _c_vp, _c_i32, _c_vp, _c_vp]),
+    "lg_kv_compact_paged": (_c_i32, [_P(_lg_pattern_t), _c_vp, _c_vp] + [_c_i32] * 4
+                            + [_c_vp, _c_vp, _c_i64, _c_vp, _c_vp, _c_i32, _c_vp, _c_vp, _c_vp]),
+    "lg_kv_append_paged": (_c_i32, [_P(_lg_pattern_t), _c_vp, _c_vp] + [_c_i32] * 3
+                           + [_c_vp, _c_vp, _c_i64, _c_vp, _c_vp, _c_i32, _c_vp, _c_vp, _c_vp]),
+    "lg_sparse_decode_paged": (_c_i32, [_c_vp, _c_vp, _c_vp, _c_i64, _c_vp, _c_i32, _c_vp, _c_vp, _c_vp]
+                               + [_c_i32] * 5 + [_c_f, _c_vp, _c_sz, _c_vp]),
     "lg_exp2_device": (_c_i32, [_c_vp, _c_vp, _c_i64, _c_i32, _c_vp]),
     "lg_wait_selftest": (_c_i32, [_c_i64, _c_vp]),
     "lg_device_status": (_c_i32, [_c_i32, _P(ctypes.c_uint32)]),
@@ -354,6 +361,80 @@ def lg_kv_compact(pattern, k, v, k_cache, v_cache, cache_lens, stream=None):
     _check(lib().lg_kv_compact(ctypes.byref(_pat(pattern)), k.data_ptr(), v.data_ptr(), B, S, Hkv, D,
                                k_cache.data_ptr(), v_cache.data_ptr(), Lmax, cache_lens.data_ptr(), _stream(stream)),
            "lg_kv_compact")
+
+
+def _expect_paged(k_pool, v_pool, block_table, block_ids, cache_lens, positions, Hkv=None, D=None):
+    import torch
+
+    P = k_pool.shape[0]
+    Hkv = k_pool.shape[2] if Hkv is None else Hkv
+    D = k_pool.shape[3] if D is None else D
+    B, MB = block_table.shape
+    dev = k_pool.device
+    _expect(k_pool, "k_pool", torch.bfloat16, (P, 64, Hkv, D), dev)
+    _expect(v_pool, "v_pool", torch.bfloat16, (P, 64, Hkv, D), dev)
+    _expect(block_table, "block_table", torch.int32, (B, MB), dev)
+    if block_ids is not None:
+        _expect(block_ids, "block_ids", torch.int32, (B, MB), dev)
+    _expect(cache_lens, "cache_lens", torch.int32, (B,), dev)
+    if positions is not None:
+        _expect(positions, "positions", torch.int32, (B,), dev)
+    return P, B, MB, Hkv, D
+
+
+def lg_kv_compact_paged(pattern, k, v, k_pool, v_pool, block_table, block_ids, cache_lens, positions, stream=None):
+    """The reduced cache of each prompt (k, v [B,S,Hkv,D] bf16) into pages:
+    k_pool, v_pool [P,64,Hkv,D] bf16; block_table, block_ids [B,max_blocks],
+    cache_lens, positions [B] int32 (see include/lg_attn.h)."""
+    import torch
+
+    B, S, Hkv, D = k.shape
+    _expect(k, "k", torch.bfloat16, (B, S, Hkv, D))
+    _expect(v, "v", torch.bfloat16, (B, S, Hkv, D), k.device)
+    P, Bt, MB, _, _ = _expect_paged(k_pool, v_pool, block_table, block_ids, cache_lens, positions, Hkv, D)
+    if Bt != B:
+        raise ValueError(f"block_table has {Bt} rows, expected {B}")
+    _check(lib().lg_kv_compact_paged(ctypes.byref(_pat(pattern)), k.data_ptr(), v.data_ptr(), B, S, Hkv, D,
+                                     k_pool.data_ptr(), v_pool.data_ptr(), P, block_table.data_ptr(),
+                                     block_ids.data_ptr(), MB, cache_lens.data_ptr(), positions.data_ptr(),
+                                     _stream(stream)), "lg_kv_compact_paged")
+
+
+def lg_kv_append_paged(pattern, k_new, v_new, k_pool, v_pool, block_table, block_ids, cache_lens, positions,
+                       stream=None):
+    """Append one token per sequence (k_new, v_new [B,Hkv,D] bf16) to a paged cache."""
+    import torch
+
+    B, Hkv, D = k_new.shape
+    _expect(k_new, "k_new", torch.bfloat16, (B, Hkv, D))
+    _expect(v_new, "v_new", torch.bfloat16, (B, Hkv, D), k_new.device)
+    P, Bt, MB, _, _ = _expect_paged(k_pool, v_pool, block_table, block_ids, cache_lens, positions, Hkv, D)
+    if Bt != B:
+        raise ValueError(f"block_table has {Bt} rows, expected {B}")
+    _check(lib().lg_kv_append_paged(ctypes.byref(_pat(pattern)), k_new.data_ptr(), v_new.data_ptr(), B, Hkv, D,
+                                    k_pool.data_ptr(), v_pool.data_ptr(), P, block_table.data_ptr(),
+                                    block_ids.data_ptr(), MB, cache_lens.data_ptr(), positions.data_ptr(),
+                                    _stream(stream)), "lg_kv_append_paged")
+
+
+def lg_sparse_decode_paged(q, k_pool, v_pool, block_table, cache_lens, o, lse, scale: float, num_splits: int = 0,
+                           workspace=None, stream=None):
+    """lg_sparse_decode over a paged cache; workspace as lg_sparse_decode_workspace(..., Lmax=64*max_blocks)."""
+    import torch
+
+    B, H, D = q.shape
+    _expect(q, "q", torch.bfloat16, (B, H, D))
+    P, Bt, MB, Hkv, _ = _expect_paged(k_pool, v_pool, block_table, None, cache_lens, None, None, D)
+    if Bt != B:
+        raise ValueError(f"block_table has {Bt} rows, expected {B}")
+    _expect(o, "o", torch.bfloat16, (B, H, D), q.device)
+    if lse is not None:
+        _expect(lse, "lse", torch.float32, (B, H), q.device)
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().lg_sparse_decode_paged(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), P,
+                                        block_table.data_ptr(), MB, cache_lens.data_ptr(), o.data_ptr(), _ptr(lse),
+                                        B, H, Hkv, D, int(num_splits), float(scale), _ptr(workspace), ws,
+                                        _stream(stream)), "lg_sparse_decode_paged")
 
 
 def lg_sparse_decode_noalloc(q, k_cache, v_cache, cache_lens, o, lse, scale: float, num_splits: int = 0,

@@ -424,6 +424,78 @@ lg_status_t lg_kv_compact(const lg_pattern_t* p, const void* k, const void* v, i
   return cuda_status(lg::launch_compact(k, v, k_cache, v_cache, cache_lens, prm, B, static_cast<cudaStream_t>(stream)));
 }
 
+// Paged cache arguments shared by the paged hand-off, append and decode calls.
+static lg_status_t check_paged(const void* k_pool, const void* v_pool, int64_t num_pages, const int32_t* block_table,
+                               int32_t max_blocks, const int32_t* cache_lens, int32_t B, int32_t Hkv, int32_t D) {
+  if (!k_pool || !v_pool || !block_table || !cache_lens) return LG_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || D <= 0 || num_pages <= 0 || max_blocks <= 0) return LG_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return LG_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv > 65535 || max_blocks > (1 << 24)) return LG_ERR_UNSUPPORTED;
+  if (num_pages > ((int64_t)1 << 31) - 1) return LG_ERR_UNSUPPORTED;
+  if (!aligned16(k_pool) || !aligned16(v_pool) || (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cache_lens) & 3u))
+    return LG_ERR_UNSUPPORTED;
+  return LG_OK;
+}
+
+static lg_status_t paged_state(const lg_pattern_t* p, void* k_pool, void* v_pool, int64_t num_pages,
+                               int32_t* block_table, int32_t* block_ids, int32_t max_blocks, int32_t* cache_lens,
+                               int32_t* positions, int32_t B, int32_t Hkv, int32_t D, lg::PagedCache* pc) {
+  lg_status_t st = check_pattern(p);
+  if (st != LG_OK) return st;
+  if (p->block_size != 64) return LG_ERR_UNSUPPORTED;
+  st = check_paged(k_pool, v_pool, num_pages, block_table, max_blocks, cache_lens, B, Hkv, D);
+  if (st != LG_OK) return st;
+  if (!block_ids || !positions) return LG_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(block_ids) & 3u) || (reinterpret_cast<uintptr_t>(positions) & 3u))
+    return LG_ERR_UNSUPPORTED;
+  pc->k_pool = k_pool;
+  pc->v_pool = v_pool;
+  pc->num_pages = num_pages;
+  pc->block_table = block_table;
+  pc->block_ids = block_ids;
+  pc->max_blocks = max_blocks;
+  pc->cache_lens = cache_lens;
+  pc->positions = positions;
+  pc->row_chunks = (long long)Hkv * D / 8;
+  pc->err = nullptr;
+  return LG_OK;
+}
+
+lg_status_t lg_kv_compact_paged(const lg_pattern_t* p, const void* k, const void* v, int32_t B, int32_t S,
+                                int32_t Hkv, int32_t D, void* k_pool, void* v_pool, int64_t num_pages,
+                                int32_t* block_table, int32_t* block_ids, int32_t max_blocks, int32_t* cache_lens,
+                                int32_t* positions, lg_stream_t stream) {
+  int32_t rows = 0;
+  lg_status_t st = lg_kv_compact_rows(p, S, &rows);
+  if (st != LG_OK) return st;
+  if (!k || !v) return LG_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v)) return LG_ERR_UNSUPPORTED;
+  lg::PagedCache pc;
+  st = paged_state(p, k_pool, v_pool, num_pages, block_table, block_ids, max_blocks, cache_lens, positions, B, Hkv, D,
+                   &pc);
+  if (st != LG_OK) return st;
+  if (rows / 64 > max_blocks) return LG_ERR_CAPACITY;
+  pc.err = error_word(&st);
+  if (st != LG_OK) return st;
+  return cuda_status(lg::launch_compact_paged(k, v, *p, S, pc, B, static_cast<cudaStream_t>(stream)));
+}
+
+lg_status_t lg_kv_append_paged(const lg_pattern_t* p, const void* k_new, const void* v_new, int32_t B, int32_t Hkv,
+                               int32_t D, void* k_pool, void* v_pool, int64_t num_pages, int32_t* block_table,
+                               int32_t* block_ids, int32_t max_blocks, int32_t* cache_lens, int32_t* positions,
+                               lg_stream_t stream) {
+  if (!k_new || !v_new) return LG_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new)) return LG_ERR_UNSUPPORTED;
+  lg::PagedCache pc;
+  lg_status_t st = paged_state(p, k_pool, v_pool, num_pages, block_table, block_ids, max_blocks, cache_lens, positions,
+                               B, Hkv, D, &pc);
+  if (st != LG_OK) return st;
+  pc.err = error_word(&st);
+  if (st != LG_OK) return st;
+  return cuda_status(lg::launch_append_paged(k_new, v_new, *p, pc, B, static_cast<cudaStream_t>(stream)));
+}
+
 // ---------------------------------------------------------------- decode
 lg_status_t lg_sparse_decode_splits(int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax, int32_t num_splits,
                                     int32_t* splits) {
@@ -450,10 +522,11 @@ lg_status_t lg_sparse_decode_workspace(int32_t B, int32_t H, int32_t Hkv, int32_
   return LG_OK;
 }
 
-lg_status_t lg_sparse_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* cache_lens,
-                             void* o, float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax,
-                             int32_t num_splits, float scale, void* workspace, size_t workspace_bytes,
-                             lg_stream_t stream) {
+static lg_status_t decode_common(const void* q, const void* k_cache, const void* v_cache, const int32_t* cache_lens,
+                                 const int32_t* block_table, int32_t max_blocks, int64_t num_pages, void* o,
+                                 float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax,
+                                 int32_t num_splits, float scale, void* workspace, size_t workspace_bytes,
+                                 lg_stream_t stream) {
   if (!q || !k_cache || !v_cache || !cache_lens || !o) return LG_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || Hkv <= 0 || D <= 0 || Lmax <= 0 || num_splits < 0) return LG_ERR_INVALID_ARG;
   if (H % Hkv != 0) return LG_ERR_INVALID_ARG;
@@ -480,6 +553,9 @@ lg_status_t lg_sparse_decode(const void* q, const void* k_cache, const void* v_c
   prm.k_cache = k_cache;
   prm.v_cache = v_cache;
   prm.lens = cache_lens;
+  prm.block_table = block_table;
+  prm.max_blocks = max_blocks;
+  prm.num_pages = num_pages;
   prm.o = o;
   prm.lse = lse;
   prm.part_o = nullptr;
@@ -504,6 +580,24 @@ lg_status_t lg_sparse_decode(const void* q, const void* k_cache, const void* v_c
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.err = err;
   return cuda_status(lg::launch_decode(D, G, prm, s));
+}
+
+lg_status_t lg_sparse_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* cache_lens,
+                             void* o, float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax,
+                             int32_t num_splits, float scale, void* workspace, size_t workspace_bytes,
+                             lg_stream_t stream) {
+  return decode_common(q, k_cache, v_cache, cache_lens, nullptr, 0, 0, o, lse, B, H, Hkv, D, Lmax, num_splits, scale,
+                       workspace, workspace_bytes, stream);
+}
+
+lg_status_t lg_sparse_decode_paged(const void* q, const void* k_pool, const void* v_pool, int64_t num_pages,
+                                   const int32_t* block_table, int32_t max_blocks, const int32_t* cache_lens, void* o,
+                                   float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t num_splits,
+                                   float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream) {
+  lg_status_t st = check_paged(k_pool, v_pool, num_pages, block_table, max_blocks, cache_lens, B, Hkv, D);
+  if (st != LG_OK) return st;
+  return decode_common(q, k_pool, v_pool, cache_lens, block_table, max_blocks, num_pages, o, lse, B, H, Hkv, D,
+                       64 * max_blocks, num_splits, scale, workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------- numerics

@@ -14,6 +14,10 @@
 // CTA, so K/V bytes are read once per KV head. Each CTA reduces its rows to a
 // partial (o, lse); with more than one split the last CTA of each (b, kv head)
 // -- found through an atomic ticket, with no waiting -- merges the partials.
+//
+// Paged caches (PAGED = true): cache row r of sequence b lives in page
+// block_table[b][r / 64] at page row r % 64, every page [64, Hkv, D]; a page
+// index outside the pool is reported (kErrPaged) and its rows are skipped.
 #include "lg_common.cuh"
 #include "lg_kernels.h"
 
@@ -51,7 +55,7 @@ __device__ __forceinline__ void merge_state(float& m, float& l, float (&a)[E], f
   m = mn;
 }
 
-template <int D, int G, int U>
+template <int D, int G, int U, bool PAGED>
 __global__ void __launch_bounds__(128) lg_decode_kernel(const DecodeParams prm) {
   constexpr int TPR = D / 8;     // threads per cache row
   constexpr int RPW = 32 / TPR;  // rows per warp per step
@@ -96,19 +100,31 @@ __global__ void __launch_bounds__(128) lg_decode_kernel(const DecodeParams prm) 
   }
 
   const size_t row_stride = (size_t)prm.Hkv * D;  // elements between consecutive cache rows
-  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(prm.k_cache) +
-                            ((size_t)b * prm.Lmax * prm.Hkv + kvh) * D + 8 * chunk;
-  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(prm.v_cache) +
-                            ((size_t)b * prm.Lmax * prm.Hkv + kvh) * D + 8 * chunk;
+  // Contiguous cache: rows of sequence b from row b * Lmax. Paged: from the pool's base.
+  const size_t seq0 = PAGED ? 0 : (size_t)b * prm.Lmax * prm.Hkv * D;
+  const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(prm.k_cache) + seq0 + (size_t)kvh * D + 8 * chunk;
+  const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(prm.v_cache) + seq0 + (size_t)kvh * D + 8 * chunk;
+  const int32_t* table = PAGED ? prm.block_table + (size_t)b * prm.max_blocks : nullptr;
 
   for (int base = r0; base < r1; base += RSTEP * U) {  // warp-uniform trip count
     uint4 kr[U], vr[U];
+    bool live[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int row = base + slot + u * RSTEP;
-      if (row < r1) {
-        kr[u] = ld_stream_v4(kb + (size_t)row * row_stride);
-        vr[u] = ld_stream_v4(vb + (size_t)row * row_stride);
+      live[u] = row < r1;
+      size_t off = (size_t)row * row_stride;
+      if (PAGED && live[u]) {
+        const int pg = __ldg(table + (row >> 6));
+        if (pg < 0 || (long long)pg >= prm.num_pages) {
+          if (prm.err != nullptr) atomicOr(prm.err, kErrPaged);
+          live[u] = false;
+        }
+        off = ((size_t)pg * 64 + (row & 63)) * row_stride;
+      }
+      if (live[u]) {
+        kr[u] = ld_stream_v4(kb + off);
+        vr[u] = ld_stream_v4(vb + off);
       } else {
         kr[u] = make_uint4(0, 0, 0, 0);
         vr[u] = make_uint4(0, 0, 0, 0);
@@ -127,7 +143,7 @@ __global__ void __launch_bounds__(128) lg_decode_kernel(const DecodeParams prm) 
         for (int e = 0; e < 8; ++e) d = fmaf(qf[g][e], kf[e], d);
 #pragma unroll
         for (int off = TPR / 2; off >= 1; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-        s[u] = (base + slot + u * RSTEP < r1) ? d : -INFINITY;
+        s[u] = live[u] ? d : -INFINITY;
         smax = fmaxf(smax, s[u]);
       }
       const float mn = fmaxf(m[g], smax);
@@ -268,7 +284,10 @@ template <int D, int G>
 static cudaError_t launch_decode_dg(const DecodeParams& prm, cudaStream_t stream) {
   constexpr int U = (G <= 2) ? 4 : 2;
   dim3 grid(prm.ns, prm.Hkv, prm.B);
-  lg_decode_kernel<D, G, U><<<grid, 128, 0, stream>>>(prm);
+  if (prm.block_table != nullptr)
+    lg_decode_kernel<D, G, U, true><<<grid, 128, 0, stream>>>(prm);
+  else
+    lg_decode_kernel<D, G, U, false><<<grid, 128, 0, stream>>>(prm);
   return cudaGetLastError();
 }
 

@@ -23,7 +23,8 @@ enum : uint32_t {
   kErrDecode = 4u,
   kErrSmemFit = 8u,
   kErrVarlen = 16u,
-  kErrSelfTest = 32u
+  kErrSelfTest = 32u,
+  kErrPaged = 64u
 };
 
 // A bounded wait gives up after this many SM clock cycles (about 2 s at 1.9 GHz).

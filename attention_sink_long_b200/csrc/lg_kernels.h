@@ -69,11 +69,34 @@ int compact_blocks(const lg_pattern_t& pat, int S);
 cudaError_t launch_compact(const void* k, const void* v, void* kc, void* vc, int32_t* lens, const CompactParams& prm,
                            int B, cudaStream_t stream);
 
+// Paged decode cache: pools [num_pages, 64, Hkv, D]; per sequence a block table
+// of pages, the pattern block each used entry holds, the cache length and the
+// position of the next token.
+struct PagedCache {
+  void* k_pool;
+  void* v_pool;
+  long long num_pages;
+  int32_t* block_table;  // [B, max_blocks]
+  int32_t* block_ids;    // [B, max_blocks]
+  int max_blocks;
+  int32_t* cache_lens;   // [B]
+  int32_t* positions;    // [B]
+  long long row_chunks;  // 16-byte chunks per token row of all KV heads
+  unsigned int* err;
+};
+cudaError_t launch_compact_paged(const void* k, const void* v, const lg_pattern_t& pat, int S, const PagedCache& pc,
+                                 int B, cudaStream_t stream);
+cudaError_t launch_append_paged(const void* k_new, const void* v_new, const lg_pattern_t& pat, const PagedCache& pc,
+                                int B, cudaStream_t stream);
+
 struct DecodeParams {
   const void* q;        // [B, H, D] bf16
   const void* k_cache;  // [B, Lmax, Hkv, D] bf16
   const void* v_cache;
   const int32_t* lens;  // [B]
+  const int32_t* block_table = nullptr;  // [B, max_blocks] page of each 64-row cache block, or nullptr (contiguous)
+  int max_blocks = 0;
+  long long num_pages = 0;  // pages in the pool (paged cache)
   void* o;              // [B, H, D] bf16
   float* lse;           // [B, H] or nullptr
   float* part_o;        // [B, H, ns, D] fp32 (ns > 1)

@@ -51,7 +51,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
-    ap.add_argument("--workload", choices=["step32k", "fwd128k", "bwd128k", "decode", "handoff", "blocksparse128k", "varlen"], default="step32k")
+    ap.add_argument("--workload", choices=["step32k", "fwd128k", "bwd128k", "decode", "handoff", "blocksparse128k", "varlen", "decode_paged"],
+                    default="step32k")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
@@ -158,6 +159,14 @@ def workload(name):
                 "prefill": None, "fwd": [], "bwd": [], "decode": None,
                 "varlen": {"lens": [32768, 16384, 8192, 4096, 2048, 1024, 512, 512], "H": 32, "Hkv": 32, "D": D,
                            "pattern": SINK_WINDOW}}
+    if name == "decode_paged":
+        # The spec sparse-layer cache (64 sink + 4096 window rows = 4160) reached the way a
+        # server reaches it: hand-off of an 8K prompt into pages, then 64 appended tokens.
+        return {"workload": "paged decode over the sink+window ring cache: B32 H32 D128, 4160 rows per sequence in "
+                            "64-row pages of a shuffled pool (hand-off of 8K prompts + 64 appended tokens)",
+                "prefill": None, "fwd": [], "bwd": [], "decode": None,
+                "paged": {"B": 32, "H": 32, "Hkv": 32, "D": D, "S": 8192, "appended": 64, "L": 4160,
+                          "pattern": SINK_WINDOW}}
     if name == "handoff":
         return {"workload": "prefill->decode hand-off: reduced sink+window KV cache of 32K-token prompts, "
                             "B32 Hkv32 D128",
@@ -304,6 +313,9 @@ class CudaStep:
             self.vcu = torch.tensor(cu, dtype=torch.int32, device=device)
             flops = sum(4 * D * pairs_of(vl["pattern"], n) * H for n in lens)
             self.parts.append(("fwd varlen sink+window", "fwd", flops, None, 1))
+        pg = wl.get("paged")
+        if pg is not None:
+            self._setup_paged(pg, device)
         ho = wl.get("handoff")
         if ho is not None:
             B, S, Hkv, D = ho["B"], ho["S"], ho["Hkv"], ho["D"]
@@ -315,6 +327,41 @@ class CudaStep:
             self.hlens = torch.empty(B, dtype=torch.int32, device=device)
             nbytes = 2 * 2 * B * rows * Hkv * D * 2  # K and V, each row read once and written once
             self.parts.append(("handoff sink+window", "copy", 0, nbytes, 1))
+
+    def _setup_paged(self, pg, device):
+        """Paged ring cache in the state a decode server reaches: lg_kv_compact_paged of a prompt, then
+        lg_kv_append_paged of `appended` tokens; the timed part is lg_sparse_decode_paged."""
+        lg, torch = self.lg, self.torch
+        import synthetic_inputs as si
+
+        B, H, Hkv, D, S, A = pg["B"], pg["H"], pg["Hkv"], pg["D"], pg["S"], pg["appended"]
+        rows = lg.lg_kv_compact_rows(pg["pattern"], S)
+        MB = rows // 64 + 2
+        P = B * MB + B
+        perm = torch.randperm(P, generator=torch.Generator().manual_seed(7))[: B * MB]
+        self.ptable = perm.view(B, MB).to(torch.int32).to(device)
+        self.pids = torch.empty(B, MB, dtype=torch.int32, device=device)
+        self.plens = torch.empty(B, dtype=torch.int32, device=device)
+        self.ppos = torch.empty(B, dtype=torch.int32, device=device)
+        self.kpool = torch.empty(P, 64, Hkv, D, dtype=torch.bfloat16, device=device)
+        self.vpool = torch.empty_like(self.kpool)
+        state = (self.kpool, self.vpool, self.ptable, self.pids, self.plens, self.ppos)
+        k = si.device_normal((B, S + A, Hkv, D), si.SEED_BASE + 1, device)
+        v = si.device_normal((B, S + A, Hkv, D), si.SEED_BASE + 2, device)
+        lg.lg_kv_compact_paged(pg["pattern"], k[:, :S].contiguous(), v[:, :S].contiguous(), *state)
+        for t in range(S, S + A):
+            lg.lg_kv_append_paged(pg["pattern"], k[:, t].contiguous(), v[:, t].contiguous(), *state)
+        del k, v
+        torch.cuda.synchronize()
+        assert int(self.plens.min()) == int(self.plens.max()) == pg["L"], self.plens
+        self.pq = si.device_normal((B, H, D), si.SEED_BASE + 0, device)
+        self.po = torch.empty(B, H, D, dtype=torch.bfloat16, device=device)
+        self.plse = torch.empty(B, H, dtype=torch.float32, device=device)
+        self.pws = torch.empty(max(lg.lg_sparse_decode_workspace(B, H, Hkv, D, 64 * MB), 1), dtype=torch.uint8,
+                               device=device)
+        L = pg["L"]
+        nbytes = 2 * B * L * Hkv * D * 2 + 2 * B * H * D * 2
+        self.parts.append(("decode paged sink+window", "decode", 4 * D * L * B * H, nbytes, 1))
 
     def _bwd_available(self, pf, pattern):
         """One tiny backward call: False when the library reports it unsupported."""
@@ -367,6 +414,12 @@ class CudaStep:
             if events is not None:
                 events[i].record(self.stream)
             i += 1
+        if wl.get("paged") is not None:
+            lg.lg_sparse_decode_paged(self.pq, self.kpool, self.vpool, self.ptable, self.plens, self.po, self.plse,
+                                      1.0 / math.sqrt(wl["paged"]["D"]), workspace=self.pws)
+            if events is not None:
+                events[i].record(self.stream)
+            i += 1
         if wl.get("handoff") is not None:
             lg.lg_kv_compact(wl["handoff"]["pattern"], self.hk, self.hv, self.hkc, self.hvc, self.hlens)
             if events is not None:
@@ -391,14 +444,15 @@ def host_buffers(step):
     torch = step.torch
     pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu())  # noqa: E731
     ins, outs = [], []
-    for name in ("q", "k", "v", "do", "dq_in", "kc", "vc", "lens", "hk", "hv", "vq", "vk", "vv"):
+    for name in ("q", "k", "v", "do", "dq_in", "kc", "vc", "lens", "hk", "hv", "vq", "vk", "vv", "pq", "kpool",
+                 "vpool", "ptable", "plens"):
         if hasattr(step, name):
             ins.append((getattr(step, name), pin(getattr(step, name))))
     for d in ("o", "lse"):
         if hasattr(step, d):
             for t in getattr(step, d).values():
                 outs.append((t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)))
-    for name in ("dq", "dk", "dv", "do_out", "dlse", "hkc", "hvc", "hlens", "vo", "vlse"):
+    for name in ("dq", "dk", "dv", "do_out", "dlse", "hkc", "hvc", "hlens", "vo", "vlse", "po", "plse"):
         if hasattr(step, name):
             t = getattr(step, name)
             outs.append((t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)))
@@ -459,9 +513,9 @@ def cuda_arm(args, rank, world, dist):
     if wl["workload"].startswith("32-layer"):
         # Reported decode step: 21 sparse-layer + 11 full-layer calls, from the per-call times.
         ms_per_step = sum(w * statistics.mean(per_part_ms[i]) for i, w in enumerate(weights))
-    # A workload without FLOPs (the hand-off copy) reports bytes moved per second.
+    # A workload of HBM-bound parts only (decode, the hand-off copy) reports bytes moved per second.
     step_bytes = sum(w * (p[3] or 0) for w, p in zip(weights, step.parts))
-    by_bytes = step_flops == 0
+    by_bytes = work_unit(wl)[0] == "GB/s"
     unit = "GB/s" if by_bytes else "TFLOP/s"
     value = world * (step_bytes / (ms_per_step * 1e-3) / 1e9 if by_bytes else
                      step_flops / (ms_per_step * 1e-3) / 1e12)
@@ -543,6 +597,8 @@ def cuda_arm(args, rank, world, dist):
         config["decode_shape"] = wl["decode"]
     if wl.get("varlen"):
         config["varlen_shape"] = {k: (list(v) if k == "pattern" else v) for k, v in wl["varlen"].items()}
+    if wl.get("paged"):
+        config["paged_shape"] = {k: (list(v) if k == "pattern" else v) for k, v in wl["paged"].items()}
     if wl.get("handoff"):
         config["handoff_shape"] = {k: (list(v) if k == "pattern" else v) for k, v in wl["handoff"].items()}
     line = {
@@ -586,8 +642,11 @@ def oracle_sample(wl, budget_s, seed=11):
             jobs.append(("fwd " + n, "fwd", p))
         for n, p in wl["bwd"]:
             jobs.append(("bwd " + n, "bwd", p))
+    by_bytes = work_unit(wl)[0] == "GB/s"
     if wl["decode"]:
         jobs.append(("decode", "decode", None))
+    if wl.get("paged"):
+        jobs.append(("decode paged", "decode", None))
     vl = wl.get("varlen")
     if vl:
         # Forward rows of the longest sequence (the pattern acts inside each sequence alone).
@@ -624,11 +683,11 @@ def oracle_sample(wl, budget_s, seed=11):
                 kc, vc, rws = oracle.reduced_cache(hk, hv, ho["S"], p)
                 job_flops += 2 * 2 * len(rws) * ho["D"] * 2  # bytes: K and V rows read and written (bf16)
             else:
-                dc = wl["decode"]
+                dc = wl["decode"] or wl["paged"]
                 L, D2 = dc["L"], dc["D"]
                 qq, kc, vc, cl = si.decode_inputs(1, 1, 1, D2, L, seed=1000 + int(rng.integers(0, 1000)))
                 oracle.decode(qq, kc, vc, cl.numpy(), 1.0 / math.sqrt(D2))
-                job_flops += 4 * D2 * L
+                job_flops += 2 * L * D2 * 2 if by_bytes else 4 * D2 * L  # K and V rows of one head (bf16)
             n_done += 1
         dt = time.perf_counter() - t_start
         flops += job_flops
@@ -639,9 +698,10 @@ def oracle_sample(wl, budget_s, seed=11):
 
 
 def work_unit(wl):
-    """(unit, scale) of oracle_sample's work count: FLOPs, or bytes for the hand-off alone."""
-    only_copy = wl.get("handoff") and not (wl["prefill"] or wl["decode"])
-    return ("GB/s", 1e9) if only_copy else ("TFLOP/s", 1e12)
+    """(unit, scale) of the work count: FLOPs, or bytes for workloads of HBM-bound parts only
+    (decode, the hand-off copy)."""
+    hbm_only = not (wl["prefill"] or wl.get("varlen")) and bool(wl["decode"] or wl.get("paged") or wl.get("handoff"))
+    return ("GB/s", 1e9) if hbm_only else ("TFLOP/s", 1e12)
 
 
 def cpu_cores():
@@ -659,7 +719,8 @@ def cpu_baseline(wl, budget_s):
     unit, sc = work_unit(wl)
     return {"value": round(flops / secs / sc, 6), "unit": unit, "cores": cpu_cores(), "kind": "oracle",
             "sample": f"fp64 numpy oracle, {secs:.1f} s: {desc}; useful FLOPs credited 4D/pair fwd, "
-                      f"6D/pair bwd dQ rows, 4D/row decode; hand-off credited its bf16 bytes"}
+                      f"6D/pair bwd dQ rows, 4D/row decode; decode-only and hand-off workloads credited their bf16 "
+                      f"bytes"}
 
 
 def reference_arm(args, rank, world):

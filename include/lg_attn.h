@@ -232,6 +232,53 @@ lg_status_t lg_kv_compact(const lg_pattern_t* pattern, const void* k, const void
                           int32_t Hkv, int32_t D, void* k_cache, void* v_cache, int32_t Lmax, int32_t* cache_lens,
                           lg_stream_t stream);
 
+/*
+ * Paged decode cache (PagedAttention-style block tables, the layout the
+ * pages' vLLM decoding runs on). One page holds one 64-token pattern block
+ * of every KV head: k_pool, v_pool are [num_pages, 64, Hkv, D] bf16. Per
+ * sequence b, all device int32:
+ *   block_table[b, 0..max_blocks)  page indices owned by the sequence. The
+ *       caller assigns them (distinct across sequences; -1 = none). Entries
+ *       [0, n) with n = ceil(cache_lens[b] / 64) hold the cache in ascending
+ *       block order, only entry n-1 may be partial; entries [n, max_blocks)
+ *       are spare pages the sequence takes as it grows. The calls below
+ *       permute the entries they manage.
+ *   block_ids[b, 0..max_blocks)    pattern block index held by each entry
+ *       in [0, n) (written by the calls below).
+ *   cache_lens[b]                  rows in the cache.
+ *   positions[b]                   position of the next token (tokens seen).
+ *
+ * lg_kv_compact_paged: the hand-off of lg_kv_compact into pages. Block i of
+ * the reduced cache goes to page block_table[b][i]; then block_ids[b][i] is
+ * that block, cache_lens[b] = lg_kv_compact_rows(S), positions[b] = S.
+ * Errors: those of lg_kv_compact; LG_ERR_CAPACITY when the reduced cache has
+ * more blocks than max_blocks. A page index outside [0, num_pages) is
+ * reported through lg_device_status (bit 6) and that block is not copied.
+ *
+ * lg_kv_append_paged: appends one token per sequence (k_new, v_new
+ * [B, Hkv, D] bf16, the token at positions[b]) and advances positions[b].
+ * When the token opens a new block qn (position % 64 == 0), the entries whose
+ * block is no longer in qn's list (the block that just left the local
+ * window) are dropped, keeping the others in order, and block qn takes the
+ * first dropped page, else the next spare one: the window's pages are reused
+ * as a ring, so a sink+window layer needs sink_blocks + local_blocks pages
+ * for any length. After the append, the cache of b holds exactly the rows
+ * prefill attention row positions[b]-1 may attend, and lg_sparse_decode_paged
+ * over it gives that row. A state that breaks the rules above (cache_lens and
+ * positions disagreeing modulo 64, cache_lens > positions, no page left, a
+ * page outside the pool) is reported (bit 6) and the sequence left as it was.
+ * Start a sequence with lg_kv_compact_paged, or with cache_lens = positions
+ * = 0.
+ */
+lg_status_t lg_kv_compact_paged(const lg_pattern_t* pattern, const void* k, const void* v, int32_t B, int32_t S,
+                                int32_t Hkv, int32_t D, void* k_pool, void* v_pool, int64_t num_pages,
+                                int32_t* block_table, int32_t* block_ids, int32_t max_blocks, int32_t* cache_lens,
+                                int32_t* positions, lg_stream_t stream);
+lg_status_t lg_kv_append_paged(const lg_pattern_t* pattern, const void* k_new, const void* v_new, int32_t B,
+                               int32_t Hkv, int32_t D, void* k_pool, void* v_pool, int64_t num_pages,
+                               int32_t* block_table, int32_t* block_ids, int32_t max_blocks, int32_t* cache_lens,
+                               int32_t* positions, lg_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Decode over the reduced KV cache                                         */
 /* ------------------------------------------------------------------------ */
@@ -270,6 +317,21 @@ lg_status_t lg_sparse_decode(const void* q, const void* k_cache, const void* v_c
                              void* o, float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax,
                              int32_t num_splits, float scale, void* workspace, size_t workspace_bytes,
                              lg_stream_t stream);
+
+/*
+ * lg_sparse_decode over a paged cache (see lg_kv_compact_paged): cache row r
+ * of sequence b is row r % 64 of page block_table[b][r / 64]. Arguments as
+ * lg_sparse_decode, with Lmax = 64 * max_blocks for the split rule and the
+ * workspace size (lg_sparse_decode_workspace with that Lmax). cache_lens[b] is
+ * clamped to [0, 64 * max_blocks]; a page index outside [0, num_pages) is
+ * reported (bit 6) and its rows left out. Errors: those of lg_sparse_decode,
+ * plus LG_ERR_INVALID_ARG for num_pages or max_blocks <= 0 and
+ * LG_ERR_UNSUPPORTED for max_blocks > 2^24.
+ */
+lg_status_t lg_sparse_decode_paged(const void* q, const void* k_pool, const void* v_pool, int64_t num_pages,
+                                   const int32_t* block_table, int32_t max_blocks, const int32_t* cache_lens, void* o,
+                                   float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t num_splits,
+                                   float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream);
 
 /*
  * Size of the fixed device scratch array behind lg_sparse_decode_noalloc:
@@ -336,7 +398,9 @@ lg_status_t lg_wait_selftest(int64_t limit_cycles, lg_stream_t stream);
  * bit 3: a kernel found its shared-memory layout would not fit the block's
  * allocation and did no work, bit 4: a variable-length call skipped a
  * sequence whose offsets broke the rules, bit 5: lg_wait_selftest's wait ran
- * out, as it should). SYNCHRONISES that device. *flags == 0 means
+ * out, as it should, bit 6: a paged-cache call met a page index outside the
+ * pool, an inconsistent sequence state or a full block table, and skipped
+ * that work). SYNCHRONISES that device. *flags == 0 means
  * every kernel since the last call ran to completion.
  */
 lg_status_t lg_device_status(int32_t device, uint32_t* flags);

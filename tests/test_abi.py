@@ -211,3 +211,54 @@ def test_wait_selftest_argument_errors():
     L = lg.lib()
     assert L.lg_wait_selftest(0, None) == 1
     assert L.lg_wait_selftest(5_000_000_000, None) == 1
+
+
+def test_paged_cache_argument_errors():
+    L = lg.lib()
+    p = lg._lg_pattern_t(64, 1, 64, 0)
+
+    def compact(k=0x10000, kp=0x30000, tbl=0x50000, ids=0x60000, lens=0x70000, pos=0x80000, B=2, S=32768, Hkv=8,
+                D=128, P=256, MB=65, pat=p):
+        return L.lg_kv_compact_paged(ctypes.byref(pat), k, 0x20000, B, S, Hkv, D, kp, 0x40000, P, tbl, ids, MB, lens,
+                                     pos, None)
+
+    assert compact(MB=63) == 6          # 64 blocks do not fit in 63 table entries
+    assert compact(k=None) == 1
+    assert compact(ids=None) == 1
+    assert compact(pos=None) == 1
+    assert compact(P=0) == 1
+    assert compact(MB=0) == 1
+    assert compact(S=1000) == 2
+    assert compact(D=96) == 2
+    assert compact(kp=0x30008) == 2     # misaligned pool
+    assert compact(tbl=0x50002) == 2    # misaligned table
+    assert compact(pat=lg._lg_pattern_t(32, 1, 64, 0)) == 2
+
+    def append(kn=0x10000, kp=0x30000, tbl=0x50000, ids=0x60000, lens=0x70000, pos=0x80000, B=2, Hkv=8, D=128, P=256,
+               MB=65):
+        return L.lg_kv_append_paged(ctypes.byref(p), kn, 0x20000, B, Hkv, D, kp, 0x40000, P, tbl, ids, MB, lens, pos,
+                                    None)
+
+    assert append(kn=None) == 1
+    assert append(tbl=None) == 1
+    assert append(B=0) == 1
+    assert append(MB=-1) == 1
+    assert append(D=80) == 2
+    assert append(kn=0x10004) == 2
+    assert append(MB=(1 << 24) + 1) == 2
+
+    def decode(q=0x10000, kp=0x30000, tbl=0x50000, lens=0x70000, B=2, H=8, Hkv=8, D=128, P=256, MB=65, ns=1,
+               scale=0.088, ws=None, wsb=0):
+        return L.lg_sparse_decode_paged(q, kp, 0x40000, P, tbl, MB, lens, 0x90000, None, B, H, Hkv, D, ns, scale, ws,
+                                        wsb, None)
+
+    assert decode(q=None) == 1
+    assert decode(lens=None) == 1
+    assert decode(P=0) == 1
+    assert decode(MB=0) == 1
+    assert decode(H=8, Hkv=3) == 1
+    assert decode(scale=0.0) == 1
+    assert decode(D=96) == 2
+    assert decode(kp=0x30008) == 2
+    assert decode(MB=(1 << 24) + 1) == 2
+    assert decode(ns=4) == 3            # four splits need a workspace

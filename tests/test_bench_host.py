@@ -77,6 +77,10 @@ def test_workloads_and_useful_work():
     assert bs["decode"]["L"] == lg.lg_kv_compact_rows(bench.BLOCK_SPARSE, bs["prefill"]["S"])
     ho = bench.workload("handoff")["handoff"]
     assert lg.lg_kv_compact_rows(ho["pattern"], ho["S"]) == 4096
+    pg = bench.workload("decode_paged")["paged"]
+    assert lg.lg_kv_compact_rows(pg["pattern"], pg["S"]) + pg["appended"] == pg["L"] == 4160
+    assert bench.work_unit(bench.workload("decode_paged"))[0] == "GB/s"
+    assert bench.work_unit(bench.workload("step32k"))[0] == "TFLOP/s"
 
 
 def _run(cmd, timeout=240):
