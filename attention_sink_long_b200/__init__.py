@@ -26,7 +26,7 @@ __all__ = [
     "LgError", "Pattern", "lib", "lg_strerror", "lg_version",
     "lg_pattern_expand", "lg_pattern_expand_t", "lg_pattern_pairs", "lg_pattern_iterate_device",
     "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd", "lg_sparse_attn_fwd_varlen",
-    "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd",
+    "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd", "lg_sparse_attn_bwd_varlen",
     "lg_sparse_decode_splits", "lg_sparse_decode_workspace", "lg_sparse_decode",
     "lg_sparse_decode_noalloc", "lg_kv_compact_rows", "lg_kv_compact", "lg_kv_compact_paged", "lg_kv_append_paged",
     "lg_sparse_decode_paged", "lg_exp2_device", "lg_wait_selftest", "lg_device_status", "EXPORTED_SYMBOLS",
@@ -35,7 +35,7 @@ __all__ = [
 EXPORTED_SYMBOLS = (
     "lg_strerror", "lg_version", "lg_pattern_expand", "lg_pattern_expand_t", "lg_pattern_pairs",
     "lg_pattern_iterate_device", "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd", "lg_sparse_attn_fwd_varlen",
-    "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd", "lg_sparse_decode_splits",
+    "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd", "lg_sparse_attn_bwd_varlen", "lg_sparse_decode_splits",
     "lg_sparse_decode_workspace", "lg_sparse_decode", "lg_sparse_decode_noalloc", "lg_kv_compact_rows",
     "lg_kv_compact", "lg_kv_compact_paged", "lg_kv_append_paged", "lg_sparse_decode_paged", "lg_exp2_device",
     "lg_wait_selftest", "lg_device_status",
@@ -83,6 +83,8 @@ _SIGS = {
     "lg_sparse_attn_bwd_workspace": (_c_i32, [_P(_lg_pattern_t)] + [_c_i32] * 5 + [_P(_c_sz)]),
     "lg_sparse_attn_bwd": (_c_i32, [_P(_lg_pattern_t)] + [_c_vp] * 4 + [_c_i32] + [_c_vp] * 5 + [_c_i32] * 6
                            + [_c_f, _c_vp, _c_sz, _c_vp]),
+    "lg_sparse_attn_bwd_varlen": (_c_i32, [_P(_lg_pattern_t)] + [_c_vp] * 4 + [_c_i32] + [_c_vp] * 5 + [_c_i32]
+                                  + [_c_vp] + [_c_i32] * 6 + [_c_f, _c_vp, _c_sz, _c_vp]),
     "lg_sparse_decode_splits": (_c_i32, [_c_i32] * 6 + [_P(_c_i32)]),
     "lg_sparse_decode_workspace": (_c_i32, [_c_i32] * 6 + [_P(_c_sz)]),
     "lg_sparse_decode": (_c_i32, [_c_vp] * 6 + [_c_i32] * 6 + [_c_f, _c_vp, _c_sz, _c_vp]),
@@ -303,6 +305,34 @@ def lg_sparse_attn_bwd(pattern, q, k, v, o, dout, lse, dq, dk, dv, scale: float,
                                     dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), gdt,
                                     B, S, H, Hkv, D, float(scale), workspace.data_ptr(), ws, _stream(stream)),
            "lg_sparse_attn_bwd")
+
+
+def lg_sparse_attn_bwd_varlen(pattern, q, k, v, o, dout, lse, dq, dk, dv, cu_seqlens, max_seqlen: int, scale: float,
+                              workspace, stream=None):
+    """Packed sequences (see lg_sparse_attn_fwd_varlen): q, dout, dq [total,H,D];
+    k, v, dk, dv [total,Hkv,D]; o [total,H,D] bf16 or fp32; lse [H,total];
+    workspace of lg_sparse_attn_bwd_workspace(pattern, 1, total, H, Hkv, D) bytes."""
+    import torch
+
+    total, H, D = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    for name, t, shp in (("q", q, (total, H, D)), ("dout", dout, (total, H, D)),
+                         ("k", k, (total, Hkv, D)), ("v", v, (total, Hkv, D))):
+        _expect(t, name, torch.bfloat16, shp, q.device)
+    odt = _dtype_code(o, "o")
+    _expect(o, "o", o.dtype, (total, H, D), q.device)
+    gdt = _dtype_code(dq, "dq")
+    for name, t, shp in (("dq", dq, (total, H, D)), ("dk", dk, (total, Hkv, D)), ("dv", dv, (total, Hkv, D))):
+        _expect(t, name, dq.dtype, shp, q.device)
+    _expect(lse, "lse", torch.float32, (H, total), q.device)
+    _expect(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,), q.device)
+    ws = workspace.numel() * workspace.element_size()
+    _check(lib().lg_sparse_attn_bwd_varlen(ctypes.byref(_pat(pattern)), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                           o.data_ptr(), odt, dout.data_ptr(), lse.data_ptr(), dq.data_ptr(),
+                                           dk.data_ptr(), dv.data_ptr(), gdt, cu_seqlens.data_ptr(), B, total,
+                                           int(max_seqlen), H, Hkv, D, float(scale), workspace.data_ptr(), ws,
+                                           _stream(stream)), "lg_sparse_attn_bwd_varlen")
 
 
 # ---------------------------------------------------------------- decode

@@ -302,12 +302,16 @@ lg_status_t lg_sparse_attn_bwd_workspace(const lg_pattern_t* p, int32_t B, int32
   return LG_OK;
 }
 
-lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* p, const void* q, const void* k, const void* v, const void* o,
-                               int32_t o_dtype, const void* dout, const float* lse, void* dq, void* dk, void* dv,
-                               int32_t grad_dtype, int32_t B, int32_t S, int32_t H, int32_t Hkv, int32_t D,
-                               float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream) {
-  lg_status_t st = check_prefill_shape(p, B, S, H, Hkv, D);
-  if (st != LG_OK) return st;
+// The backward of one (B, S) batch, or of B packed sequences (cu_seqlens given:
+// S = total rows, every tensor one batch of S rows, max_len the longest sequence).
+static lg_status_t bwd_common(const lg_pattern_t* p, const void* q, const void* k, const void* v, const void* o,
+                              int32_t o_dtype, const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                              int32_t grad_dtype, const int32_t* cu_seqlens, int32_t B, int32_t S, int32_t max_len,
+                              int32_t H, int32_t Hkv, int32_t D, float scale, void* workspace, size_t workspace_bytes,
+                              lg_stream_t stream) {
+  const bool varlen = cu_seqlens != nullptr;
+  const int Bm = varlen ? 1 : B;  // batches of the tensors
+  lg_status_t st = LG_OK;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return LG_ERR_INVALID_ARG;
   if (grad_dtype != LG_BF16 && grad_dtype != LG_F32) return LG_ERR_INVALID_ARG;
   if (o_dtype != LG_BF16 && o_dtype != LG_F32) return LG_ERR_INVALID_ARG;
@@ -317,32 +321,31 @@ lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* p, const void* q, const void*
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return LG_ERR_UNSUPPORTED;
   size_t need = 0;
-  lg_sparse_attn_bwd_workspace(p, B, S, H, Hkv, D, &need);
+  lg_sparse_attn_bwd_workspace(p, Bm, S, H, Hkv, D, &need);
   if (workspace == nullptr || workspace_bytes < need) return LG_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LG_ERR_UNSUPPORTED;
   unsigned int* err = error_word(&st);
   if (st != LG_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* dq_acc = static_cast<float*>(workspace);
-  float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + round256((size_t)B * H * S * D * 4));
-  float* lse2 = reinterpret_cast<float*>(reinterpret_cast<char*>(delta) + round256((size_t)B * H * S * 4));
+  float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + round256((size_t)Bm * H * S * D * 4));
+  float* lse2 = reinterpret_cast<float*>(reinterpret_cast<char*>(delta) + round256((size_t)Bm * H * S * 4));
 
   // Head dim 128 without query-head groups runs the 128-row-step kernel, whose
   // KV tiles are two separately placed 64-row blocks (BlockPairing); the other
-  // kernel's tiles are 128 consecutive rows.
+  // kernel's tiles are 128 consecutive rows, also moved as two 64-row boxes.
   const bool paired = (D == 128 && H == Hkv);
-  const int kv_box = paired ? 64 : 128;
   CUtensorMap tq, tk, tv, tdo, tdk, tdv;
-  if ((st = make_map(&tq, q, B, S, H, D, 64)) != LG_OK) return st;
-  if ((st = make_map(&tk, k, B, S, Hkv, D, kv_box)) != LG_OK) return st;
-  if ((st = make_map(&tv, v, B, S, Hkv, D, kv_box)) != LG_OK) return st;
-  if ((st = make_map(&tdo, dout, B, S, H, D, 64)) != LG_OK) return st;
+  if ((st = make_map(&tq, q, Bm, S, H, D, 64)) != LG_OK) return st;
+  if ((st = make_map(&tk, k, Bm, S, Hkv, D, 64)) != LG_OK) return st;
+  if ((st = make_map(&tv, v, Bm, S, Hkv, D, 64)) != LG_OK) return st;
+  if ((st = make_map(&tdo, dout, Bm, S, H, D, 64)) != LG_OK) return st;
   // With fp32 gradients the kernel stores dK / dV directly; the bf16 maps are
   // then built over K / V only to have valid (unused) descriptors.
-  if ((st = make_map(&tdk, grad_f32 ? k : dk, B, S, Hkv, D, kv_box)) != LG_OK) return st;
-  if ((st = make_map(&tdv, grad_f32 ? v : dv, B, S, Hkv, D, kv_box)) != LG_OK) return st;
+  if ((st = make_map(&tdk, grad_f32 ? k : dk, Bm, S, Hkv, D, 64)) != LG_OK) return st;
+  if ((st = make_map(&tdv, grad_f32 ? v : dv, Bm, S, Hkv, D, 64)) != LG_OK) return st;
 
-  st = cuda_status(lg::launch_bwd_pre(o, o_dtype == LG_F32, dout, delta, dq_acc, lse, lse2, B, S, H, D, s));
+  st = cuda_status(lg::launch_bwd_pre(o, o_dtype == LG_F32, dout, delta, dq_acc, lse, lse2, Bm, S, H, D, s));
   if (st != LG_OK) return st;
   lg::BwdParams prm;
   prm.pat = *p;
@@ -354,8 +357,10 @@ lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* p, const void* q, const void*
   prm.H = H;
   prm.Hkv = Hkv;
   prm.D = D;
-  prm.nqb = S / 64;
-  prm.nkt = (S + 127) / 128;
+  prm.nqb = max_len / 64;  // the launch order is laid out for the longest sequence
+  prm.nkt = (max_len + 127) / 128;
+  prm.cu_seqlens = cu_seqlens;
+  prm.max_len = max_len;
   prm.scale = scale;
   prm.scale_log2 = scale * 1.4426950408889634f;
   // Heavy KV tiles: query-list length above twice the median (e.g. the sink
@@ -391,7 +396,35 @@ lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* p, const void* q, const void*
   prm.err = err;
   st = cuda_status(lg::launch_bwd(D, tq, tk, tv, tdo, tdk, tdv, prm, B, s));
   if (st != LG_OK) return st;
-  return cuda_status(lg::launch_bwd_dq(dq_acc, dq, grad_f32, scale, B, S, H, D, s));
+  return cuda_status(lg::launch_bwd_dq(dq_acc, dq, grad_f32, scale, Bm, S, H, D, s));
+}
+
+lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* p, const void* q, const void* k, const void* v, const void* o,
+                               int32_t o_dtype, const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                               int32_t grad_dtype, int32_t B, int32_t S, int32_t H, int32_t Hkv, int32_t D,
+                               float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream) {
+  lg_status_t st = check_prefill_shape(p, B, S, H, Hkv, D);
+  if (st != LG_OK) return st;
+  return bwd_common(p, q, k, v, o, o_dtype, dout, lse, dq, dk, dv, grad_dtype, nullptr, B, S, S, H, Hkv, D, scale,
+                    workspace, workspace_bytes, stream);
+}
+
+lg_status_t lg_sparse_attn_bwd_varlen(const lg_pattern_t* p, const void* q, const void* k, const void* v,
+                                      const void* o, int32_t o_dtype, const void* dout, const float* lse, void* dq,
+                                      void* dk, void* dv, int32_t grad_dtype, const int32_t* cu_seqlens, int32_t B,
+                                      int32_t total, int32_t max_seqlen, int32_t H, int32_t Hkv, int32_t D,
+                                      float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream) {
+  lg_status_t st = check_pattern(p);
+  if (st != LG_OK) return st;
+  if (cu_seqlens == nullptr) return LG_ERR_INVALID_ARG;
+  if (B <= 0 || total <= 0 || max_seqlen <= 0 || H <= 0 || Hkv <= 0 || D <= 0 || H % Hkv != 0)
+    return LG_ERR_INVALID_ARG;
+  if (p->block_size != 64 || max_seqlen % 64 != 0 || total % 4 != 0 || (D != 64 && D != 128))
+    return LG_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535 || max_seqlen > total) return LG_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return LG_ERR_UNSUPPORTED;
+  return bwd_common(p, q, k, v, o, o_dtype, dout, lse, dq, dk, dv, grad_dtype, cu_seqlens, B, total, max_seqlen, H,
+                    Hkv, D, scale, workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------- prefill -> decode hand-off

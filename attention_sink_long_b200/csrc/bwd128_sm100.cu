@@ -132,12 +132,34 @@ __global__ void __launch_bounds__(448, 1)
     }
   }
   const int b = blockIdx.y;
+  // Sequence b occupies rows [base, base + len) at tensor-map batch coordinate
+  // bc: the (B, S) layout, or the packed variable-length layout whose offsets
+  // come from cu_seqlens and are checked here (a bad list is reported and its
+  // sequence skipped). Per head, LSE, Delta and dQ-accumulator rows of the
+  // sequence start at hrow0 + h * S; its dK / dV rows at lin0.
+  int len = prm.S, base = 0, bc = b;
+  if (prm.cu_seqlens != nullptr) {
+    const int s0 = prm.cu_seqlens[b], s1 = prm.cu_seqlens[b + 1];
+    // (s0 % 4 == 0 keeps the 64-row LSE / Delta copies 16-byte aligned.)
+    if (s0 < 0 || (s0 & 3) != 0 || s1 < s0 || ((s1 - s0) & 63) != 0 || s1 > prm.S || s1 - s0 > prm.max_len) {
+      if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(prm.err, kErrVarlen);
+      return;
+    }
+    len = s1 - s0;
+    base = s0;
+    bc = 0;
+  }
+  const int nqb = len / 64;
+  const size_t hrow0 = prm.cu_seqlens != nullptr ? (size_t)base : (size_t)b * prm.H * prm.S;
+  const long long lin0 = prm.cu_seqlens != nullptr ? (long long)base : (long long)b * prm.S;
   // The tile's two KV blocks (ky = -1: the tile holds one block; its rows
-  // 64..127 load past the sequence end, i.e. as zeros, and stay masked).
-  const BlockPairing bp(prm.pat, prm.nqb);
+  // 64..127 load past the sequence end -- zeros, or the next packed sequence's
+  // rows -- stay masked and are never stored).
+  const BlockPairing bp(prm.pat, nqb);
+  if (u >= bp.tiles()) return;  // past a shorter sequence's last tile (uniform exit)
   int kx, ky;
   bp.pair(u, &kx, &ky);
-  const int kload[2] = {kx, ky >= 0 ? ky : prm.nqb};
+  const int kload[2] = {kx, ky >= 0 ? ky : nqb};
   // Query blocks [q_first, last] see the tile (the union of both blocks' lists).
   const int q_first = ky >= 0 ? imin(kx, ky) : kx;
   const int last = ky >= 0 ? imax(bp.reach(kx), bp.reach(ky)) : bp.reach(kx);
@@ -178,8 +200,8 @@ __global__ void __launch_bounds__(448, 1)
       mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
       for (int hb = 0; hb < 2; ++hb)
         for (int p = 0; p < 2; ++p) {
-          tma_load_4d(smem + L::OFF_K + p * L::PANEL + hb * 8192, &tmK, kv_full, 64 * p, h, 64 * kload[hb], b);
-          tma_load_4d(smem + L::OFF_V + p * L::PANEL + hb * 8192, &tmV, kv_full, 64 * p, h, 64 * kload[hb], b);
+          tma_load_4d(smem + L::OFF_K + p * L::PANEL + hb * 8192, &tmK, kv_full, 64 * p, h, base + 64 * kload[hb], bc);
+          tma_load_4d(smem + L::OFF_V + p * L::PANEL + hb * 8192, &tmV, kv_full, 64 * p, h, base + 64 * kload[hb], bc);
         }
       int issued_o = 0, issued_q = 0;  // steps whose dO / Q copies were issued
       for (int n = 0; n < N; ++n) {
@@ -189,16 +211,16 @@ __global__ void __launch_bounds__(448, 1)
         // Both 64-row halves always load (rows past the sequence arrive as
         // zeros), so a stage never holds stale operands; LSE / Delta only
         // exist for blocks inside the sequence.
-        const int nl = (i0 + 1 < prm.nqb) ? 2 : 1;
+        const int nl = (i0 + 1 < nqb) ? 2 : 1;
         if (use > 0 && !mbar_wait(&qo_empty[st], (use - 1) & 1, abort_flag, err, kErrBwdWait)) break;
         mbar_arrive_expect_tx(&qo_full[st], L::TILE + nl * 256);
         issued_o = n + 1;
         for (int hb = 0; hb < 2; ++hb)
           for (int p = 0; p < 2; ++p)
             tma_load_4d(smem + L::OFF_DO + st * L::TILE + p * L::PANEL + hb * 8192, &tmdO, &qo_full[st], 64 * p, h,
-                        64 * (i0 + hb), b);
+                        base + 64 * (i0 + hb), bc);
         for (int hb = 0; hb < nl; ++hb) {
-          const size_t row = ((size_t)b * prm.H + h) * prm.S + 64 * (size_t)(i0 + hb);
+          const size_t row = hrow0 + (size_t)h * prm.S + 64 * (size_t)(i0 + hb);
           bulk_load(smem + L::OFF_DEL + st * 512 + hb * 256, prm.delta + row, 256, &qo_full[st]);
         }
         if (use > 0 && !mbar_wait(&qq_empty[st], (use - 1) & 1, abort_flag, err, kErrBwdWait)) break;
@@ -207,9 +229,9 @@ __global__ void __launch_bounds__(448, 1)
         for (int hb = 0; hb < 2; ++hb)
           for (int p = 0; p < 2; ++p)
             tma_load_4d(smem + L::OFF_Q + st * L::TILE + p * L::PANEL + hb * 8192, &tmQ, &qq_full[st], 64 * p, h,
-                        64 * (i0 + hb), b);
+                        base + 64 * (i0 + hb), bc);
         for (int hb = 0; hb < nl; ++hb) {
-          const size_t row = ((size_t)b * prm.H + h) * prm.S + 64 * (size_t)(i0 + hb);
+          const size_t row = hrow0 + (size_t)h * prm.S + 64 * (size_t)(i0 + hb);
           bulk_load(smem + L::OFF_LSE + st * 512 + hb * 256, prm.lse2 + row, 256, &qq_full[st]);
         }
       }
@@ -475,7 +497,7 @@ __global__ void __launch_bounds__(448, 1)
       for (int which = 0; which < 2; ++which) {
         const uint32_t tcol = which == 0 ? L::T_DV : L::T_DK;
         const float mul = which == 0 ? 1.f : prm.scale;
-        float* dst = (which == 0 ? prm.dv_f32 : prm.dk_f32) + (((size_t)b * prm.S + krow) * prm.Hkv + h) * L::D;
+        float* dst = (which == 0 ? prm.dv_f32 : prm.dk_f32) + (((size_t)lin0 + krow) * prm.Hkv + h) * L::D;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const int col = c0 + 32 * q;
@@ -518,8 +540,8 @@ __global__ void __launch_bounds__(448, 1)
     if (threadIdx.x == 0 && ok && !prm.grad_f32) {
       for (int hb = 0; hb < (ky >= 0 ? 2 : 1); ++hb)
         for (int p = 0; p < 2; ++p) {
-          tma_store_4d(&tmdV, smem + L::OFF_V + p * L::PANEL + hb * 8192, 64 * p, h, 64 * kload[hb], b);
-          tma_store_4d(&tmdK, smem + L::OFF_K + p * L::PANEL + hb * 8192, 64 * p, h, 64 * kload[hb], b);
+          tma_store_4d(&tmdV, smem + L::OFF_V + p * L::PANEL + hb * 8192, 64 * p, h, base + 64 * kload[hb], bc);
+          tma_store_4d(&tmdK, smem + L::OFF_K + p * L::PANEL + hb * 8192, 64 * p, h, base + 64 * kload[hb], bc);
         }
       bulk_commit();
       bulk_wait_all();
@@ -537,7 +559,7 @@ __global__ void __launch_bounds__(448, 1)
       const bool second = i0 + 1 <= last;  // the step's second query block is in the list range
       if (!__all_sync(0xffffffffu, mbar_wait(dq_full, (uint32_t)n & 1, abort_flag, err, kErrBwdWait))) break;
       tc_fence_after();
-      float* dst = prm.dq_acc + (((size_t)b * prm.H + h) * prm.S + 64 * (size_t)i0) * L::D + d;
+      float* dst = prm.dq_acc + (hrow0 + (size_t)h * prm.S + 64 * (size_t)i0) * L::D + d;
       // Read all 128 columns first, so R_d is released before any reduction is
       // issued (the reductions run at the L2's rate and would otherwise hold
       // up the next dP^T).

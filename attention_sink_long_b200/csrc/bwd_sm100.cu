@@ -247,10 +247,31 @@ __global__ void __launch_bounds__(448, 1)
     }
   }
   const int b = blockIdx.y;
+  // Sequence b occupies rows [base, base + len) at tensor-map batch coordinate
+  // bc: the (B, S) layout, or the packed variable-length layout whose offsets
+  // come from cu_seqlens and are checked here (a bad list is reported and its
+  // sequence skipped). Per head, LSE, Delta and dQ-accumulator rows of the
+  // sequence start at hrow0 + h * S; its dK / dV rows at lin0.
+  int len = prm.S, base = 0, bc = b;
+  if (prm.cu_seqlens != nullptr) {
+    const int s0 = prm.cu_seqlens[b], s1 = prm.cu_seqlens[b + 1];
+    // (s0 % 4 == 0 keeps the 64-row LSE / Delta copies 16-byte aligned.)
+    if (s0 < 0 || (s0 & 3) != 0 || s1 < s0 || ((s1 - s0) & 63) != 0 || s1 > prm.S || s1 - s0 > prm.max_len) {
+      if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(prm.err, kErrVarlen);
+      return;
+    }
+    len = s1 - s0;
+    base = s0;
+    bc = 0;
+  }
+  const int nqb = len / 64;
+  const size_t hrow0 = prm.cu_seqlens != nullptr ? (size_t)base : (size_t)b * prm.H * prm.S;
+  const long long lin0 = prm.cu_seqlens != nullptr ? (long long)base : (long long)b * prm.S;
   const int G = prm.H / prm.Hkv;
   const int j_lo = 2 * u;
-  const int j_hi = imin(2 * u + 1, prm.nqb - 1);
-  const QIter qit(prm.pat, j_lo, j_hi, prm.nqb);
+  if (j_lo >= nqb) return;  // past a shorter sequence's last tile (uniform exit)
+  const int j_hi = imin(2 * u + 1, nqb - 1);
+  const QIter qit(prm.pat, j_lo, j_hi, nqb);
   const int cnt = qit.count();
   const int N = G * cnt;
   constexpr bool split = SPLIT;
@@ -290,10 +311,14 @@ __global__ void __launch_bounds__(448, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       mbar_arrive_expect_tx(kv_full, 2 * L::KV_BYTES);
-      for (int p = 0; p < DP; ++p) {
-        tma_load_4d(smem + L::OFF_K + p * 16384, &tmK, kv_full, 64 * p, kvh, 128 * u, b);
-        tma_load_4d(smem + L::OFF_V + p * 16384, &tmV, kv_full, 64 * p, kvh, 128 * u, b);
-      }
+      // Two 64-row boxes per panel; rows past the sequence stay masked.
+      for (int hb = 0; hb < 2; ++hb)
+        for (int p = 0; p < DP; ++p) {
+          tma_load_4d(smem + L::OFF_K + p * 16384 + hb * 8192, &tmK, kv_full, 64 * p, kvh, base + 128 * u + 64 * hb,
+                      bc);
+          tma_load_4d(smem + L::OFF_V + p * 16384 + hb * 8192, &tmV, kv_full, 64 * p, kvh, base + 128 * u + 64 * hb,
+                      bc);
+        }
       for (int n = 0; n < N; ++n) {
         const int h = kvh * G + n / cnt;
         const int i = qit.first_blk + n % cnt;
@@ -302,10 +327,10 @@ __global__ void __launch_bounds__(448, 1)
         if (use > 0 && !mbar_wait(&q_empty[st], (use - 1) & 1, abort_flag, err, kErrBwdWait)) break;
         mbar_arrive_expect_tx(&q_full[st], 2 * L::QB_BYTES + 512);
         for (int p = 0; p < DP; ++p) {
-          tma_load_4d(smem + L::OFF_Q + st * L::QB_BYTES + p * 8192, &tmQ, &q_full[st], 64 * p, h, 64 * i, b);
-          tma_load_4d(smem + L::OFF_DO + st * L::QB_BYTES + p * 8192, &tmdO, &q_full[st], 64 * p, h, 64 * i, b);
+          tma_load_4d(smem + L::OFF_Q + st * L::QB_BYTES + p * 8192, &tmQ, &q_full[st], 64 * p, h, base + 64 * i, bc);
+          tma_load_4d(smem + L::OFF_DO + st * L::QB_BYTES + p * 8192, &tmdO, &q_full[st], 64 * p, h, base + 64 * i, bc);
         }
-        const size_t row = ((size_t)b * prm.H + h) * prm.S + 64 * (size_t)i;
+        const size_t row = hrow0 + (size_t)h * prm.S + 64 * (size_t)i;
         bulk_load(smem + L::OFF_LSE + st * 256, prm.lse + row, 256, &q_full[st]);
         bulk_load(smem + L::OFF_DEL + st * 256, prm.delta + row, 256, &q_full[st]);
       }
@@ -403,7 +428,7 @@ __global__ void __launch_bounds__(448, 1)
     const int r = (warp & 3) * 32 + lane;  // KV row of the tile == TMEM lane
     const int kvb = 2 * u + (r >> 6);
     const int rr = r & 63;
-    const bool krow_live = kvb < prm.nqb;
+    const bool krow_live = kvb < nqb;
     const uint32_t t_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const float sl2 = prm.scale_log2;
     constexpr float kLog2e = 1.4426950408889634f;
@@ -521,13 +546,13 @@ __global__ void __launch_bounds__(448, 1)
       for (int which = 0; which < 2; ++which) {
         const uint32_t tcol = which == 0 ? L::T_DV : L::T_DK;
         const float mul = which == 0 ? 1.f : prm.scale;
-        float* dst = (which == 0 ? prm.dv_f32 : prm.dk_f32) + (((size_t)b * prm.S + krow) * prm.Hkv + kvh) * D;
+        float* dst = (which == 0 ? prm.dv_f32 : prm.dk_f32) + (((size_t)lin0 + krow) * prm.Hkv + kvh) * D;
 #pragma unroll
         for (int q = 0; q < CH; ++q) {
           const int col = hf * (D / 2) + 32 * q;
           uint32_t o[32];
           tmem_ld32(t_lane + tcol + col, o);
-          if (krow < prm.S) {
+          if (krow < len) {
             float4* d4 = reinterpret_cast<float4*>(dst + col);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
@@ -563,10 +588,12 @@ __global__ void __launch_bounds__(448, 1)
     fence_async_smem();
     named_bar_sync(1, 256);
     if (threadIdx.x == 0 && !*abort_flag && !prm.grad_f32) {
-      for (int p = 0; p < DP; ++p) {
-        tma_store_4d(&tmdV, smem + L::OFF_V + p * 16384, 64 * p, kvh, 128 * u, b);
-        tma_store_4d(&tmdK, smem + L::OFF_K + p * 16384, 64 * p, kvh, 128 * u, b);
-      }
+      // One 64-row box per block inside the sequence: never into the next packed sequence.
+      for (int hb = 0; hb < (2 * u + 1 < nqb ? 2 : 1); ++hb)
+        for (int p = 0; p < DP; ++p) {
+          tma_store_4d(&tmdV, smem + L::OFF_V + p * 16384 + hb * 8192, 64 * p, kvh, base + 128 * u + 64 * hb, bc);
+          tma_store_4d(&tmdK, smem + L::OFF_K + p * 16384 + hb * 8192, 64 * p, kvh, base + 128 * u + 64 * hb, bc);
+        }
       bulk_commit();
       bulk_wait_all();
     }
@@ -590,7 +617,7 @@ __global__ void __launch_bounds__(448, 1)
       tc_fence_before();
       mbar_arrive(&dq_free[bb]);
       if (dvalid) {
-        float* dst = prm.dq_acc + (((size_t)b * prm.H + h) * prm.S + 64 * (size_t)i) * D + d;
+        float* dst = prm.dq_acc + (hrow0 + (size_t)h * prm.S + 64 * (size_t)i) * D + d;
 #pragma unroll
         for (int c = 0; c < 64; ++c) red_add_f32(dst + (size_t)c * D, __uint_as_float(v[c]));
       }

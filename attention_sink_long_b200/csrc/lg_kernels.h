@@ -42,6 +42,8 @@ struct BwdParams {
   int grad_f32;      // 1: dK / dV written as fp32 straight from the accumulators
   float* dk_f32;     // [B, S, Hkv, D] when grad_f32
   float* dv_f32;
+  const int32_t* cu_seqlens = nullptr;  // device [B + 1] offsets of packed sequences (S = total rows), or nullptr
+  int max_len = 0;                      // with cu_seqlens: the longest sequence (nkt covers it)
   unsigned int* err;
 };
 

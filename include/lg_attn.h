@@ -197,6 +197,27 @@ lg_status_t lg_sparse_attn_bwd(const lg_pattern_t* pattern, const void* q, const
                                void* dk, void* dv, int32_t grad_dtype, int32_t B, int32_t S, int32_t H, int32_t Hkv,
                                int32_t D, float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream);
 
+/*
+ * The backward above for packed sequences of different lengths, the
+ * counterpart of lg_sparse_attn_fwd_varlen (training on a batch of documents
+ * of mixed lengths; summary, "Key results": 1.55x training). Tensors and the
+ * offsets as in lg_sparse_attn_fwd_varlen: q, o, dout, dq [total,H,D];
+ * k, v, dk, dv [total,Hkv,D]; lse [H,total] as that forward wrote it;
+ * cu_seqlens [B+1] int32 on the device. In addition every offset must be a
+ * multiple of 4 (16-byte aligned LSE rows) and total a multiple of 4
+ * (LG_ERR_UNSUPPORTED otherwise, on the host for total). Gradients of a
+ * sequence depend only on its own rows. dq rows outside every sequence are
+ * written as zero; dk / dv rows outside every sequence are not written. A
+ * cu_seqlens entry that breaks the rules is found on the device: that
+ * sequence is skipped and lg_device_status reports bit 4. Workspace:
+ * lg_sparse_attn_bwd_workspace(pattern, 1, total, H, Hkv, D) bytes.
+ */
+lg_status_t lg_sparse_attn_bwd_varlen(const lg_pattern_t* pattern, const void* q, const void* k, const void* v,
+                                      const void* o, int32_t o_dtype, const void* dout, const float* lse, void* dq,
+                                      void* dk, void* dv, int32_t grad_dtype, const int32_t* cu_seqlens, int32_t B,
+                                      int32_t total, int32_t max_seqlen, int32_t H, int32_t Hkv, int32_t D,
+                                      float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Prefill -> decode hand-off: the reduced KV cache                         */
 /* ------------------------------------------------------------------------ */

@@ -262,3 +262,31 @@ def test_paged_cache_argument_errors():
     assert decode(kp=0x30008) == 2
     assert decode(MB=(1 << 24) + 1) == 2
     assert decode(ns=4) == 3            # four splits need a workspace
+
+
+def test_bwd_varlen_argument_errors():
+    L = lg.lib()
+    p = lg._lg_pattern_t(64, 1, 4, 0)
+
+    def call(q=0x10000, cu=0x60000, B=2, total=1024, mx=512, H=4, Hkv=4, D=128, odt=0, gdt=0, scale=0.125,
+             ws=0x100000, wsb=1 << 30):
+        return L.lg_sparse_attn_bwd_varlen(ctypes.byref(p), q, 0x20000, 0x30000, 0x40000, odt, 0x50000, 0x70000,
+                                           0x80000, 0x90000, 0xa0000, gdt, cu, B, total, mx, H, Hkv, D, scale, ws, wsb,
+                                           None)
+
+    assert call(q=None) == 1
+    assert call(cu=None) == 1
+    assert call(B=0) == 1
+    assert call(H=4, Hkv=3) == 1
+    assert call(odt=3) == 1
+    assert call(gdt=2) == 1
+    assert call(scale=float("nan")) == 1
+    assert call(mx=500) == 2          # max_seqlen not a multiple of 64
+    assert call(mx=2048) == 2         # longer than the packed tensor
+    assert call(total=1022) == 2      # LSE rows would not be 16-byte aligned
+    assert call(D=96) == 2
+    assert call(q=0x10008) == 2       # misaligned
+    assert call(cu=0x60002) == 2      # misaligned offsets
+    assert call(ws=None) == 3
+    assert call(wsb=1024) == 3
+    assert call(ws=0x100080) == 2     # workspace not 256-byte aligned

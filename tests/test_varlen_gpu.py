@@ -106,3 +106,120 @@ def test_bad_offsets_are_reported_and_skipped():
     ro, _ = oracle.attention_forward(q[None, :128], k[None, :128], v[None, :128], p, scale)
     assert_close("O seq0", o[:128].float().cpu().numpy(), ro[0])
     assert torch.all(o[128:228].view(torch.int16) == SENTINEL)  # the skipped sequence
+
+
+# ---------------------------------------------------------------- backward
+def run_varlen_fwd_bwd(pat, q, k, v, do, cu, max_len, scale, odt=torch.float32, gdt=torch.float32,
+                       dq_fill=float("nan")):
+    total, H, D = q.shape
+    Hkv = k.shape[1]
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    cu_d = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    o = torch.zeros(total, H, D, dtype=odt, device="cuda")
+    lse = torch.zeros(H, total, dtype=torch.float32, device="cuda")
+    lg.lg_sparse_attn_fwd_varlen(pat, qd, kd, vd, o, lse, cu_d, max_len, scale)
+    dq = torch.full((total, H, D), dq_fill, dtype=gdt, device="cuda")
+    dk = torch.full((total, Hkv, D), SENTINEL, dtype=torch.int16, device="cuda")
+    dv = torch.full((total, Hkv, D), SENTINEL, dtype=torch.int16, device="cuda")
+    if gdt == torch.float32:
+        dk = torch.full((total, Hkv, D), float("nan"), device="cuda")
+        dv = torch.full((total, Hkv, D), float("nan"), device="cuda")
+    else:
+        dk, dv = dk.view(torch.bfloat16), dv.view(torch.bfloat16)
+    ws = torch.full((lg.lg_sparse_attn_bwd_workspace(pat, 1, total, H, Hkv, D),), 0xFF, dtype=torch.uint8,
+                    device="cuda")
+    lg.lg_sparse_attn_bwd_varlen(pat, qd, kd, vd, o, dod, lse, dq, dk, dv, cu_d, max_len, scale, ws)
+    torch.cuda.synchronize()
+    return dq, dk, dv
+
+
+BWD_CASES = [
+    # lens, H, Hkv, D, pattern, O dtype: both backward kernels (head dim 128 with H == Hkv; GQA / head dim 64)
+    ([192, 64, 512, 1024, 320], 2, 2, 128, (64, 1, 4, 0), torch.float32),
+    ([256, 640, 128], 2, 2, 128, (64, 1, 2, 4), torch.float32),
+    ([384, 64, 448], 4, 2, 128, (64, 0, 2, 3), torch.float32),
+    ([320, 192, 576], 2, 1, 64, (64, 0, 2**31 - 1, 0), torch.float32),
+    ([1024, 512], 2, 2, 128, (64, 1, 4, 0), torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("lens,H,Hkv,D,pat,odt", BWD_CASES)
+def test_varlen_bwd_matches_oracle_per_sequence(lens, H, Hkv, D, pat, odt):
+    total = int(sum(lens))
+    q, k, v, do = si.prefill_inputs(1, total, H, Hkv, D, seed=si.SEED_BASE + 110, with_dout=True)
+    q, k, v, do = q[0], k[0], v[0], do[0]
+    cu = [0] + list(np.cumsum(lens))
+    scale = 1.0 / math.sqrt(D)
+    dq, dk, dv = run_varlen_fwd_bwd(pat, q, k, v, do, cu, max(lens), scale, odt)
+    assert lg.lg_device_status(0) == 0
+    p = oracle.Pattern(*pat)
+    for b in range(len(lens)):
+        s0, s1 = cu[b], cu[b + 1]
+        rdq, rdk, rdv, _ = oracle.attention_backward(q[None, s0:s1], k[None, s0:s1], v[None, s0:s1],
+                                                     do[None, s0:s1], p, scale)
+        assert_close(f"dQ seq{b}", dq[s0:s1].cpu().numpy(), rdq[0])
+        assert_close(f"dK seq{b}", dk[s0:s1].cpu().numpy(), rdk[0])
+        assert_close(f"dV seq{b}", dv[s0:s1].cpu().numpy(), rdv[0])
+
+
+@pytest.mark.parametrize("H,Hkv,D", [(4, 4, 128), (4, 2, 64)])
+def test_varlen_bwd_equal_lengths_match_the_fixed_length_call(H, Hkv, D):
+    """dK / dV bit for bit (each written by one CTA); dQ to within the order of
+    its reduce-adds."""
+    B, S = 3, 768
+    pat = (64, 1, 4, 0)
+    scale = 1.0 / math.sqrt(D)
+    q, k, v, do = si.prefill_inputs(B, S, H, Hkv, D, with_dout=True)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o = torch.empty(B, S, H, D, dtype=torch.float32, device="cuda")
+    lse = torch.empty(B, H, S, dtype=torch.float32, device="cuda")
+    lg.lg_sparse_attn_fwd(pat, qd, kd, vd, o, lse, scale)
+    dq = torch.empty(B, S, H, D, device="cuda")
+    dk = torch.empty(B, S, Hkv, D, device="cuda")
+    dv = torch.empty_like(dk)
+    ws = torch.empty(lg.lg_sparse_attn_bwd_workspace(pat, B, S, H, Hkv, D), dtype=torch.uint8, device="cuda")
+    lg.lg_sparse_attn_bwd(pat, qd, kd, vd, o, dod, lse, dq, dk, dv, scale, ws)
+    flat = lambda t: t.reshape(B * S, *t.shape[2:])  # noqa: E731
+    vdq, vdk, vdv = run_varlen_fwd_bwd(pat, flat(q), flat(k), flat(v), flat(do), [b * S for b in range(B + 1)], S,
+                                       scale)
+    assert lg.lg_device_status(0) == 0
+    assert torch.equal(vdk, flat(dk)) and torch.equal(vdv, flat(dv))
+    assert torch.allclose(vdq, flat(dq), rtol=1e-5, atol=1e-5)
+
+
+def test_varlen_bwd_rows_outside_every_sequence():
+    lens, H, Hkv, D = [128, 256], 2, 2, 128
+    total = 64 + 128 + 256 + 64
+    q, k, v, do = si.prefill_inputs(1, total, H, Hkv, D, seed=si.SEED_BASE + 111, with_dout=True)
+    q, k, v, do = q[0], k[0], v[0], do[0]
+    cu = [64, 64 + 128, 64 + 128 + 256]
+    pat = (64, 1, 2, 0)
+    dq, dk, dv = run_varlen_fwd_bwd(pat, q, k, v, do, cu, 256, 0.125, gdt=torch.bfloat16, dq_fill=7.0)
+    assert lg.lg_device_status(0) == 0
+    for t in (dk, dv):
+        assert torch.all(t[:64].view(torch.int16) == SENTINEL)
+        assert torch.all(t[total - 64:].view(torch.int16) == SENTINEL)
+        assert not torch.any(t[64:total - 64].view(torch.int16) == SENTINEL)
+    assert torch.all(dq[:64] == 0) and torch.all(dq[total - 64:] == 0)
+    # The bf16 gradients are the fp32 ones rounded (the fp32 run is checked against the oracle above).
+    fq, fk, fv = run_varlen_fwd_bwd(pat, q, k, v, do, cu, 256, 0.125)
+    for name, g, f in (("dK", dk, fk), ("dV", dv, fv)):
+        r = f[64:total - 64].to(torch.bfloat16).float()
+        ulp = torch.where(r == 0, torch.full_like(r, 2.0 ** -133), torch.abs(r) * 2.0 ** -7)
+        assert (torch.abs(g[64:total - 64].float() - r) > ulp * 1.0001).sum().item() == 0, name
+
+
+def test_varlen_bwd_bad_offsets_are_reported_and_skipped():
+    lens, H, Hkv, D = [128, 192, 256], 2, 2, 128
+    total = sum(lens)
+    q, k, v, do = si.prefill_inputs(1, total, H, Hkv, D, seed=si.SEED_BASE + 112, with_dout=True)
+    q, k, v, do = q[0], k[0], v[0], do[0]
+    cu = [0, 128, 128 + 100, total]  # sequence 1 has 100 rows: not a multiple of 64
+    dq, dk, dv = run_varlen_fwd_bwd((64, 1, 2, 0), q, k, v, do, cu, 256, 0.125)
+    st = lg.lg_device_status(0)
+    assert st & 16, st
+    assert lg.lg_device_status(0) == 0
+    rdq, rdk, rdv, _ = oracle.attention_backward(q[None, :128], k[None, :128], v[None, :128], do[None, :128],
+                                                 oracle.Pattern(64, 1, 2, 0), 0.125)
+    assert_close("dK seq0", dk[:128].cpu().numpy(), rdk[0])
+    assert torch.all(torch.isnan(dk[128:228]))  # the skipped sequence's rows are not written
