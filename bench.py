@@ -154,8 +154,8 @@ def workload(name):
                 "fwd": [("block-sparse", BLOCK_SPARSE)], "bwd": [("block-sparse", BLOCK_SPARSE)],
                 "decode": {"B": 32, "H": 32, "Hkv": 32, "D": D, "L": 5056}}
     if name == "varlen":
-        return {"workload": "variable-length prefill forward: 8 packed sink+window prompts of 32K..512 tokens "
-                            "(64K rows), H32 D128",
+        return {"workload": "variable-length sink+window forward + training backward: 8 packed sequences of "
+                            "32K..512 tokens (64K rows), H32 D128",
                 "prefill": None, "fwd": [], "bwd": [], "decode": None,
                 "varlen": {"lens": [32768, 16384, 8192, 4096, 2048, 1024, 512, 512], "H": 32, "Hkv": 32, "D": D,
                            "pattern": SINK_WINDOW}}
@@ -313,6 +313,12 @@ class CudaStep:
             self.vcu = torch.tensor(cu, dtype=torch.int32, device=device)
             flops = sum(4 * D * pairs_of(vl["pattern"], n) * H for n in lens)
             self.parts.append(("fwd varlen sink+window", "fwd", flops, None, 1))
+            self.vdo = si.device_normal((total, H, D), si.SEED_BASE + 3, device)
+            self.vdq, self.vdk, self.vdv = (torch.empty_like(self.vq), torch.empty_like(self.vk),
+                                            torch.empty_like(self.vv))
+            self.vws = torch.empty(lg.lg_sparse_attn_bwd_workspace(vl["pattern"], 1, total, H, Hkv, D),
+                                   dtype=torch.uint8, device=device)
+            self.parts.append(("bwd varlen sink+window", "bwd", 10 * flops // 4, None, 3))
         pg = wl.get("paged")
         if pg is not None:
             self._setup_paged(pg, device)
@@ -414,6 +420,12 @@ class CudaStep:
             if events is not None:
                 events[i].record(self.stream)
             i += 1
+            lg.lg_sparse_attn_bwd_varlen(vl["pattern"], self.vq, self.vk, self.vv, self.vo, self.vdo, self.vlse,
+                                         self.vdq, self.vdk, self.vdv, self.vcu, max(vl["lens"]), self.scale,
+                                         self.vws)
+            if events is not None:
+                events[i].record(self.stream)
+            i += 1
         if wl.get("paged") is not None:
             lg.lg_sparse_decode_paged(self.pq, self.kpool, self.vpool, self.ptable, self.plens, self.po, self.plse,
                                       1.0 / math.sqrt(wl["paged"]["D"]), workspace=self.pws)
@@ -444,7 +456,7 @@ def host_buffers(step):
     torch = step.torch
     pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu())  # noqa: E731
     ins, outs = [], []
-    for name in ("q", "k", "v", "do", "dq_in", "kc", "vc", "lens", "hk", "hv", "vq", "vk", "vv", "pq", "kpool",
+    for name in ("q", "k", "v", "do", "dq_in", "kc", "vc", "lens", "hk", "hv", "vq", "vk", "vv", "vdo", "pq", "kpool",
                  "vpool", "ptable", "plens"):
         if hasattr(step, name):
             ins.append((getattr(step, name), pin(getattr(step, name))))
@@ -452,7 +464,7 @@ def host_buffers(step):
         if hasattr(step, d):
             for t in getattr(step, d).values():
                 outs.append((t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)))
-    for name in ("dq", "dk", "dv", "do_out", "dlse", "hkc", "hvc", "hlens", "vo", "vlse", "po", "plse"):
+    for name in ("dq", "dk", "dv", "do_out", "dlse", "hkc", "hvc", "hlens", "vo", "vlse", "vdq", "vdk", "vdv", "po", "plse"):
         if hasattr(step, name):
             t = getattr(step, name)
             outs.append((t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)))
@@ -652,10 +664,11 @@ def oracle_sample(wl, budget_s, seed=11):
         # Forward rows of the longest sequence (the pattern acts inside each sequence alone).
         S, D = max(vl["lens"]), vl["D"]
         nqb = S // 64
-        q, k, v = si.prefill_inputs(1, S, 1, 1, D)
-        qh, kh, vh = (t[0, :, 0].double().numpy() for t in (q, k, v))
+        q, k, v, do = si.prefill_inputs(1, S, 1, 1, D, with_dout=True)
+        qh, kh, vh, doh = (t[0, :, 0].double().numpy() for t in (q, k, v, do))
         scale = 1.0 / math.sqrt(D)
         jobs.append(("fwd varlen", "fwd", vl["pattern"]))
+        jobs.append(("bwd varlen", "bwd", vl["pattern"]))
     ho = wl.get("handoff")
     if ho:
         # One KV head of one prompt, drawn on the host with the same seed as head 0.
