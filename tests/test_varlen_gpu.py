@@ -223,3 +223,47 @@ def test_varlen_bwd_bad_offsets_are_reported_and_skipped():
                                                  oracle.Pattern(64, 1, 2, 0), 0.125)
     assert_close("dK seq0", dk[:128].cpu().numpy(), rdk[0])
     assert torch.all(torch.isnan(dk[128:228]))  # the skipped sequence's rows are not written
+
+
+def test_varlen_bench_workload_sampled():
+    """The packed workload bench.py times (8 sink+window sequences of 32K..512
+    tokens, H32 D128, bf16 O as in training): O rows, dQ rows and dK / dV rows
+    of sampled blocks of the first, a middle and the last sequence vs the
+    oracle run on that sequence alone."""
+    lens = [32768, 16384, 8192, 4096, 2048, 1024, 512, 512]
+    H, D = 32, 128
+    pat = (64, 1, 64, 0)
+    op = oracle.Pattern(*pat)
+    total = sum(lens)
+    cu = [0] + list(np.cumsum(lens))
+    dev = torch.device("cuda")
+    q = si.device_normal((total, H, D), si.SEED_BASE + 0, dev)
+    k = si.device_normal((total, H, D), si.SEED_BASE + 1, dev)
+    v = si.device_normal((total, H, D), si.SEED_BASE + 2, dev)
+    do = si.device_normal((total, H, D), si.SEED_BASE + 3, dev)
+    scale = 1.0 / math.sqrt(D)
+    cu_d = torch.tensor(cu, dtype=torch.int32, device=dev)
+    o = torch.empty(total, H, D, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(H, total, dtype=torch.float32, device=dev)
+    lg.lg_sparse_attn_fwd_varlen(pat, q, k, v, o, lse, cu_d, max(lens), scale)
+    dq, dk, dv = (torch.empty(total, H, D, dtype=torch.float32, device=dev) for _ in range(3))
+    ws = torch.empty(lg.lg_sparse_attn_bwd_workspace(pat, 1, total, H, H, D), dtype=torch.uint8, device=dev)
+    lg.lg_sparse_attn_bwd_varlen(pat, q, k, v, o, do, lse, dq, dk, dv, cu_d, max(lens), scale, ws)
+    torch.cuda.synchronize()
+    assert lg.lg_device_status(0) == 0
+    rng = np.random.default_rng(3)
+    for b, h in ((0, 0), (3, 17), (7, H - 1)):
+        s0, n = cu[b], lens[b]
+        nqb = n // 64
+        qh, kh, vh, doh = (t[s0:s0 + n, h].float().cpu().numpy() for t in (q, k, v, do))
+        blocks = sorted({0, nqb - 1, *rng.choice(np.arange(nqb), min(nqb, 3), replace=False).tolist()})
+        rows = np.concatenate([np.arange(i * 64, i * 64 + 64) for i in blocks])
+        ro, rl = oracle.attention_rows(qh, kh, vh, rows, op, scale)
+        assert_close(f"O seq{b} h{h}", o[s0 + rows, h].float().cpu().numpy(), ro)
+        assert np.max(np.abs(lse[h, s0 + rows].cpu().numpy() - rl)) <= LSE_TOL
+        rdq, _ = oracle.attention_backward_rows(qh, kh, vh, doh, rows, op, scale)
+        assert_close(f"dQ seq{b} h{h}", dq[s0 + rows, h].cpu().numpy(), rdq)
+        krows = np.concatenate([np.arange(j * 64, j * 64 + 64) for j in blocks[:3]])
+        rdk, rdv = oracle.attention_backward_kv_rows(qh, kh, vh, doh, krows, op, scale, chunk=256)
+        assert_close(f"dK seq{b} h{h}", dk[s0 + krows, h].cpu().numpy(), rdk)
+        assert_close(f"dV seq{b} h{h}", dv[s0 + krows, h].cpu().numpy(), rdv)
