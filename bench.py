@@ -459,7 +459,7 @@ def host_buffers(step):
     for name in ("q", "k", "v", "do", "dq_in", "kc", "vc", "lens", "hk", "hv", "vq", "vk", "vv", "vdo", "pq", "kpool",
                  "vpool", "ptable", "plens"):
         if hasattr(step, name):
-            ins.append((getattr(step, name), pin(getattr(step, name))))
+            ins.append((name, getattr(step, name), pin(getattr(step, name))))
     for d in ("o", "lse"):
         if hasattr(step, d):
             for t in getattr(step, d).values():
@@ -469,6 +469,51 @@ def host_buffers(step):
             t = getattr(step, name)
             outs.append((t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)))
     return ins, outs
+
+
+def e2e_steps(step, ins, outs, nsteps):
+    """nsteps end-to-end steps: upload inputs, run, download outputs. Inputs have two device sets used in
+    turn, so step k+1's upload runs while step k computes; uploads and downloads run on their own streams,
+    so step k's download overlaps step k+1's upload. Events keep each buffer's uses in order: an input set is
+    overwritten only after the kernels of the step before last read it, outputs only after the previous
+    step's download. Returns device ms from the first upload to the last download."""
+    torch = step.torch
+    comp = step.stream
+    s_in = torch.cuda.Stream(device=step.dev)
+    s_out = torch.cuda.Stream(device=step.dev)
+    sets = [{name: d for name, d, _ in ins}, {name: torch.empty_like(d) for name, d, _ in ins}]
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    free_set, free_out = [e0, e0], e0
+    for k in range(nsteps):
+        cur = sets[k % 2]
+        s_in.wait_event(free_set[k % 2])
+        with torch.cuda.stream(s_in):
+            for name, _, h in ins:
+                cur[name].copy_(h, non_blocking=True)
+        ready = torch.cuda.Event()
+        ready.record(s_in)
+        comp.wait_event(ready)
+        comp.wait_event(free_out)
+        for name, t in cur.items():
+            setattr(step, name, t)
+        step.run()
+        done = torch.cuda.Event()
+        done.record(comp)
+        s_out.wait_event(done)
+        with torch.cuda.stream(s_out):
+            for d, h in outs:
+                h.copy_(d, non_blocking=True)
+        downloaded = torch.cuda.Event()
+        downloaded.record(s_out)
+        free_set[k % 2], free_out = done, downloaded
+    comp.wait_event(free_out)
+    e1.record(comp)
+    torch.cuda.synchronize()
+    for name, t in sets[0].items():  # the step keeps its original input tensors
+        setattr(step, name, t)
+    return e0.elapsed_time(e1)
 
 
 def cuda_arm(args, rank, world, dist):
@@ -567,33 +612,20 @@ def cuda_arm(args, rank, world, dist):
     e2e = None
     if not args.no_e2e:
         ins, outs = host_buffers(step)
-        bi = sum(h.numel() * h.element_size() for _, h in ins)
+        bi = sum(h.numel() * h.element_size() for _, _, h in ins)
         bo = sum(h.numel() * h.element_size() for _, h in outs)
-        for _ in range(1):
-            for d, h in ins:
-                d.copy_(h, non_blocking=True)
-            step.run()
-            for d, h in outs:
-                h.copy_(d, non_blocking=True)
+        e2e_steps(step, ins, outs, 1)  # warm-up
         torch.cuda.synchronize()
         if dist is not None:
             dist.barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
         ek = max(1, min(args.steps, 5))
-        e0.record(step.stream)
-        for _ in range(ek):
-            for d, h in ins:
-                d.copy_(h, non_blocking=True)
-            step.run()
-            for d, h in outs:
-                h.copy_(d, non_blocking=True)
-        e1.record(step.stream)
-        torch.cuda.synchronize()
-        ems = max_over_ranks(e0.elapsed_time(e1) / ek, dist, device)
+        ems = max_over_ranks(e2e_steps(step, ins, outs, ek) / ek, dist, device)
         e2e_v = step_bytes / (ems * 1e-3) / 1e9 if by_bytes else step_flops / (ems * 1e-3) / 1e12
         e2e = {"value": round(world * e2e_v, 3), "unit": unit,
-               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(ems, 3), "steps": ek}
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(ems, 3), "steps": ek,
+               "copies": "every step uploads all its inputs and downloads all its outputs (pinned host memory); "
+                         "inputs alternate between two device sets and uploads / downloads run on their own "
+                         "streams, so step k+1's upload overlaps step k's compute and download"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
