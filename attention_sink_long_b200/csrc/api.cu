@@ -331,10 +331,10 @@ static lg_status_t bwd_common(const lg_pattern_t* p, const void* q, const void* 
   float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + round256((size_t)Bm * H * S * D * 4));
   float* lse2 = reinterpret_cast<float*>(reinterpret_cast<char*>(delta) + round256((size_t)Bm * H * S * 4));
 
-  // Head dim 128 without query-head groups runs the 128-row-step kernel, whose
-  // KV tiles are two separately placed 64-row blocks (BlockPairing); the other
-  // kernel's tiles are 128 consecutive rows, also moved as two 64-row boxes.
-  const bool paired = (D == 128 && H == Hkv);
+  // Head dim 128 runs the 128-row-step kernel, whose KV tiles are two
+  // separately placed 64-row blocks (BlockPairing); the head-dim-64 kernel's
+  // tiles are 128 consecutive rows, also moved as two 64-row boxes.
+  const bool paired = (D == 128);
   CUtensorMap tq, tk, tv, tdo, tdk, tdv;
   if ((st = make_map(&tq, q, Bm, S, H, D, 64)) != LG_OK) return st;
   if ((st = make_map(&tk, k, Bm, S, Hkv, D, 64)) != LG_OK) return st;

@@ -1,5 +1,5 @@
 // bwd128_sm100.cu -- LongGen sparse causal attention, training backward for
-// head dim 128 without query-head groups (H == Hkv), on sm_100a.
+// head dim 128, on sm_100a.
 //
 // "A Little Goes a Long Way" (LongGen), Abstract insights 1-2 and the
 // atlas.scime.ai summary, "Approach": the sparse layers are trained, so the
@@ -10,11 +10,12 @@
 //   dS = P o (dP - Delta) with Delta = rowsum(dO o O),
 //   dK = scale * dS^T Q,  dQ = scale * dS K.
 //
-// One CTA owns a 128-row KV tile of one head -- two 64-row KV blocks paired
+// One CTA owns a 128-row KV tile of one KV head -- two 64-row KV blocks paired
 // by BlockPairing (blocks every later query sees pair with each other, then
 // the window-only blocks pair in order), so both halves of the tile see nearly
 // the same query blocks -- and walks those query blocks two at a time: a
-// 128-row query step.
+// 128-row query step (with query-head groups, the steps of every query head
+// of the group in turn, dK and dV accumulating over all of them).
 // Every GEMM of a step is then an M = 128, N = 128 tcgen05 MMA -- the shape
 // the tensor core runs at full rate (an N = 64 instruction takes about as
 // long as an N = 128 one):
@@ -28,6 +29,10 @@
 // The P/dS warps read S^T and write P^T (bf16, two per column) over the first
 // half of the columns they read, so no warp overwrites columns another warp
 // still reads. R_d holds dP^T until the warps have read it, then dQ^T.
+// With query-head groups dV and dK sum over the group's heads and grow with
+// it, so P and dS also enter them as bf16 residuals (x - bf16(x)): P^T's into
+// the second half of each warp's S^T columns, dS^T's into the first half of
+// each warp's dP^T columns (both already read), each an extra TS MMA.
 //
 // MMA order (one thread; tcgen05 MMAs of one thread execute in order):
 //   S^T(0), dP^T(0), dV(0), S^T(1), then per step n:
@@ -72,6 +77,7 @@ struct Bwd128Layout {
   static_assert(OFF_LSE % 16 == 0, "bulk copies need 16-byte aligned destinations");
 };
 
+template <bool GQA>
 __global__ void __launch_bounds__(448, 1)
     lg_bwd128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -164,6 +170,11 @@ __global__ void __launch_bounds__(448, 1)
   const int q_first = ky >= 0 ? imin(kx, ky) : kx;
   const int last = ky >= 0 ? imax(bp.reach(kx), bp.reach(ky)) : bp.reach(kx);
   const int N = (last - q_first + 2) / 2;  // 128-row query steps (the last one may hold one block)
+  // With query-head groups the CTA walks every query head of its KV head:
+  // step m is query step m % N of query head h * G + m / N, and dK / dV
+  // accumulate over the whole group.
+  const int G = GQA ? prm.H / prm.Hkv : 1;
+  const int NT = G * N;
   unsigned int* err = prm.err;
 
   if (threadIdx.x == 0) {
@@ -204,34 +215,35 @@ __global__ void __launch_bounds__(448, 1)
           tma_load_4d(smem + L::OFF_V + p * L::PANEL + hb * 8192, &tmV, kv_full, 64 * p, h, base + 64 * kload[hb], bc);
         }
       int issued_o = 0, issued_q = 0;  // steps whose dO / Q copies were issued
-      for (int n = 0; n < N; ++n) {
-        const int st = n & 1;
-        const uint32_t use = (uint32_t)(n >> 1);
-        const int i0 = q_first + 2 * n;
+      for (int m = 0; m < NT; ++m) {
+        const int st = m & 1;
+        const uint32_t use = (uint32_t)(m >> 1);
+        const int hq = GQA ? h * G + m / N : h;  // query head
+        const int i0 = q_first + 2 * (GQA ? m % N : m);
         // Both 64-row halves always load (rows past the sequence arrive as
         // zeros), so a stage never holds stale operands; LSE / Delta only
         // exist for blocks inside the sequence.
         const int nl = (i0 + 1 < nqb) ? 2 : 1;
         if (use > 0 && !mbar_wait(&qo_empty[st], (use - 1) & 1, abort_flag, err, kErrBwdWait)) break;
         mbar_arrive_expect_tx(&qo_full[st], L::TILE + nl * 256);
-        issued_o = n + 1;
+        issued_o = m + 1;
         for (int hb = 0; hb < 2; ++hb)
           for (int p = 0; p < 2; ++p)
-            tma_load_4d(smem + L::OFF_DO + st * L::TILE + p * L::PANEL + hb * 8192, &tmdO, &qo_full[st], 64 * p, h,
+            tma_load_4d(smem + L::OFF_DO + st * L::TILE + p * L::PANEL + hb * 8192, &tmdO, &qo_full[st], 64 * p, hq,
                         base + 64 * (i0 + hb), bc);
         for (int hb = 0; hb < nl; ++hb) {
-          const size_t row = hrow0 + (size_t)h * prm.S + 64 * (size_t)(i0 + hb);
+          const size_t row = hrow0 + (size_t)hq * prm.S + 64 * (size_t)(i0 + hb);
           bulk_load(smem + L::OFF_DEL + st * 512 + hb * 256, prm.delta + row, 256, &qo_full[st]);
         }
         if (use > 0 && !mbar_wait(&qq_empty[st], (use - 1) & 1, abort_flag, err, kErrBwdWait)) break;
         mbar_arrive_expect_tx(&qq_full[st], L::TILE + nl * 256);
-        issued_q = n + 1;
+        issued_q = m + 1;
         for (int hb = 0; hb < 2; ++hb)
           for (int p = 0; p < 2; ++p)
-            tma_load_4d(smem + L::OFF_Q + st * L::TILE + p * L::PANEL + hb * 8192, &tmQ, &qq_full[st], 64 * p, h,
+            tma_load_4d(smem + L::OFF_Q + st * L::TILE + p * L::PANEL + hb * 8192, &tmQ, &qq_full[st], 64 * p, hq,
                         base + 64 * (i0 + hb), bc);
         for (int hb = 0; hb < nl; ++hb) {
-          const size_t row = hrow0 + (size_t)h * prm.S + 64 * (size_t)(i0 + hb);
+          const size_t row = hrow0 + (size_t)hq * prm.S + 64 * (size_t)(i0 + hb);
           bulk_load(smem + L::OFF_LSE + st * 512 + hb * 256, prm.lse2 + row, 256, &qq_full[st]);
         }
       }
@@ -302,6 +314,12 @@ __global__ void __launch_bounds__(448, 1)
         for (int kk = 0; kk < 8; ++kk)
           tc_mma_ts_if(leader, tmem + L::T_DV, tmem + L::T_RS + 64 * (kk >> 2) + 8 * (kk & 3), o + mofs(kk), idesc_kmn,
                     (n > 0 || kk > 0) ? 1u : 0u);
+        if (GQA) {  // + the bf16 residual of P^T, 32 columns further on
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc_mma_ts_if(leader, tmem + L::T_DV, tmem + L::T_RS + 32 + 64 * (kk >> 2) + 8 * (kk & 3), o + mofs(kk),
+                         idesc_kmn, 1u);
+        }
       };
       // dK += dS^T(n) Q(n).
       auto issue_dk = [&](int n) {
@@ -309,6 +327,12 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           tc_mma_ss_if(leader, tmem + L::T_DK, dS_k + kofs(kk), q + mofs(kk), idesc_kmn, (n > 0 || kk > 0) ? 1u : 0u);
+        if (GQA) {  // + the bf16 residual of dS^T, left in R_d by the dS phase (dQ^T overwrites it next)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc_mma_ts_if(leader, tmem + L::T_DK, tmem + L::T_RD + 64 * (kk >> 2) + 8 * (kk & 3), q + mofs(kk),
+                         idesc_kmn, 1u);
+        }
       };
       // dQ^T(n) = K^T dS^T(n) into R_d (fresh each step).
       auto issue_dq = [&](int n) {
@@ -336,7 +360,7 @@ __global__ void __launch_bounds__(448, 1)
         tc_fence_after();
         issue_dv(0);
         tc_commit_if(leader, &qo_empty[0]);
-        if (N > 1) {
+        if (NT > 1) {
           ok = mbar_wait(&qq_full[1], 0, abort_flag, err, kErrBwdWait);
           if (ok) {
             tc_fence_after();
@@ -345,7 +369,7 @@ __global__ void __launch_bounds__(448, 1)
           }
         }
       }
-      for (int n = 0; n < N && ok; ++n) {
+      for (int n = 0; n < NT && ok; ++n) {  // n: global step
         const uint32_t par = (uint32_t)n & 1;
         if (!mbar_wait(ds_full, par, abort_flag, err, kErrBwdWait)) break;
         tc_fence_after();
@@ -356,7 +380,7 @@ __global__ void __launch_bounds__(448, 1)
         issue_dq(n);
         tc_commit_if(leader, dq_full);
         tc_commit_if(leader, dss_free);
-        if (n + 1 < N) {
+        if (n + 1 < NT) {
           // R_d takes dP^T(n+1) once the drain warps have read dQ^T(n).
           if (!mbar_wait(dq_free, par, abort_flag, err, kErrBwdWait)) break;
           if (!mbar_wait(&qo_full[(n + 1) & 1], (uint32_t)((n + 1) >> 1) & 1, abort_flag, err, kErrBwdWait)) break;
@@ -367,7 +391,7 @@ __global__ void __launch_bounds__(448, 1)
           tc_fence_after();
           issue_dv(n + 1);
           tc_commit_if(leader, &qo_empty[(n + 1) & 1]);
-          if (n + 2 < N) {
+          if (n + 2 < NT) {
             // S^T(n+2) overwrites P^T(n+1), which dV(n+1) -- issued just before --
             // reads first; its Q stage was refilled after dK(n) completed.
             if (!mbar_wait(&qq_full[n & 1], (uint32_t)((n + 2) >> 1) & 1, abort_flag, err, kErrBwdWait)) break;
@@ -393,10 +417,10 @@ __global__ void __launch_bounds__(448, 1)
     const uint32_t t_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const float sl2 = prm.scale_log2;
     int n = 0;
-    for (; n < N; ++n) {
+    for (; n < NT; ++n) {  // n: global step (query head h * G + n / N)
       const int st = n & 1;
       const uint32_t par = (uint32_t)n & 1;
-      const int i = q_first + 2 * n + hf;  // this warp's query block
+      const int i = q_first + 2 * (GQA ? n % N : n) + hf;  // this warp's query block
       const bool vis = krow_live && i <= last && in_list(prm.pat, i, kvb);
       const bool diag = (i == kvb);
       if (!__all_sync(0xffffffffu, mbar_wait(&qq_full[st], (uint32_t)(n >> 1) & 1, abort_flag, err, kErrBwdWait)))
@@ -438,6 +462,22 @@ __global__ void __launch_bounds__(448, 1)
         for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pf[32 * ch + 2 * e], pf[32 * ch + 2 * e + 1]);
         tmem_st16(t_lane + L::T_RS + c0 + 16 * ch, pk);
       }
+      if (GQA) {
+        // The bf16 residual P - bf16(P) into columns [32, 64) of this warp's
+        // S^T range (read above): dV takes P^T as a hi + lo pair, exact to the
+        // fp32 accumulation, since its sum over the group grows with it.
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          uint32_t pl[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float a = pf[32 * ch + 2 * e], b = pf[32 * ch + 2 * e + 1];
+            const uint32_t hi = pack_bf16x2(a, b);
+            pl[e] = pack_bf16x2(a - __uint_as_float(hi << 16), b - __uint_as_float(hi & 0xffff0000u));
+          }
+          tmem_st16(t_lane + L::T_RS + c0 + 32 + 16 * ch, pl);
+        }
+      }
       tc_fence_before();
       mbar_arrive(p_full);
       mbar_arrive(&qq_empty[st]);  // done with this step's LSE
@@ -455,6 +495,7 @@ __global__ void __launch_bounds__(448, 1)
       for (int ch = 0; ch < 2; ++ch) {
         uint32_t dpr[32];
         tmem_ld32(t_lane + L::T_RD + c0 + 32 * ch, dpr);
+        uint32_t dlo[16];  // with query-head groups: dS - bf16(dS), packed, back into R_d
         // eight columns (one 16-byte chunk of the row) at a time
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -470,13 +511,22 @@ __global__ void __launch_bounds__(448, 1)
                                                      __uint_as_float(dpr[8 * c + 2 * e + 1])),
                                          make_float2(dl[2 * e], dl[2 * e + 1])));
               pk[e] = pack_bf16x2(d.x, d.y);
+              if (GQA)
+                dlo[4 * c + e] = pack_bf16x2(d.x - __uint_as_float(pk[e] << 16), d.y - __uint_as_float(pk[e] & 0xffff0000u));
             }
           } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) pk[e] = 0u;
+            for (int e = 0; e < 4; ++e) {
+              pk[e] = 0u;
+              if (GQA) dlo[4 * c + e] = 0u;
+            }
           }
           st_shared_v4(drow + sw128_offset(r, 4 * ch + c), pk[0], pk[1], pk[2], pk[3]);
         }
+        // Columns [16 ch, +16) of this warp's R_d range were read by the load
+        // above (ch = 0 read all 32 of them), and dK reads them as an MMA
+        // operand before dQ^T overwrites R_d.
+        if (GQA) tmem_st16(t_lane + L::T_RD + c0 + 16 * ch, dlo);
       }
       fence_async_smem();
       tc_fence_before();
@@ -486,7 +536,7 @@ __global__ void __launch_bounds__(448, 1)
 
     // ------------------------------------------------------------ dK, dV epilogue
     // Warp (quarter, half) writes rows of its quarter, columns [64 half, +64).
-    bool ok = (n == N) && !*abort_flag;
+    bool ok = (n == NT) && !*abort_flag;
     if (ok) ok = mbar_wait(acc_done, 0, abort_flag, err, kErrBwdWait);
     ok = __all_sync(0xffffffffu, ok);
     if (ok && prm.grad_f32) {
@@ -554,12 +604,13 @@ __global__ void __launch_bounds__(448, 1)
     const int quarter = warp & 3;
     const int d = quarter * 32 + lane;
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
-    for (int n = 0; n < N; ++n) {
-      const int i0 = q_first + 2 * n;
+    for (int n = 0; n < NT; ++n) {  // n: global step
+      const int hq = GQA ? h * G + n / N : h;  // query head
+      const int i0 = q_first + 2 * (GQA ? n % N : n);
       const bool second = i0 + 1 <= last;  // the step's second query block is in the list range
       if (!__all_sync(0xffffffffu, mbar_wait(dq_full, (uint32_t)n & 1, abort_flag, err, kErrBwdWait))) break;
       tc_fence_after();
-      float* dst = prm.dq_acc + (hrow0 + (size_t)h * prm.S + 64 * (size_t)i0) * L::D + d;
+      float* dst = prm.dq_acc + (hrow0 + (size_t)hq * prm.S + 64 * (size_t)i0) * L::D + d;
       // Read all 128 columns first, so R_d is released before any reduction is
       // issued (the reductions run at the L2's rate and would otherwise hold
       // up the next dP^T).
@@ -573,7 +624,7 @@ __global__ void __launch_bounds__(448, 1)
       // Loads before the second half of the reductions: the Q / dO copies of
       // step n+2 (issued once dK(n) freed their stage) go through L2 first, so
       // the next S^T is not starved by this step's reductions.
-      if (n + 2 < N &&
+      if (n + 2 < NT &&
           !__all_sync(0xffffffffu, mbar_wait(&qq_full[n & 1], (uint32_t)((n + 2) >> 1) & 1, abort_flag, err,
                                              kErrBwdWait)))
         break;
@@ -597,10 +648,15 @@ cudaError_t launch_bwd128(const CUtensorMap& tq, const CUtensorMap& tk, const CU
                           cudaStream_t stream) {
   using L = Bwd128Layout;
   static_assert(L::BYTES <= L::ALLOC, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(lg_bwd128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+  const bool gqa = prm.H != prm.Hkv;
+  cudaError_t e = cudaFuncSetAttribute(gqa ? lg_bwd128_kernel<true> : lg_bwd128_kernel<false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (e != cudaSuccess) return e;
   dim3 grid(prm.nkt * prm.Hkv, B);
-  lg_bwd128_kernel<<<grid, 448, L::ALLOC, stream>>>(tq, tk, tv, tdo, tdk, tdv, prm);
+  if (gqa)
+    lg_bwd128_kernel<true><<<grid, 448, L::ALLOC, stream>>>(tq, tk, tv, tdo, tdk, tdv, prm);
+  else
+    lg_bwd128_kernel<false><<<grid, 448, L::ALLOC, stream>>>(tq, tk, tv, tdo, tdk, tdv, prm);
   return cudaGetLastError();
 }
 

@@ -649,7 +649,7 @@ static cudaError_t launch_bwd_impl(const CUtensorMap& tq, const CUtensorMap& tk,
 cudaError_t launch_bwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv, const BwdParams& prm,
                        int B, cudaStream_t stream) {
-  if (D == 128 && !prm.split_lo) return launch_bwd128(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
+  if (D == 128) return launch_bwd128(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
   if (prm.split_lo) {
     if (D == 64) return launch_bwd_impl<64, true>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
     return launch_bwd_impl<128, true>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);

@@ -51,7 +51,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
-    ap.add_argument("--workload", choices=["step32k", "fwd128k", "bwd128k", "decode", "handoff", "blocksparse128k", "varlen", "decode_paged"],
+    ap.add_argument("--workload", choices=["step32k", "fwd128k", "bwd128k", "decode", "handoff", "blocksparse128k", "varlen", "decode_paged",
+                                               "gqa32k"],
                     default="step32k")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -138,6 +139,10 @@ def workload(name):
         return {"workload": "128K block-sparse prefill forward {64,1,16,32}",
                 "prefill": {"B": 1, "S": 131072, "H": 32, "Hkv": 32, "D": D},
                 "fwd": [("block-sparse", BLOCK_SPARSE)], "bwd": [], "decode": None}
+    if name == "gqa32k":
+        return {"workload": "grouped-query 32K: fwd + training bwd sink+window {64,1,64,0}, H32 Hkv8 D128",
+                "prefill": {"B": 1, "S": 32768, "H": 32, "Hkv": 8, "D": D},
+                "fwd": [("sink+window", SINK_WINDOW)], "bwd": [("sink+window", SINK_WINDOW)], "decode": None}
     if name == "bwd128k":
         return {"workload": "128K sink+window training backward {64,1,64,0}",
                 "prefill": {"B": 1, "S": 131072, "H": 32, "Hkv": 32, "D": D},
