@@ -110,3 +110,45 @@ def test_bwd_128k_sampled(pat):
         rdk, rdv = oracle.attention_backward_kv_rows(qh, kh, vh, doh, krows, op, scale, chunk=256)
         assert_close(f"dK h{h}", dk[0, krows, h].cpu().numpy(), rdk)
         assert_close(f"dV h{h}", dv[0, krows, h].cpu().numpy(), rdv)
+
+
+def test_gqa_32k_sampled():
+    """The grouped-query workload bench.py times (32K sink+window, H32 Hkv8
+    D128, bf16 O as in training): O and dQ rows of sampled query blocks, and
+    dK / dV rows of sampled KV blocks -- the oracle sums those over the four
+    query heads of the KV head."""
+    B, S, H, Hkv, D = 1, 32768, 32, 8, 128
+    pat = lg.Pattern(64, 1, 64, 0)
+    op = oracle.Pattern(*pat)
+    G = H // Hkv
+    dev = torch.device("cuda")
+    q, k, v, do = si.prefill_inputs_device(B, S, H, Hkv, D, dev, with_dout=True)
+    scale = 1.0 / math.sqrt(D)
+    o = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, H, S, dtype=torch.float32, device=dev)
+    lg.lg_sparse_attn_fwd(pat, q, k, v, o, lse, scale)
+    dq, dk, dv = (torch.empty(t.shape, dtype=torch.float32, device=dev) for t in (q, k, v))
+    ws = torch.empty(lg.lg_sparse_attn_bwd_workspace(pat, B, S, H, Hkv, D), dtype=torch.uint8, device=dev)
+    lg.lg_sparse_attn_bwd(pat, q, k, v, o, do, lse, dq, dk, dv, scale, ws)
+    torch.cuda.synchronize()
+    assert lg.lg_device_status(0) == 0
+    nqb = S // 64
+    qrows = np.concatenate([np.arange(i * 64, i * 64 + 64) for i in (0, 7, nqb // 2, nqb - 1)])
+    krows = np.concatenate([np.arange(j * 64, j * 64 + 64) for j in (0, 1, nqb // 3, nqb - 1)])
+    for kvh in (0, Hkv - 1):
+        kh, vh = (t[0, :, kvh].float().cpu().numpy() for t in (k, v))
+        rdk = np.zeros((len(krows), D))
+        rdv = np.zeros((len(krows), D))
+        for g in range(G):
+            h = kvh * G + g
+            qh, doh = (t[0, :, h].float().cpu().numpy() for t in (q, do))
+            if g in (0, G - 1):
+                ro, _ = oracle.attention_rows(qh, kh, vh, qrows, op, scale)
+                assert_close(f"O h{h}", o[0, qrows, h].float().cpu().numpy(), ro)
+                rdq, _ = oracle.attention_backward_rows(qh, kh, vh, doh, qrows, op, scale)
+                assert_close(f"dQ h{h}", dq[0, qrows, h].cpu().numpy(), rdq)
+            a, b = oracle.attention_backward_kv_rows(qh, kh, vh, doh, krows, op, scale, chunk=256)
+            rdk += a
+            rdv += b
+        assert_close(f"dK kvh{kvh}", dk[0, krows, kvh].cpu().numpy(), rdk)
+        assert_close(f"dV kvh{kvh}", dv[0, krows, kvh].cpu().numpy(), rdv)
