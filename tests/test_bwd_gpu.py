@@ -70,6 +70,7 @@ SMALL = [
     (1, 1280, 2, 2, 128, lg.Pattern(64, 0, 1, 0), torch.float32),   # diagonal only
     (2, 640, 2, 2, 128, lg.Pattern.full(64), torch.float32),        # dense causal, odd 128-row step count
     (1, 1024, 2, 2, 128, lg.Pattern(64, 1, 4, 0), torch.bfloat16),  # attention sink at head dim 128, bf16 O
+    (1, 512, 8, 1, 128, lg.Pattern(64, 1, 2, 0), torch.float32),    # 8 query heads per KV head
 ]
 
 
