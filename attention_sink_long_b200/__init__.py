@@ -25,7 +25,7 @@ INT32_MAX = 2**31 - 1
 __all__ = [
     "LgError", "Pattern", "lib", "lg_strerror", "lg_version",
     "lg_pattern_expand", "lg_pattern_expand_t", "lg_pattern_pairs", "lg_pattern_iterate_device",
-    "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd", "lg_sparse_attn_fwd_varlen",
+    "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd", "lg_sparse_attn_fwd_varlen", "lg_sparse_attn_fwd_fp8qk",
     "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd", "lg_sparse_attn_bwd_varlen",
     "lg_sparse_decode_splits", "lg_sparse_decode_workspace", "lg_sparse_decode",
     "lg_sparse_decode_noalloc", "lg_kv_compact_rows", "lg_kv_compact", "lg_kv_compact_paged", "lg_kv_append_paged",
@@ -35,6 +35,7 @@ __all__ = [
 EXPORTED_SYMBOLS = (
     "lg_strerror", "lg_version", "lg_pattern_expand", "lg_pattern_expand_t", "lg_pattern_pairs",
     "lg_pattern_iterate_device", "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd", "lg_sparse_attn_fwd_varlen",
+    "lg_sparse_attn_fwd_fp8qk",
     "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd", "lg_sparse_attn_bwd_varlen", "lg_sparse_decode_splits",
     "lg_sparse_decode_workspace", "lg_sparse_decode", "lg_sparse_decode_noalloc", "lg_kv_compact_rows",
     "lg_kv_compact", "lg_kv_compact_paged", "lg_kv_append_paged", "lg_sparse_decode_paged", "lg_exp2_device",
@@ -80,6 +81,8 @@ _SIGS = {
                            + [_c_f, _c_vp, _c_sz, _c_vp]),
     "lg_sparse_attn_fwd_varlen": (_c_i32, [_P(_lg_pattern_t), _c_vp, _c_vp, _c_vp, _c_vp, _c_i32, _c_vp, _c_vp]
                                   + [_c_i32] * 6 + [_c_f, _c_vp]),
+    "lg_sparse_attn_fwd_fp8qk": (_c_i32, [_P(_lg_pattern_t), _c_vp, _c_vp, _c_vp, _c_f, _c_f, _c_vp, _c_i32, _c_vp]
+                                 + [_c_i32] * 5 + [_c_f, _c_vp]),
     "lg_sparse_attn_bwd_workspace": (_c_i32, [_P(_lg_pattern_t)] + [_c_i32] * 5 + [_P(_c_sz)]),
     "lg_sparse_attn_bwd": (_c_i32, [_P(_lg_pattern_t)] + [_c_vp] * 4 + [_c_i32] + [_c_vp] * 5 + [_c_i32] * 6
                            + [_c_f, _c_vp, _c_sz, _c_vp]),
@@ -271,6 +274,26 @@ def lg_sparse_attn_fwd_varlen(pattern, q, k, v, o, lse, cu_seqlens, max_seqlen: 
                                            o.data_ptr(), odt, _ptr(lse), cu_seqlens.data_ptr(), B, total,
                                            int(max_seqlen), H, Hkv, D, float(scale), _stream(stream)),
            "lg_sparse_attn_fwd_varlen")
+
+
+def lg_sparse_attn_fwd_fp8qk(pattern, q8, k8, v, q_descale: float, k_descale: float, o, lse, scale: float,
+                             stream=None):
+    """q8 [B,S,H,128], k8 [B,S,Hkv,128] torch.float8_e4m3fn; v bf16; o bf16 or fp32; lse [B,H,S] or None.
+    S = q8 k8^T * q_descale * k_descale on the fp8 tensor-core path."""
+    import torch
+
+    B, S, H, D = q8.shape
+    Hkv = k8.shape[2]
+    _expect(q8, "q8", torch.float8_e4m3fn, (B, S, H, D))
+    _expect(k8, "k8", torch.float8_e4m3fn, (B, S, Hkv, D), q8.device)
+    _expect(v, "v", torch.bfloat16, (B, S, Hkv, D), q8.device)
+    odt = _dtype_code(o, "o")
+    _expect(o, "o", o.dtype, (B, S, H, D), q8.device)
+    if lse is not None:
+        _expect(lse, "lse", torch.float32, (B, H, S), q8.device)
+    _check(lib().lg_sparse_attn_fwd_fp8qk(ctypes.byref(_pat(pattern)), q8.data_ptr(), k8.data_ptr(), v.data_ptr(),
+                                          float(q_descale), float(k_descale), o.data_ptr(), odt, _ptr(lse), B, S, H,
+                                          Hkv, D, float(scale), _stream(stream)), "lg_sparse_attn_fwd_fp8qk")
 
 
 # ---------------------------------------------------------------- backward

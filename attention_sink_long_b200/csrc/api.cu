@@ -93,6 +93,21 @@ lg_status_t make_map(CUtensorMap* m, const void* base, int B, int S, int Hx, int
   return r == CUDA_SUCCESS ? LG_OK : LG_ERR_CUDA;
 }
 
+// The same over a byte tensor (fp8 e4m3 Q or K, head dim 128): box {128, 1, rows, 1},
+// one 128-byte panel per row.
+lg_status_t make_map_u8(CUtensorMap* m, const void* base, int B, int S, int Hx, int D, int rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (enc == nullptr) return LG_ERR_CUDA;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)Hx, (cuuint64_t)S, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)D, (cuuint64_t)Hx * D, (cuuint64_t)S * Hx * D};
+  const cuuint32_t box[4] = {128, 1, (cuuint32_t)rows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LG_OK : LG_ERR_CUDA;
+}
+
 // Decode split rule: about 256 KB of K+V per CTA, more splits when there are
 // too few (b, kv head) rows to fill the GPU.
 void decode_split_rule(int B, int Hkv, int D, int Lmax, int requested, int* ns_out, int* rps_out) {
@@ -249,6 +264,41 @@ lg_status_t lg_sparse_attn_fwd(const lg_pattern_t* p, const void* q, const void*
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.err = err;
   return cuda_status(lg::launch_fwd(D, tq, tk, tv, to, prm, B, static_cast<cudaStream_t>(stream)));
+}
+
+lg_status_t lg_sparse_attn_fwd_fp8qk(const lg_pattern_t* p, const void* q8, const void* k8, const void* v,
+                                     float q_descale, float k_descale, void* o, int32_t o_dtype, float* lse, int32_t B,
+                                     int32_t S, int32_t H, int32_t Hkv, int32_t D, float scale, lg_stream_t stream) {
+  lg_status_t st = check_prefill_shape(p, B, S, H, Hkv, D);
+  if (st != LG_OK) return st;
+  if (q8 == nullptr || k8 == nullptr || v == nullptr || o == nullptr) return LG_ERR_INVALID_ARG;
+  if (o_dtype != LG_BF16 && o_dtype != LG_F32) return LG_ERR_INVALID_ARG;
+  const float sc = scale * q_descale * k_descale;
+  if (!(scale > 0.f) || !(q_descale > 0.f) || !(k_descale > 0.f) || !isfinite(sc) || !(sc > 0.f))
+    return LG_ERR_INVALID_ARG;
+  if (D != 128) return LG_ERR_UNSUPPORTED;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return LG_ERR_UNSUPPORTED;
+  unsigned int* err = error_word(&st);
+  if (st != LG_OK) return st;
+  CUtensorMap tq, tk, tv, to;
+  if ((st = make_map_u8(&tq, q8, B, S, H, D, 128)) != LG_OK) return st;
+  if ((st = make_map_u8(&tk, k8, B, S, Hkv, D, 64)) != LG_OK) return st;
+  if ((st = make_map(&tv, v, B, S, Hkv, D, 64)) != LG_OK) return st;
+  if ((st = make_map(&to, o_dtype == LG_F32 ? v : o, B, S, H, D, 64)) != LG_OK) return st;
+  lg::FwdParams prm;
+  prm.pat = *p;
+  prm.lse = lse;
+  prm.o_f32 = o_dtype == LG_F32 ? static_cast<float*>(o) : nullptr;
+  prm.S = S;
+  prm.H = H;
+  prm.Hkv = Hkv;
+  prm.nqb = S / 64;
+  prm.nqt = (S + 255) / 256;
+  prm.cu_seqlens = nullptr;
+  prm.max_len = S;
+  prm.scale_log2 = sc * 1.4426950408889634f;  // the dequantisation scales fold into the softmax scale
+  prm.err = err;
+  return cuda_status(lg::launch_fwd_fp8qk(tq, tk, tv, to, prm, B, static_cast<cudaStream_t>(stream)));
 }
 
 lg_status_t lg_sparse_attn_fwd_varlen(const lg_pattern_t* p, const void* q, const void* k, const void* v, void* o,

@@ -36,17 +36,25 @@
 
 namespace lg {
 
-template <int D>
+// F8: Q and K in fp8 e4m3 (S = Q K^T on the fp8 tensor-core path, K = 32 per
+// MMA; head dim 128 only, one 128-byte panel per row); V, P and O as in bf16.
+template <int D, bool F8 = false>
 struct FwdLayout {
-  static constexpr int DP = D / 64;              // 64-element (128-byte) panels per row
+  static constexpr int DP = D / 64;              // 64-element (128-byte) bf16 panels per row
   static constexpr int NT = 2;                   // 128-row query tiles per CTA
   static constexpr int NS = 2;                   // K/V chunk stages
-  static constexpr int Q_BYTES = 128 * D * 2;    // one query tile
-  static constexpr int KVC_BYTES = 128 * D * 2;  // one K or V chunk (up to 128 rows)
+  static constexpr int QK_ELEM = F8 ? 1 : 2;     // bytes per Q / K element
+  static constexpr int Q_BYTES = 128 * D * QK_ELEM;   // one query tile
+  static constexpr int K_BYTES = 128 * D * QK_ELEM;   // one K chunk (up to 128 rows)
+  static constexpr int KVC_BYTES = 128 * D * 2;       // one V chunk
   static constexpr int OFF_Q = 0;                // NT tiles
   static constexpr int OFF_K = OFF_Q + NT * Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NS * KVC_BYTES;
+  static constexpr int OFF_V = OFF_K + NS * K_BYTES;
   static constexpr int OFF_BAR = OFF_V + NS * KVC_BYTES;
+  // The bf16 O tile of query tile t is staged at OFF_Q + t * O_STAGE for its
+  // TMA store: the Q tiles (and with F8 the K stages) are free by then.
+  static constexpr int O_STAGE = 128 * D * 2;
+  static_assert(NT * O_STAGE <= OFF_V, "O staging must fit in the Q / K area");
   static constexpr int NBAR = 1 + 3 * NS + NT * 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
@@ -56,12 +64,13 @@ struct FwdLayout {
   static constexpr int THREADS = 320;
 };
 
-template <int D>
-__global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
+template <int D, bool F8>
+__global__ void __launch_bounds__(FwdLayout<D, F8>::THREADS, 1)
     lg_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const FwdParams prm) {
-  using L = FwdLayout<D>;
+  using L = FwdLayout<D, F8>;
+  static_assert(!F8 || D == 128, "fp8 Q/K: head dim 128");
   constexpr int NS = L::NS;
   constexpr int NT = L::NT;
   extern __shared__ uint8_t smem_raw[];
@@ -143,7 +152,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
     if (lane == 0) {
       mbar_arrive_expect_tx(q_full, NT * L::Q_BYTES);
       for (int t = 0; t < NT; ++t)
-        for (int p = 0; p < L::DP; ++p)
+        for (int p = 0; p < (F8 ? 1 : L::DP); ++p)  // fp8: one 128-byte panel holds a whole row
           tma_load_4d(smem + L::OFF_Q + t * L::Q_BYTES + p * 16384, &tmQ, q_full, 64 * p, h,
                       base + 256 * span + 128 * t, bc);
       int c = 0;
@@ -154,10 +163,10 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
         const int st = c % NS;
         const uint32_t use = (uint32_t)(c / NS);
         if (use > 0 && !mbar_wait(&kv_empty[st], (use - 1) & 1, abort_flag, err, kErrFwdWait)) break;
-        mbar_arrive_expect_tx(&k_full[st], nb * 64 * D * 2);
+        mbar_arrive_expect_tx(&k_full[st], nb * 64 * D * L::QK_ELEM);
         for (int hb = 0; hb < nb; ++hb)
-          for (int p = 0; p < L::DP; ++p)
-            tma_load_4d(smem + L::OFF_K + st * L::KVC_BYTES + p * 16384 + hb * 8192, &tmK, &k_full[st], 64 * p, kvh,
+          for (int p = 0; p < (F8 ? 1 : L::DP); ++p)
+            tma_load_4d(smem + L::OFF_K + st * L::K_BYTES + p * 16384 + hb * 8192, &tmK, &k_full[st], 64 * p, kvh,
                         base + 64 * (hb == 0 ? j : j2), bc);
         mbar_arrive_expect_tx(&v_full[st], nb * 64 * D * 2);
         for (int hb = 0; hb < nb; ++hb)
@@ -201,14 +210,22 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
         const int st = c % NS;
         if (t == 0 && !mbar_wait(&k_full[st], (uint32_t)(c / NS) & 1, abort_flag, err, kErrFwdWait)) return false;
         tc_fence_after();
-        const uint32_t idesc = nb == 2 ? idesc_bf16(128, 128, false, false) : idesc_bf16(128, 64, false, false);
         const uint64_t a0 = dQ0 + (uint32_t)((t * L::Q_BYTES) >> 4);
-        const uint64_t b0 = dK0 + (uint32_t)((st * L::KVC_BYTES) >> 4);
+        const uint64_t b0 = dK0 + (uint32_t)((st * L::K_BYTES) >> 4);
         const uint32_t d = tmem + L::T_S + 128 * t;
+        if (F8) {
+          // e4m3 x e4m3, fp32 accumulate: K = 32 per MMA, 32 bytes per k-step in the row's panel
+          const uint32_t idesc = nb == 2 ? idesc_e4m3(128, 128) : idesc_e4m3(128, 64);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-          tc_mma_ss_if(leader, d, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 32; ++kk)
+            tc_mma_f8_ss_if(leader, d, a0 + (uint32_t)(kk * 2), b0 + (uint32_t)(kk * 2), idesc, kk > 0 ? 1u : 0u);
+        } else {
+          const uint32_t idesc = nb == 2 ? idesc_bf16(128, 128, false, false) : idesc_bf16(128, 64, false, false);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (uint32_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            tc_mma_ss_if(leader, d, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
+          }
         }
         tc_commit_if(leader, &tile_bars[4 * t + 0]);
         return true;
@@ -421,7 +438,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t o[32];
         tmem_ld32(t_o + (uint32_t)(32 * ch), o);
-        const uint32_t panel = sbase + L::OFF_Q + t * L::Q_BYTES + (uint32_t)((32 * ch) >> 6) * 16384;
+        const uint32_t panel = sbase + L::OFF_Q + t * L::O_STAGE + (uint32_t)((32 * ch) >> 6) * 16384;
         const int c0 = ((32 * ch) & 63) >> 3;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
@@ -445,7 +462,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
       // the next sequence of a packed batch.
       for (int hb = 0; hb < 2 && row0 + 64 * hb < len; ++hb)
         for (int p = 0; p < L::DP; ++p)
-          tma_store_4d(&tmO, smem + L::OFF_Q + t * L::Q_BYTES + p * 16384 + hb * 8192, 64 * p, h,
+          tma_store_4d(&tmO, smem + L::OFF_Q + t * L::O_STAGE + p * 16384 + hb * 8192, 64 * p, h,
                        base + row0 + 64 * hb, bc);
       bulk_commit();
       bulk_wait_all();
@@ -460,22 +477,27 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
   }
 }
 
-template <int D>
+template <int D, bool F8>
 cudaError_t launch_fwd_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
                             const FwdParams& prm, int B, cudaStream_t stream) {
-  using L = FwdLayout<D>;
+  using L = FwdLayout<D, F8>;
   static_assert(L::ALLOC <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(lg_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+  cudaError_t e = cudaFuncSetAttribute(lg_fwd_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (e != cudaSuccess) return e;
   dim3 grid(prm.nqt, prm.H, B);
-  lg_fwd_kernel<D><<<grid, L::THREADS, L::ALLOC, stream>>>(tq, tk, tv, to, prm);
+  lg_fwd_kernel<D, F8><<<grid, L::THREADS, L::ALLOC, stream>>>(tq, tk, tv, to, prm);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const FwdParams& prm, int B, cudaStream_t stream) {
-  if (D == 64) return launch_fwd_impl<64>(tq, tk, tv, to, prm, B, stream);
-  return launch_fwd_impl<128>(tq, tk, tv, to, prm, B, stream);
+  if (D == 64) return launch_fwd_impl<64, false>(tq, tk, tv, to, prm, B, stream);
+  return launch_fwd_impl<128, false>(tq, tk, tv, to, prm, B, stream);
+}
+
+cudaError_t launch_fwd_fp8qk(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& to, const FwdParams& prm, int B, cudaStream_t stream) {
+  return launch_fwd_impl<128, true>(tq, tk, tv, to, prm, B, stream);
 }
 
 }  // namespace lg

@@ -52,7 +52,7 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--workload", choices=["step32k", "fwd128k", "bwd128k", "decode", "handoff", "blocksparse128k", "varlen", "decode_paged",
-                                               "gqa32k"],
+                                               "gqa32k", "fp8qk32k"],
                     default="step32k")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -139,6 +139,14 @@ def workload(name):
         return {"workload": "128K block-sparse prefill forward {64,1,16,32}",
                 "prefill": {"B": 1, "S": 131072, "H": 32, "Hkv": 32, "D": D},
                 "fwd": [("block-sparse", BLOCK_SPARSE)], "bwd": [], "decode": None}
+    if name == "fp8qk32k":
+        # Throughput experiment (no fp8 claim on the pages): Q and K arrive in fp8 e4m3 with
+        # dequantisation scales, S runs on the fp8 tensor-core path, P V in bf16.
+        return {"workload": "fp8 Q/K forward 32K (S on the fp8 path, P V bf16): sink+window + dense, "
+                            "B1 H32 D128",
+                "prefill": {"B": 1, "S": 32768, "H": 32, "Hkv": 32, "D": D},
+                "fwd": [("sink+window fp8qk", SINK_WINDOW), ("dense fp8qk", FULL)], "bwd": [], "decode": None,
+                "fp8qk": True}
     if name == "gqa32k":
         return {"workload": "grouped-query 32K: fwd + training bwd sink+window {64,1,64,0}, H32 Hkv8 D128",
                 "prefill": {"B": 1, "S": 32768, "H": 32, "Hkv": 8, "D": D},
@@ -268,10 +276,15 @@ class CudaStep:
             B, S, H, Hkv, D = pf["B"], pf["S"], pf["H"], pf["Hkv"], pf["D"]
             self.scale = 1.0 / math.sqrt(D)
             self.q, self.k, self.v, self.do = si.prefill_inputs_device(B, S, H, Hkv, D, device, with_dout=True)
+            if wl.get("fp8qk"):
+                # caller-side quantisation (outside the timed step): e4m3 with scales 4 and 2
+                self.q8 = (self.q.float() * 4.0).to(torch.float8_e4m3fn)
+                self.k8 = (self.k.float() * 2.0).to(torch.float8_e4m3fn)
             self.o = {n: torch.empty_like(self.q) for n, _ in wl["fwd"]}
             self.lse = {n: torch.empty(B, H, S, dtype=torch.float32, device=device) for n, _ in wl["fwd"]}
             for n, p in wl["fwd"]:
-                self.parts.append((f"fwd {n}", "fwd", 4 * D * pairs_of(p, S) * B * H, None, 1))
+                self.parts.append((f"fwd {n}", "fwd_fp8qk" if wl.get("fp8qk") else "fwd",
+                                   4 * D * pairs_of(p, S) * B * H, None, 1))
             if wl["bwd"] and not self._bwd_available(pf, wl["bwd"][0][1]):
                 wl = dict(wl, bwd=[], workload=wl["workload"] + " (backward not available in this build)")
                 self.wl = wl
@@ -396,7 +409,11 @@ class CudaStep:
         lg, wl = self.lg, self.wl
         i = 0
         for n, p in wl["fwd"]:
-            lg.lg_sparse_attn_fwd(p, self.q, self.k, self.v, self.o[n], self.lse[n], self.scale)
+            if wl.get("fp8qk"):
+                lg.lg_sparse_attn_fwd_fp8qk(p, self.q8, self.k8, self.v, 0.25, 0.5, self.o[n], self.lse[n],
+                                            self.scale)
+            else:
+                lg.lg_sparse_attn_fwd(p, self.q, self.k, self.v, self.o[n], self.lse[n], self.scale)
             if events is not None:
                 events[i].record(self.stream)
             i += 1
@@ -476,7 +493,8 @@ def host_buffers(step):
     torch = step.torch
     pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu())  # noqa: E731
     ins, outs = [], []
-    for name in ("q", "k", "v", "do", "dq_in", "kc", "vc", "lens", "hk", "hv", "vq", "vk", "vv", "vdo", "pq", "kpool",
+    names = ("q8", "k8", "v") if step.wl.get("fp8qk") else ("q", "k", "v", "do")
+    for name in names + ("dq_in", "kc", "vc", "lens", "hk", "hv", "vq", "vk", "vv", "vdo", "pq", "kpool",
                  "vpool", "ptable", "plens"):
         if hasattr(step, name):
             ins.append((name, getattr(step, name), pin(getattr(step, name))))
@@ -607,6 +625,9 @@ def cuda_arm(args, rank, world, dist):
         if kind.startswith("decode") or kind == "copy":
             r["gbs"] = round(nbytes / (ms * 1e-3) / 1e9, 1)
             r["frac_hbm"] = round(r["gbs"] / peaks["hbm_gbs"], 4)
+        elif kind == "fwd_fp8qk":
+            # half of the FLOPs (S) at the fp8 rate, twice bf16: the mixed peak is 4/3 of bf16's
+            r["frac_mixed_fp8_bf16_peak"] = round(r["useful_tflops"] / (tensor_peak * 4 / 3), 4)
         else:
             r["frac_bf16"] = round(r["useful_tflops"] / tensor_peak, 4)
         rows[name] = r
@@ -622,9 +643,12 @@ def cuda_arm(args, rank, world, dist):
         roof["peak_source"] = f"{peak_src} (copy bandwidth)"
     else:
         achieved = dflops / (dms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": tensor_peak, "unit": "TFLOP/s",
-                "frac": round(achieved / tensor_peak, 4)}
-        roof["peak_source"] = f"{peak_src} bf16 dense, {tensor_kind}"
+        pk = tensor_peak * 4 / 3 if dkind == "fwd_fp8qk" else tensor_peak
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(pk, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / pk, 4)}
+        roof["peak_source"] = f"{peak_src} bf16 dense, {tensor_kind}" + (
+            "; x 4/3: S (half the FLOPs) on the fp8 path at twice the bf16 rate (nominal ratio)"
+            if dkind == "fwd_fp8qk" else "")
     roof["traffic"] = recorded_traffic(dname)
     roof["kernel"] = dname
 

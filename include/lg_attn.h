@@ -151,6 +151,21 @@ lg_status_t lg_sparse_attn_fwd(const lg_pattern_t* pattern, const void* q, const
                                int32_t D, float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream);
 
 /*
+ * The forward above with Q and K in fp8 e4m3 (one byte each, head dim 128):
+ * S = (q8 k8^T) * q_descale * k_descale, computed on the fp8 tensor-core path
+ * at twice the bf16 rate; the softmax, P V (bf16) and the outputs are those of
+ * lg_sparse_attn_fwd. A throughput experiment: the pages make no fp8 claim,
+ * and the result is exact attention over the dequantised Q and K (the
+ * quantisation error is the caller's). Device pointers: q8 [B,S,H,128],
+ * k8 [B,S,Hkv,128] e4m3 bytes; v bf16; o, lse as lg_sparse_attn_fwd.
+ * Errors: those of lg_sparse_attn_fwd; LG_ERR_INVALID_ARG for a descale that
+ * is not positive and finite; LG_ERR_UNSUPPORTED for D != 128.
+ */
+lg_status_t lg_sparse_attn_fwd_fp8qk(const lg_pattern_t* pattern, const void* q8, const void* k8, const void* v,
+                                     float q_descale, float k_descale, void* o, int32_t o_dtype, float* lse, int32_t B,
+                                     int32_t S, int32_t H, int32_t Hkv, int32_t D, float scale, lg_stream_t stream);
+
+/*
  * The forward above for a batch of sequences of different lengths, packed
  * one after another (the prefill of several prompts; Abstract and summary,
  * "Key results": 1.67x prefill). Sequence b is rows [cu_seqlens[b],

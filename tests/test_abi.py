@@ -290,3 +290,21 @@ def test_bwd_varlen_argument_errors():
     assert call(ws=None) == 3
     assert call(wsb=1024) == 3
     assert call(ws=0x100080) == 2     # workspace not 256-byte aligned
+
+
+def test_fwd_fp8qk_argument_errors():
+    L = lg.lib()
+    p = lg._lg_pattern_t(64, 1, 64, 0)
+
+    def call(q=0x10000, qd=1.0, kd=1.0, B=1, S=1024, H=4, Hkv=4, D=128, odt=0, scale=0.088):
+        return L.lg_sparse_attn_fwd_fp8qk(ctypes.byref(p), q, 0x20000, 0x30000, qd, kd, 0x40000, odt, 0x50000, B, S,
+                                          H, Hkv, D, scale, None)
+
+    assert call(q=None) == 1
+    assert call(qd=0.0) == 1
+    assert call(kd=-2.0) == 1
+    assert call(qd=float("inf")) == 1
+    assert call(odt=5) == 1
+    assert call(D=64) == 2            # fp8 Q/K: head dim 128 only
+    assert call(S=1000) == 2
+    assert call(q=0x10008) == 2
