@@ -133,7 +133,8 @@ cudaError_t launch_bwd_dq(const float* dq_acc, void* dq, int dq_f32, float scale
 }
 
 // ---------------------------------------------------------------------------
-// 2. main kernel.
+// 2. main kernel for head dim 64 (head dim 128 runs lg_bwd128_kernel, in
+// bwd128_sm100.cu). The template keeps D general; only D = 64 is instantiated.
 //
 // CTA per (128-row KV tile = KV blocks 2u and 2u+1, KV head, batch); it walks
 // the union of the two blocks' query-block lists (a contiguous range, see
@@ -649,13 +650,11 @@ static cudaError_t launch_bwd_impl(const CUtensorMap& tq, const CUtensorMap& tk,
 cudaError_t launch_bwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv, const BwdParams& prm,
                        int B, cudaStream_t stream) {
+  // Head dim 128 (with or without query-head groups) runs the 128-row-step
+  // kernel; this one serves head dim 64.
   if (D == 128) return launch_bwd128(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
-  if (prm.split_lo) {
-    if (D == 64) return launch_bwd_impl<64, true>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
-    return launch_bwd_impl<128, true>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
-  }
-  if (D == 64) return launch_bwd_impl<64, false>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
-  return launch_bwd_impl<128, false>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
+  if (prm.split_lo) return launch_bwd_impl<64, true>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
+  return launch_bwd_impl<64, false>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
 }
 
 }  // namespace lg
