@@ -52,7 +52,7 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--workload", choices=["step32k", "fwd128k", "bwd128k", "decode", "handoff", "blocksparse128k", "varlen", "decode_paged",
-                                               "gqa32k", "fp8qk32k"],
+                                               "gqa32k", "fp8qk32k", "decode_gqa"],
                     default="step32k")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -139,6 +139,9 @@ def workload(name):
         return {"workload": "128K block-sparse prefill forward {64,1,16,32}",
                 "prefill": {"B": 1, "S": 131072, "H": 32, "Hkv": 32, "D": D},
                 "fwd": [("block-sparse", BLOCK_SPARSE)], "bwd": [], "decode": None}
+    if name == "decode_gqa":
+        return {"workload": "grouped-query decode over the sink+window cache: B32 H32 Hkv8 D128, 4160 rows",
+                "prefill": None, "fwd": [], "bwd": [], "decode": {"B": 32, "H": 32, "Hkv": 8, "D": D, "L": 4160}}
     if name == "fp8qk32k":
         # Throughput experiment (no fp8 claim on the pages): Q and K arrive in fp8 e4m3 with
         # dequantisation scales, S runs on the fp8 tensor-core path, P V in bf16.
@@ -307,7 +310,8 @@ class CudaStep:
             self.dws = torch.empty(max(lg.lg_sparse_decode_workspace(B, H, Hkv, D, L), 1), dtype=torch.uint8,
                                    device=device)
             nbytes = 2 * B * L * Hkv * D * 2 + 2 * B * H * D * 2
-            self.parts.append(("decode sparse layer", "decode", 4 * D * L * B * H, nbytes, 1))
+            name = "decode sparse layer" if Hkv == H else f"decode sparse layer, {H // Hkv} query heads per KV head"
+            self.parts.append((name, "decode", 4 * D * L * B * H, nbytes, 1))
             if "L_full" in dc:
                 Lf = dc["L_full"]
                 self.fq, self.fkc, self.fvc, self.flens = si.decode_inputs_device(B, H, Hkv, D, Lf, device, seed=2000)

@@ -86,3 +86,21 @@ def test_decode_full_layer_full_size_sampled():
                                vc[b:b + 1, :, h:h + 1].cpu(), [L], scale)
         assert_close(f"o[{b},{h}]", o[b, h].float().cpu().numpy(), ro[0, 0])
         assert_lse(f"lse[{b},{h}]", lse[b, h].cpu().numpy(), rl[0, 0])
+
+
+def test_gqa_decode_at_bench_size_sampled():
+    """Grouped-query decode (H32, Hkv8: the tensor-core path) at the batch-32,
+    4160-row size the bench times, ragged lengths: sampled (b, h) vs the oracle."""
+    B, H, Hkv, D, L = 32, 32, 8, 128, 4160
+    dev = torch.device("cuda")
+    lens = [L - 61 * b for b in range(B)]
+    q, kc, vc, cl = si.decode_inputs_device(B, H, Hkv, D, L, dev, lens=lens)
+    scale = 1.0 / math.sqrt(D)
+    o, lse = run_decode(q, kc, vc, cl, scale)
+    G = H // Hkv
+    for b, h in ((0, 0), (5, 17), (31, 31), (16, 3), (9, 12)):
+        n = lens[b]
+        ro, rl = oracle.decode(q[b:b + 1, h:h + 1].cpu(), kc[b:b + 1, :n, h // G:h // G + 1].cpu(),
+                               vc[b:b + 1, :n, h // G:h // G + 1].cpu(), np.array([n]), scale)
+        assert_close(f"o[{b},{h}]", o[b, h].float().cpu().numpy(), ro[0, 0])
+        assert_lse(f"lse[{b},{h}]", lse[b, h].cpu().numpy(), rl[0, 0])
