@@ -267,3 +267,23 @@ def test_varlen_bench_workload_sampled():
         rdk, rdv = oracle.attention_backward_kv_rows(qh, kh, vh, doh, krows, op, scale, chunk=256)
         assert_close(f"dK seq{b} h{h}", dk[s0 + krows, h].cpu().numpy(), rdk)
         assert_close(f"dV seq{b} h{h}", dv[s0 + krows, h].cpu().numpy(), rdv)
+
+
+def test_varlen_zero_length_sequence():
+    """An empty sequence between two others: forward and backward leave it
+    out, the others match the oracle."""
+    lens, H, Hkv, D = [192, 0, 320], 2, 2, 128
+    total = sum(lens)
+    q, k, v, do = si.prefill_inputs(1, total, H, Hkv, D, seed=si.SEED_BASE + 113, with_dout=True)
+    q, k, v, do = q[0], k[0], v[0], do[0]
+    cu = [0, 192, 192, 512]
+    scale = 1.0 / math.sqrt(D)
+    dq, dk, dv = run_varlen_fwd_bwd((64, 1, 2, 0), q, k, v, do, cu, 320, scale)
+    assert lg.lg_device_status(0) == 0
+    p = oracle.Pattern(64, 1, 2, 0)
+    for s0, s1 in ((0, 192), (192, 512)):
+        rdq, rdk, rdv, _ = oracle.attention_backward(q[None, s0:s1], k[None, s0:s1], v[None, s0:s1],
+                                                     do[None, s0:s1], p, scale)
+        assert_close(f"dQ {s0}", dq[s0:s1].cpu().numpy(), rdq[0])
+        assert_close(f"dK {s0}", dk[s0:s1].cpu().numpy(), rdk[0])
+        assert_close(f"dV {s0}", dv[s0:s1].cpu().numpy(), rdv[0])
