@@ -7,13 +7,18 @@
 // static pattern can still reach, a full layer's holds all of them; decode is
 // one query row attending to every cached row, so it is a pure HBM stream.
 //
-// Grid (splits, Hkv, B), 128 threads. D/8 threads share one cache row (16 B
-// each, one non-allocating vector load for K and one for V); a warp covers
-// 32*8/D rows per step and U steps are unrolled so each thread has 2*U loads
-// in flight. All G = H/Hkv query heads of a KV head are served by the same
-// CTA, so K/V bytes are read once per KV head. Each CTA reduces its rows to a
-// partial (o, lse); with more than one split the last CTA of each (b, kv head)
-// -- found through an atomic ticket, with no waiting -- merges the partials.
+// Two kernels, both with grid (splits, Hkv, B) and 128 threads, and both
+// serving all G = H/Hkv query heads of a KV head from one CTA so K/V bytes are
+// read once per KV head:
+//   lg_decode_kernel (G = 1): D/8 threads share one cache row (16 B each, one
+//     non-allocating vector load for K and one for V); a warp covers 32*8/D
+//     rows per step and U steps are unrolled so each thread has 2*U loads in
+//     flight.
+//   lg_decode_mma_kernel (G >= 2): cache blocks staged in shared memory and
+//     computed with warp tensor-core MMAs, the heads on the M side (below).
+// Each CTA reduces its rows to a partial (o, lse); with more than one split
+// the last CTA of each (b, kv head) -- found through an atomic ticket, with no
+// waiting -- merges the partials.
 //
 // Paged caches (PAGED = true): cache row r of sequence b lives in page
 // block_table[b][r / 64] at page row r % 64, every page [64, Hkv, D]; a page
@@ -21,6 +26,9 @@
 #include "lg_common.cuh"
 #include "lg_kernels.h"
 
+// Grouped-query kernel: cache rows per staged block and stages in flight
+// (measured: 64 rows and two stages beat 128-row blocks and three or four
+// stages, which leave fewer CTAs per SM).
 #ifndef LG_DECODE_MMA_BR
 #define LG_DECODE_MMA_BR 64
 #endif
