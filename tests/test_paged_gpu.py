@@ -146,8 +146,9 @@ def test_sink_window_ring_never_needs_more_pages():
     assert sorted(pc.table[0].tolist()) == list(range(4))  # the same four pages, permuted
 
 
-def test_paged_decode_equals_contiguous_bitwise_at_decode_size():
-    B, H, Hkv, D, L = 32, 32, 32, 128, 4160
+@pytest.mark.parametrize("H,Hkv", [(32, 32), (32, 8)], ids=["mha", "gqa4"])
+def test_paged_decode_equals_contiguous_bitwise_at_decode_size(H, Hkv):
+    B, D, L = 32, 128, 4160
     MB = L // 64
     dev = torch.device("cuda")
     q = si.device_normal((B, H, D), si.SEED_BASE + 0, dev)
@@ -172,10 +173,12 @@ def test_paged_decode_equals_contiguous_bitwise_at_decode_size():
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
     assert torch.equal(l1, l2)
     # and one sampled (b, h) against the oracle
+    G = H // Hkv
     for b, h in ((0, 0), (31, 17)):
         n = int(lens[b])
-        ro, rl = oracle.decode(q[b:b + 1, h:h + 1].cpu(), kc[b:b + 1, :n, h:h + 1].cpu(),
-                               vc[b:b + 1, :n, h:h + 1].cpu(), np.array([n]), 1 / math.sqrt(D))
+        kv = h // G
+        ro, rl = oracle.decode(q[b:b + 1, h:h + 1].cpu(), kc[b:b + 1, :n, kv:kv + 1].cpu(),
+                               vc[b:b + 1, :n, kv:kv + 1].cpu(), np.array([n]), 1 / math.sqrt(D))
         assert_close(f"o b{b} h{h}", o2[b, h].float().cpu().numpy()[None], ro[0])
         assert abs(l2[b, h].item() - rl[0, 0]) <= LSE_TOL
 
