@@ -119,24 +119,6 @@ __global__ void __launch_bounds__(448, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Launch order: first the heavy KV tiles (those a sink or strided block makes
-  // visible to many more queries, listed by the host) of every head, then the
-  // other tiles head by head in ascending order.
-  int u, h;
-  {
-    const int Lx = blockIdx.x;
-    const int nh = prm.n_heavy;
-    if (Lx < nh * prm.Hkv) {
-      u = prm.heavy[Lx / prm.Hkv];
-      h = Lx % prm.Hkv;
-    } else {
-      const int rest = prm.nkt - nh;
-      const int L2 = Lx - nh * prm.Hkv;
-      h = L2 / rest;
-      u = L2 % rest;
-      for (int k = 0; k < nh; ++k) u += (prm.heavy[k] <= u) ? 1 : 0;  // skip the heavy tiles
-    }
-  }
   const int b = blockIdx.y;
   // Sequence b occupies rows [base, base + len) at tensor-map batch coordinate
   // bc: the (B, S) layout, or the packed variable-length layout whose offsets
@@ -156,6 +138,40 @@ __global__ void __launch_bounds__(448, 1)
     bc = 0;
   }
   const int nqb = len / 64;
+  // Launch order: first the heavy KV tiles (those a sink or strided block makes
+  // visible to many more queries, listed by the host), then the other tiles
+  // head by head in ascending order. A heavy tile walks the query blocks from
+  // its own block to the end of the sequence, streaming the head's Q, dO and
+  // fp32 dQ accumulator (len x 1 KB). From 64K rows on that no longer fits
+  // beside other heads in the 126 MB L2, so when a head has several heavy
+  // tiles they run together, head by head, and all walk the query blocks
+  // downwards from the end: they then read and reduce into the same blocks at
+  // about the same time, and L2 serves one sweep to all of them (measured on
+  // the 128K block-sparse {64,1,16,32} backward: 22.0 ms against 24.3-26.5;
+  // at 32K, where each tile's own order hits L2 anyway, the change was within
+  // +-4 %). Otherwise the heavy tiles run interleaved across heads, ascending.
+  int u, h;
+  bool down = false;  // walk the query steps from the last to the first
+  {
+    const int Lx = blockIdx.x;
+    const int nh = prm.n_heavy;
+    if (Lx < nh * prm.Hkv) {
+      if (nh > 1 && len >= 65536) {
+        u = prm.heavy[Lx % nh];
+        h = Lx / nh;
+        down = true;
+      } else {
+        u = prm.heavy[Lx / prm.Hkv];
+        h = Lx % prm.Hkv;
+      }
+    } else {
+      const int rest = prm.nkt - nh;
+      const int L2 = Lx - nh * prm.Hkv;
+      h = L2 / rest;
+      u = L2 % rest;
+      for (int k = 0; k < nh; ++k) u += (prm.heavy[k] <= u) ? 1 : 0;  // skip the heavy tiles
+    }
+  }
   const size_t hrow0 = prm.cu_seqlens != nullptr ? (size_t)base : (size_t)b * prm.H * prm.S;
   const long long lin0 = prm.cu_seqlens != nullptr ? (long long)base : (long long)b * prm.S;
   // The tile's two KV blocks (ky = -1: the tile holds one block; its rows
@@ -175,6 +191,11 @@ __global__ void __launch_bounds__(448, 1)
   // accumulate over the whole group.
   const int G = GQA ? prm.H / prm.Hkv : 1;
   const int NT = G * N;
+  // First query block of step m (of its query head), in the tile's walk order.
+  auto step_block = [&](int m) -> int {
+    const int t = GQA ? m % N : m;
+    return q_first + 2 * (down ? N - 1 - t : t);
+  };
   unsigned int* err = prm.err;
 
   if (threadIdx.x == 0) {
@@ -219,7 +240,7 @@ __global__ void __launch_bounds__(448, 1)
         const int st = m & 1;
         const uint32_t use = (uint32_t)(m >> 1);
         const int hq = GQA ? h * G + m / N : h;  // query head
-        const int i0 = q_first + 2 * (GQA ? m % N : m);
+        const int i0 = step_block(m);
         // Both 64-row halves always load (rows past the sequence arrive as
         // zeros), so a stage never holds stale operands; LSE / Delta only
         // exist for blocks inside the sequence.
@@ -420,7 +441,7 @@ __global__ void __launch_bounds__(448, 1)
     for (; n < NT; ++n) {  // n: global step (query head h * G + n / N)
       const int st = n & 1;
       const uint32_t par = (uint32_t)n & 1;
-      const int i = q_first + 2 * (GQA ? n % N : n) + hf;  // this warp's query block
+      const int i = step_block(n) + hf;  // this warp's query block
       const bool vis = krow_live && i <= last && in_list(prm.pat, i, kvb);
       const bool diag = (i == kvb);
       if (!__all_sync(0xffffffffu, mbar_wait(&qq_full[st], (uint32_t)(n >> 1) & 1, abort_flag, err, kErrBwdWait)))
@@ -606,7 +627,7 @@ __global__ void __launch_bounds__(448, 1)
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
     for (int n = 0; n < NT; ++n) {  // n: global step
       const int hq = GQA ? h * G + n / N : h;  // query head
-      const int i0 = q_first + 2 * (GQA ? n % N : n);
+      const int i0 = step_block(n);
       const bool second = i0 + 1 <= last;  // the step's second query block is in the list range
       if (!__all_sync(0xffffffffu, mbar_wait(dq_full, (uint32_t)n & 1, abort_flag, err, kErrBwdWait))) break;
       tc_fence_after();

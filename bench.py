@@ -95,20 +95,21 @@ def sources_sha256(files):
     return h.hexdigest()
 
 
-def recorded_traffic(part_name):
-    """DRAM bytes per launch of this part from the committed ncu capture, or
-    None when there is none or the kernel's sources changed since."""
+def recorded_traffic(part_name, workload_name):
+    """DRAM bytes per launch of this part of this workload (the same launch
+    shape) from the committed ncu capture, or None when there is none or the
+    kernel's sources changed since."""
     try:
         with open(TRAFFIC_FILE) as f:
             table = json.load(f)
     except Exception:
         return None
-    e = table.get(part_name)
-    if not e:
-        return None
-    if sources_sha256(e["sources"]) != e["sources_sha256"]:
-        return None
-    return int(e["dram_bytes_per_launch"])
+    for e in table:
+        if e["part"] == part_name and workload_name in e["workloads"]:
+            if sources_sha256(e["sources"]) != e["sources_sha256"]:
+                return None
+            return int(e["dram_bytes_per_launch"])
+    return None
 
 
 def load_peaks():
@@ -653,7 +654,7 @@ def cuda_arm(args, rank, world, dist):
         roof["peak_source"] = f"{peak_src} bf16 dense, {tensor_kind}" + (
             "; x 4/3: S (half the FLOPs) on the fp8 path at twice the bf16 rate (nominal ratio)"
             if dkind == "fwd_fp8qk" else "")
-    roof["traffic"] = recorded_traffic(dname)
+    roof["traffic"] = recorded_traffic(dname, args.workload)
     roof["kernel"] = dname
 
     # End-to-end through the public API with pinned host buffers.

@@ -50,19 +50,28 @@ def test_peak_choice():
 
 
 def test_recorded_traffic_is_tied_to_kernel_sources(tmp_path, monkeypatch):
-    assert bench.recorded_traffic("no such part") is None
+    assert bench.recorded_traffic("no such part", "step32k") is None
     with open(bench.TRAFFIC_FILE) as f:
         table = json.load(f)
-    for name, e in table.items():
-        assert set(e) >= {"sources", "sources_sha256", "dram_bytes_per_launch", "capture"}
+    keys = [(e["part"], w) for e in table for w in e["workloads"]]
+    assert len(keys) == len(set(keys)), "one entry per part and workload"
+    for n, e in enumerate(table):
+        assert set(e) >= {"part", "workloads", "sources", "sources_sha256", "dram_bytes_per_launch", "capture"}
+        fresh = bench.sources_sha256(e["sources"]) == e["sources_sha256"]
+        for w in e["workloads"]:
+            bench.workload(w)  # a known workload
+            assert bench.recorded_traffic(e["part"], w) == (e["dram_bytes_per_launch"] if fresh else None)
         # a stale hash reads as "no capture for this kernel"
-        bad = dict(table)
-        bad[name] = dict(e, sources_sha256="0" * 64)
+        bad = [dict(x) for x in table]
+        bad[n]["sources_sha256"] = "0" * 64
         p = tmp_path / "t.json"
         p.write_text(json.dumps(bad))
         monkeypatch.setattr(bench, "TRAFFIC_FILE", str(p))
-        assert bench.recorded_traffic(name) is None
+        assert bench.recorded_traffic(e["part"], e["workloads"][0]) is None
         monkeypatch.setattr(bench, "TRAFFIC_FILE", os.path.join(ROOT, "profiles", "kernel_traffic.json"))
+    # the same part name in another workload (another launch shape) has no figure of its own
+    assert bench.recorded_traffic("bwd sink+window", "bwd128k") is None or any(
+        e["part"] == "bwd sink+window" and "bwd128k" in e["workloads"] for e in table)
 
 
 def test_workloads_and_useful_work():

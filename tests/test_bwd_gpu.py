@@ -113,13 +113,11 @@ def test_bwd_128k_sampled(pat):
         assert_close(f"dV h{h}", dv[0, krows, h].cpu().numpy(), rdv)
 
 
-def test_gqa_32k_sampled():
-    """The grouped-query workload bench.py times (32K sink+window, H32 Hkv8
-    D128, bf16 O as in training): O and dQ rows of sampled query blocks, and
-    dK / dV rows of sampled KV blocks -- the oracle sums those over the four
-    query heads of the KV head."""
-    B, S, H, Hkv, D = 1, 32768, 32, 8, 128
-    pat = lg.Pattern(64, 1, 64, 0)
+def _gqa_sampled(S, H, Hkv, pat, qblocks, kvblocks):
+    """O and dQ rows of sampled query blocks and dK / dV rows of sampled KV
+    blocks against the oracle, which sums dK / dV over the query heads of the
+    KV head (bf16 O as in training)."""
+    B, D = 1, 128
     op = oracle.Pattern(*pat)
     G = H // Hkv
     dev = torch.device("cuda")
@@ -133,9 +131,8 @@ def test_gqa_32k_sampled():
     lg.lg_sparse_attn_bwd(pat, q, k, v, o, do, lse, dq, dk, dv, scale, ws)
     torch.cuda.synchronize()
     assert lg.lg_device_status(0) == 0
-    nqb = S // 64
-    qrows = np.concatenate([np.arange(i * 64, i * 64 + 64) for i in (0, 7, nqb // 2, nqb - 1)])
-    krows = np.concatenate([np.arange(j * 64, j * 64 + 64) for j in (0, 1, nqb // 3, nqb - 1)])
+    qrows = np.concatenate([np.arange(i * 64, i * 64 + 64) for i in qblocks])
+    krows = np.concatenate([np.arange(j * 64, j * 64 + 64) for j in kvblocks])
     for kvh in (0, Hkv - 1):
         kh, vh = (t[0, :, kvh].float().cpu().numpy() for t in (k, v))
         rdk = np.zeros((len(krows), D))
@@ -153,3 +150,19 @@ def test_gqa_32k_sampled():
             rdv += b
         assert_close(f"dK kvh{kvh}", dk[0, krows, kvh].cpu().numpy(), rdk)
         assert_close(f"dV kvh{kvh}", dv[0, krows, kvh].cpu().numpy(), rdv)
+
+
+def test_gqa_32k_sampled():
+    """The grouped-query workload bench.py times: 32K sink+window, H32 Hkv8 D128."""
+    nqb = 32768 // 64
+    _gqa_sampled(32768, 32, 8, lg.Pattern(64, 1, 64, 0), (0, 7, nqb // 2, nqb - 1), (0, 1, nqb // 3, nqb - 1))
+
+
+def test_gqa_64k_block_sparse_sampled():
+    """64K block-sparse {64,1,16,32}, H8 Hkv2: a head has 17 heavy (sink /
+    strided) KV tiles, which then run together and walk the query blocks from
+    the end of the sequence downwards. Sampled: the sink and strided KV blocks
+    (each a heavy tile), a window-only block, the last block."""
+    nqb = 65536 // 64
+    _gqa_sampled(65536, 8, 2, lg.Pattern(64, 1, 16, 32), (0, 33, nqb // 2 + 5, nqb - 1),
+                 (0, 32, nqb // 2, nqb // 2 + 7, nqb - 1))
