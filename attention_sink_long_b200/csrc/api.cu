@@ -110,11 +110,24 @@ lg_status_t make_map_u8(CUtensorMap* m, const void* base, int B, int S, int Hx, 
 
 // Decode split rule: about 256 KB of K+V per CTA, more splits when there are
 // too few (b, kv head) rows to fill the GPU.
-void decode_split_rule(int B, int Hkv, int D, int Lmax, int requested, int* ns_out, int* rps_out) {
+void decode_split_rule(int B, int H, int Hkv, int D, int Lmax, int requested, int* ns_out, int* rps_out) {
   int rps, ns;
   if (requested > 0) {
     ns = imin(requested, Lmax);
     rps = (Lmax + ns - 1) / ns;
+  } else if (H / Hkv >= 2) {
+    // Query-head groups (the staged tensor-core kernel, three or more CTAs
+    // per SM): about 1024 cache rows per CTA, halved only while the grid
+    // would not cover the SMs. Shorter pieces lose more to each CTA's
+    // pipeline ramp and merge than they gain in balance (measured at B32
+    // x 4160 rows: 5.9 TB/s with 5 pieces against 5.65 with 9, and 3.3 ->
+    // 4.3 TB/s at B8; at 64K rows 6.7 against 6.5).
+    rps = 1024;
+    ns = (Lmax + rps - 1) / rps;
+    while (rps > 64 && (long long)B * Hkv * ns < 148LL) {
+      rps /= 2;
+      ns = (Lmax + rps - 1) / rps;
+    }
   } else {
     rps = (D == 128) ? 512 : 1024;
     ns = (Lmax + rps - 1) / rps;
@@ -586,7 +599,7 @@ lg_status_t lg_sparse_decode_splits(int32_t B, int32_t H, int32_t Hkv, int32_t D
     return LG_ERR_INVALID_ARG;
   if (H % Hkv != 0) return LG_ERR_INVALID_ARG;
   int ns, rps;
-  decode_split_rule(B, Hkv, D, Lmax, num_splits, &ns, &rps);
+  decode_split_rule(B, H, Hkv, D, Lmax, num_splits, &ns, &rps);
   *splits = ns;
   return LG_OK;
 }
@@ -622,7 +635,7 @@ static lg_status_t decode_common(const void* q, const void* k_cache, const void*
       (reinterpret_cast<uintptr_t>(cache_lens) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
     return LG_ERR_UNSUPPORTED;
   int ns, rps;
-  decode_split_rule(B, Hkv, D, Lmax, num_splits, &ns, &rps);
+  decode_split_rule(B, H, Hkv, D, Lmax, num_splits, &ns, &rps);
   size_t need = 0;
   lg_sparse_decode_workspace(B, H, Hkv, D, Lmax, num_splits, &need);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LG_ERR_WORKSPACE;
