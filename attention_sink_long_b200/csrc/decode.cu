@@ -317,16 +317,18 @@ __global__ void __launch_bounds__(128) lg_decode_kernel(const DecodeParams prm) 
 // accumulate) with the G heads on the M side (padded to 16). The scalar
 // kernel above spends 4 shuffles and 16 redundant exponentials per (row,
 // head) and falls to 0.2-0.5 of HBM bandwidth at G = 4-8.
-// The CTA stages 128-row blocks of K and V in shared memory with cp.async
+// The CTA stages 64-row blocks of K and V in shared memory with cp.async
 // (two stages, 16-byte chunks XOR-swizzled by row, zero-filled past the
 // cache), so a whole block is in flight while the previous one is computed;
-// warp w computes rows [32 w, 32 w + 32) of each block:
+// warp w computes rows [16 w, 16 w + 16) of each block:
 //   S (16 heads x 8 rows per MMA), K fragments by ldmatrix;
 //   P: the S accumulators of two 8-row tiles are, element for element, the A
 //     fragment of P for the next MMA;
 //   O (16 heads x 8 d per MMA) += P V, V fragments by ldmatrix.trans.
 // Each warp keeps an online softmax per head; the warps and the splits merge
-// as in the scalar kernel.
+// as in the scalar kernel, the warps' partial O passing through the (by then
+// idle) K/V stages, so the CTA's shared memory is the stages alone (64 KB at
+// D = 128: three CTAs per SM for every group size).
 __device__ __forceinline__ void mma_16816_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
@@ -377,8 +379,8 @@ __global__ void __launch_bounds__(128) lg_decode_mma_kernel(const DecodeParams p
   extern __shared__ __align__(128) uint8_t dsm[];
   __shared__ float sm_m[NW][G];
   __shared__ float sm_l[NW][G];
-  __shared__ float sm_acc[NW][G][D];
   __shared__ int sm_last;
+  static_assert(NW * G * D * 4 <= L::SMEM, "the warps' partial O fits the K/V stages");
 
   const int split = blockIdx.x;
   const int kvh = blockIdx.y;
@@ -546,6 +548,11 @@ __global__ void __launch_bounds__(128) lg_decode_mma_kernel(const DecodeParams p
     __syncthreads();  // the stage may be refilled once every warp has read it
   }
 
+  // Every copy has landed and every warp is past its last read of the
+  // stages (the loop ends on a barrier): they now hold the warps' partial O.
+  cp_async_wait<0>();
+  __syncthreads();
+  float(&sm_acc)[NW][G][D] = *reinterpret_cast<float(*)[NW][G][D]>(dsm);
   // Row sums over the four lanes of a fragment row group.
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
   l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
