@@ -116,18 +116,22 @@ void decode_split_rule(int B, int H, int Hkv, int D, int Lmax, int requested, in
     ns = imin(requested, Lmax);
     rps = (Lmax + ns - 1) / ns;
   } else if (H / Hkv >= 2) {
-    // Query-head groups (the staged tensor-core kernel, three or more CTAs
-    // per SM): about 1024 cache rows per CTA, halved only while the grid
-    // would not cover the SMs. Shorter pieces lose more to each CTA's
-    // pipeline ramp and merge than they gain in balance (measured at B32
-    // x 4160 rows: 5.9 TB/s with 5 pieces against 5.65 with 9, and 3.3 ->
-    // 4.3 TB/s at B8; at 64K rows 6.7 against 6.5).
-    rps = 1024;
-    ns = (Lmax + rps - 1) / rps;
-    while (rps > 64 && (long long)B * Hkv * ns < 148LL) {
-      rps /= 2;
-      ns = (Lmax + rps - 1) / rps;
+    // Query-head groups (the staged tensor-core kernel, three CTAs per SM).
+    // Many (b, kv head) pairs: about 1024 cache rows per CTA -- shorter
+    // pieces lose more to each CTA's pipeline ramp and merge than they gain
+    // in balance (B32 x 4160 rows, 8 KV heads: 5.9 TB/s with 5 pieces
+    // against 5.65 with 9; 64K rows: 6.7 against 6.5). At most 128 pairs:
+    // about 256 CTAs in one wave, which measured best from 16 to 128 pairs
+    // (e.g. 32 pairs: 3.5 TB/s with 8 pieces against 2.9-3.0 with 5; 128
+    // pairs: 5.4-5.7 with 2 against 4.5-5.0 with 5).
+    const long long pairs = (long long)B * Hkv;
+    if (pairs <= 128) {
+      ns = (int)((256 + pairs / 2) / pairs);
+      ns = imax(1, imin(ns, (Lmax + 63) / 64));
+    } else {
+      ns = (Lmax + 1023) / 1024;
     }
+    rps = (Lmax + ns - 1) / ns;
   } else {
     rps = (D == 128) ? 512 : 1024;
     ns = (Lmax + rps - 1) / rps;
