@@ -324,7 +324,7 @@ lg_status_t lg_kv_append_paged(const lg_pattern_t* pattern, const void* k_new, c
  * written to *splits. Always >= 1. One query head per KV head: pieces of 512
  * cache rows (1024 at D = 64), halved while B * Hkv * splits < 1184. Query-
  * head groups: pieces of 1024 rows when B * Hkv > 128, else about 256 / (B *
- * Hkv) pieces (about 256 CTAs). Pieces never go below 64 rows.
+ * Hkv) pieces (about 256 CTAs). Never more than ceil(Lmax / 64) pieces.
  */
 lg_status_t lg_sparse_decode_splits(int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax,
                                     int32_t num_splits, int32_t* splits);

@@ -155,6 +155,24 @@ def test_workspace_queries():
     assert lg.lg_sparse_decode_splits(2, 8, 8, 128, 100, 7) == 7
 
 
+@pytest.mark.parametrize("shape,splits", [
+    # one query head per KV head: 512-row pieces, halved while B * Hkv * splits < 1184
+    ((32, 32, 32, 128, 4160), 9), ((1, 32, 32, 128, 4160), 65), ((32, 32, 32, 64, 4160), 5),
+    # query-head groups, more than 128 (b, kv head) pairs: ~1024-row pieces
+    ((32, 32, 8, 128, 4160), 5), ((32, 32, 8, 128, 65536), 64), ((128, 32, 8, 128, 4160), 5),
+    # at most 128 pairs: about 256 CTAs, never more pieces than 64-row blocks
+    ((32, 32, 4, 128, 4160), 2), ((8, 32, 8, 128, 4160), 4), ((8, 32, 4, 128, 4160), 8),
+    ((1, 32, 8, 128, 4160), 32), ((1, 8, 1, 128, 100), 2), ((1, 8, 1, 128, 64), 1),
+])
+def test_decode_split_rule(shape, splits):
+    """The automatic split count the header documents (host logic only)."""
+    B, H, Hkv, D, L = shape
+    ns = lg.lg_sparse_decode_splits(B, H, Hkv, D, L)
+    assert ns == splits
+    rps = -(-L // ns)
+    assert -(-L // rps) == ns and ns <= -(-L // 64)  # equal pieces cover the cache, none empty
+
+
 # ---------------------------------------------------------------- prefill -> decode hand-off (host side)
 
 @pytest.mark.parametrize("p", [(64, 1, 64, 0), (64, 1, 16, 32), (64, 0, 2**31 - 1, 0), (64, 0, 1, 0), (64, 1, 4, 0),
