@@ -180,14 +180,21 @@ def attention_forward(q, k, v, p: Pattern, scale: float, mask=None):
     return o, lse
 
 
-def attention_backward(q, k, v, do, p: Pattern, scale: float, mask=None):
+def attention_backward(q, k, v, do, p: Pattern, scale: float, mask=None, o=None):
     """Analytic gradients of sum(O * dO) w.r.t. Q, K, V (dense per head).
 
     dV = P^T dO;  dP = dO V^T;  Delta = rowsum(P * dP);  dS = P (dP - Delta);
     dQ = scale dS K;  dK = scale dS^T Q.  GQA: dK, dV sum over the query heads
     of a KV group. Returns (dq, dk, dv, delta[B,H,S]).
+
+    With ``o`` given ([B,S,H,D], e.g. the forward output as stored in bf16),
+    Delta is taken as rowsum(dO * o) instead -- the identity rowsum(P * dP) =
+    dO . O evaluated on the O the backward is handed, which is how a
+    FlashAttention-2-style training backward (atlas.scime.ai summary,
+    "Approach") forms it. Everything else is unchanged.
     """
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    o_in = None if o is None else _f64(o)
     B, S, H, D = q.shape
     Hkv = k.shape[2]
     g = H // Hkv
@@ -204,7 +211,10 @@ def attention_backward(q, k, v, do, p: Pattern, scale: float, mask=None):
             P, _ = _masked_softmax(scale * (qh @ kk.T), mask)
             dv[b, :, kh] += P.T @ doh
             dP = doh @ vv.T
-            delta[b, h] = (P * dP).sum(axis=1)
+            if o_in is None:
+                delta[b, h] = (P * dP).sum(axis=1)
+            else:
+                delta[b, h] = (doh * o_in[b, :, h]).sum(axis=1)
             dS = P * (dP - delta[b, h][:, None])
             dq[b, :, h] = scale * (dS @ kk)
             dk[b, :, kh] += scale * (dS.T @ qh)

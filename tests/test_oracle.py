@@ -257,6 +257,26 @@ def test_gradients_match_torch_autograd(p):
     np.testing.assert_allclose(delta[0, 0], (out.detach().numpy() * do).sum(axis=1), atol=1e-12)
 
 
+def test_gradients_with_given_output_follow_its_delta():
+    """Delta from a given O: with the exact O the gradients are the autograd-pinned
+    ones (Delta = dO . O); with a perturbed O, Delta is rowsum(dO * O_given), and
+    dV (which has no Delta term) does not move while dQ and dK do."""
+    S, D, scale = 96, 8, 0.35
+    p = Pattern(16, 1, 2, 3)
+    q, do = rnd((1, S, 2, D), 50), rnd((1, S, 2, D), 51)
+    k, v = rnd((1, S, 1, D), 52), rnd((1, S, 1, D), 53)
+    o, _ = oracle.attention_forward(q, k, v, p, scale)
+    ref = oracle.attention_backward(q, k, v, do, p, scale)
+    got = oracle.attention_backward(q, k, v, do, p, scale, o=o)
+    for a, b in zip(ref, got):
+        np.testing.assert_allclose(a, b, atol=1e-12)
+    o2 = o + 0.01 * rnd(o.shape, 54)
+    dq2, dk2, dv2, delta2 = oracle.attention_backward(q, k, v, do, p, scale, o=o2)
+    np.testing.assert_allclose(delta2, np.einsum("bshd,bshd->bhs", do, o2), atol=1e-12)
+    np.testing.assert_allclose(dv2, ref[2], atol=1e-12)
+    assert np.abs(dq2 - ref[0]).max() > 1e-4 and np.abs(dk2 - ref[1]).max() > 1e-4
+
+
 def test_gqa_gradients_sum_over_group():
     S, D = 96, 8
     p = Pattern(16, 1, 2, 0)
