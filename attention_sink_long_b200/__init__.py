@@ -90,15 +90,15 @@ _SIGS = {
                                   + [_c_vp] + [_c_i32] * 6 + [_c_f, _c_vp, _c_sz, _c_vp]),
     "lg_sparse_decode_splits": (_c_i32, [_c_i32] * 6 + [_P(_c_i32)]),
     "lg_sparse_decode_workspace": (_c_i32, [_c_i32] * 6 + [_P(_c_sz)]),
-    "lg_sparse_decode": (_c_i32, [_c_vp] * 6 + [_c_i32] * 6 + [_c_f, _c_vp, _c_sz, _c_vp]),
-    "lg_sparse_decode_noalloc": (_c_i32, [_c_vp] * 6 + [_c_i32] * 6 + [_c_f, _c_vp]),
+    "lg_sparse_decode": (_c_i32, [_c_vp] * 5 + [_c_i32, _c_vp] + [_c_i32] * 6 + [_c_f, _c_vp, _c_sz, _c_vp]),
+    "lg_sparse_decode_noalloc": (_c_i32, [_c_vp] * 5 + [_c_i32, _c_vp] + [_c_i32] * 6 + [_c_f, _c_vp]),
     "lg_kv_compact_rows": (_c_i32, [_P(_lg_pattern_t), _c_i32, _P(_c_i32)]),
     "lg_kv_compact": (_c_i32, [_P(_lg_pattern_t), _c_vp, _c_vp] + [_c_i32] * 4 + [_c_vp, _c_vp, _c_i32, _c_vp, _c_vp]),
     "lg_kv_compact_paged": (_c_i32, [_P(_lg_pattern_t), _c_vp, _c_vp] + [_c_i32] * 4
                             + [_c_vp, _c_vp, _c_i64, _c_vp, _c_vp, _c_i32, _c_vp, _c_vp, _c_vp]),
     "lg_kv_append_paged": (_c_i32, [_P(_lg_pattern_t), _c_vp, _c_vp] + [_c_i32] * 3
                            + [_c_vp, _c_vp, _c_i64, _c_vp, _c_vp, _c_i32, _c_vp, _c_vp, _c_vp]),
-    "lg_sparse_decode_paged": (_c_i32, [_c_vp, _c_vp, _c_vp, _c_i64, _c_vp, _c_i32, _c_vp, _c_vp, _c_vp]
+    "lg_sparse_decode_paged": (_c_i32, [_c_vp, _c_vp, _c_vp, _c_i64, _c_vp, _c_i32, _c_vp, _c_vp, _c_i32, _c_vp]
                                + [_c_i32] * 5 + [_c_f, _c_vp, _c_sz, _c_vp]),
     "lg_exp2_device": (_c_i32, [_c_vp, _c_vp, _c_i64, _c_i32, _c_vp]),
     "lg_wait_selftest": (_c_i32, [_c_i64, _c_vp]),
@@ -206,10 +206,12 @@ def lg_pattern_pairs(pattern, seqlen: int) -> int:
     return out.value
 
 
-def lg_pattern_iterate_device(pattern, seqlen: int, tile_blocks: int, transpose: int, out, cap: int, stream=None):
-    """Runs the kernels' block iterator on the device into ``out`` (int32 CUDA tensor)."""
+def lg_pattern_iterate_device(pattern, seqlen: int, tile_blocks: int, mode: int, out, cap: int, stream=None):
+    """Runs the kernels' block iterators on the device into ``out`` (int32 CUDA
+    tensor); mode 0/1 forward/backward unions, 2 the forward's chunked walk,
+    3 the backward's paired KV tiles (see include/lg_attn.h)."""
     p = _pat(pattern)
-    _check(lib().lg_pattern_iterate_device(ctypes.byref(p), seqlen, tile_blocks, transpose, out.data_ptr(), cap,
+    _check(lib().lg_pattern_iterate_device(ctypes.byref(p), seqlen, tile_blocks, mode, out.data_ptr(), cap,
                                            _stream(stream)), "lg_pattern_iterate_device")
 
 
@@ -374,7 +376,8 @@ def lg_sparse_decode_workspace(B, H, Hkv, D, Lmax, num_splits=0) -> int:
 
 def lg_sparse_decode(q, k_cache, v_cache, cache_lens, o, lse, scale: float, num_splits: int = 0, workspace=None,
                      stream=None):
-    """q [B,H,D] bf16, caches [B,Lmax,Hkv,D] bf16, cache_lens [B] int32, o [B,H,D] bf16, lse [B,H] fp32 or None."""
+    """q [B,H,D] bf16, caches [B,Lmax,Hkv,D] bf16, cache_lens [B] int32, o [B,H,D] bf16 or fp32 (the
+    unrounded result), lse [B,H] fp32 or None."""
     import torch
 
     B, H, D = q.shape
@@ -383,12 +386,13 @@ def lg_sparse_decode(q, k_cache, v_cache, cache_lens, o, lse, scale: float, num_
     _expect(k_cache, "k_cache", torch.bfloat16, (B, Lmax, Hkv, D), q.device)
     _expect(v_cache, "v_cache", torch.bfloat16, (B, Lmax, Hkv, D), q.device)
     _expect(cache_lens, "cache_lens", torch.int32, (B,), q.device)
-    _expect(o, "o", torch.bfloat16, (B, H, D), q.device)
+    odt = _dtype_code(o, "o")
+    _expect(o, "o", o.dtype, (B, H, D), q.device)
     if lse is not None:
         _expect(lse, "lse", torch.float32, (B, H), q.device)
     ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().lg_sparse_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), cache_lens.data_ptr(),
-                                  o.data_ptr(), _ptr(lse), B, H, Hkv, D, Lmax, int(num_splits), float(scale),
+                                  o.data_ptr(), odt, _ptr(lse), B, H, Hkv, D, Lmax, int(num_splits), float(scale),
                                   _ptr(workspace), ws, _stream(stream)), "lg_sparse_decode")
 
 
@@ -480,12 +484,14 @@ def lg_sparse_decode_paged(q, k_pool, v_pool, block_table, cache_lens, o, lse, s
     P, Bt, MB, Hkv, _ = _expect_paged(k_pool, v_pool, block_table, None, cache_lens, None, None, D)
     if Bt != B:
         raise ValueError(f"block_table has {Bt} rows, expected {B}")
-    _expect(o, "o", torch.bfloat16, (B, H, D), q.device)
+    odt = _dtype_code(o, "o")
+    _expect(o, "o", o.dtype, (B, H, D), q.device)
     if lse is not None:
         _expect(lse, "lse", torch.float32, (B, H), q.device)
     ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().lg_sparse_decode_paged(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), P,
-                                        block_table.data_ptr(), MB, cache_lens.data_ptr(), o.data_ptr(), _ptr(lse),
+                                        block_table.data_ptr(), MB, cache_lens.data_ptr(), o.data_ptr(), odt,
+                                        _ptr(lse),
                                         B, H, Hkv, D, int(num_splits), float(scale), _ptr(workspace), ws,
                                         _stream(stream)), "lg_sparse_decode_paged")
 
@@ -496,20 +502,24 @@ def lg_sparse_decode_noalloc(q, k_cache, v_cache, cache_lens, o, lse, scale: flo
     workspace argument; the library's fixed 16 MiB device scratch array holds
     the split partials. Calls that overlap on the GPU share that array and race,
     so serialise them. The first call on a device resolves the array's address;
-    make it before any stream capture."""
+    make it before any stream capture. The tensors must live on the current
+    device: that device's array is the one the call uses."""
     import torch
 
     B, H, D = q.shape
     Lmax, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if q.device.type != "cuda" or q.device.index != torch.cuda.current_device():
+        raise ValueError(f"q: expected the current device cuda:{torch.cuda.current_device()}, got {q.device}")
     _expect(q, "q", torch.bfloat16, (B, H, D))
     _expect(k_cache, "k_cache", torch.bfloat16, (B, Lmax, Hkv, D), q.device)
     _expect(v_cache, "v_cache", torch.bfloat16, (B, Lmax, Hkv, D), q.device)
     _expect(cache_lens, "cache_lens", torch.int32, (B,), q.device)
-    _expect(o, "o", torch.bfloat16, (B, H, D), q.device)
+    odt = _dtype_code(o, "o")
+    _expect(o, "o", o.dtype, (B, H, D), q.device)
     if lse is not None:
         _expect(lse, "lse", torch.float32, (B, H), q.device)
     _check(lib().lg_sparse_decode_noalloc(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
-                                          cache_lens.data_ptr(), o.data_ptr(), _ptr(lse), B, H, Hkv, D, Lmax,
+                                          cache_lens.data_ptr(), o.data_ptr(), odt, _ptr(lse), B, H, Hkv, D, Lmax,
                                           int(num_splits), float(scale), _stream(stream)),
            "lg_sparse_decode_noalloc")
 

@@ -166,7 +166,7 @@ const char* lg_strerror(lg_status_t s) {
   return "unknown status";
 }
 
-int32_t lg_version(void) { return (1 << 16) | 0; }
+int32_t lg_version(void) { return (2 << 16) | 0; }
 
 // ---------------------------------------------------------------- pattern (host)
 lg_status_t lg_pattern_expand(const lg_pattern_t* p, int32_t seqlen, int32_t* row_ptr, int32_t* col, int64_t cap,
@@ -226,15 +226,20 @@ lg_status_t lg_pattern_pairs(const lg_pattern_t* p, int32_t seqlen, int64_t* pai
   return LG_OK;
 }
 
-lg_status_t lg_pattern_iterate_device(const lg_pattern_t* p, int32_t seqlen, int32_t tile_blocks, int32_t transpose,
+lg_status_t lg_pattern_iterate_device(const lg_pattern_t* p, int32_t seqlen, int32_t tile_blocks, int32_t mode,
                                       int32_t* out, int32_t cap, lg_stream_t stream) {
   lg_status_t st = check_pattern(p);
   if (st != LG_OK) return st;
   if (out == nullptr || seqlen <= 0 || seqlen % p->block_size != 0 || cap < 0) return LG_ERR_INVALID_ARG;
-  if (tile_blocks != 1 && tile_blocks != 2) return LG_ERR_UNSUPPORTED;
-  if (transpose != 0 && transpose != 1) return LG_ERR_INVALID_ARG;
+  if (mode < 0 || mode > 3) return LG_ERR_INVALID_ARG;
+  if (p->block_size != 64) return LG_ERR_UNSUPPORTED;
+  const bool ok_tiles = (mode == 0 && (tile_blocks == 1 || tile_blocks == 2 || tile_blocks == 4 || tile_blocks == 8)) ||
+                        (mode == 1 && (tile_blocks == 1 || tile_blocks == 2)) ||
+                        (mode == 2 && (tile_blocks == 4 || tile_blocks == 8)) || (mode == 3 && tile_blocks == 2);
+  if (!ok_tiles) return LG_ERR_UNSUPPORTED;
+  if (seqlen / 64 >= (1 << 23)) return LG_ERR_UNSUPPORTED;  // block << 8 must fit an int32
   return cuda_status(
-      lg::launch_pattern_iterate(*p, seqlen, tile_blocks, transpose, out, cap, static_cast<cudaStream_t>(stream)));
+      lg::launch_pattern_iterate(*p, seqlen, tile_blocks, mode, out, cap, static_cast<cudaStream_t>(stream)));
 }
 
 // ---------------------------------------------------------------- forward
@@ -614,22 +619,30 @@ lg_status_t lg_sparse_decode_workspace(int32_t B, int32_t H, int32_t Hkv, int32_
   lg_status_t st = lg_sparse_decode_splits(B, H, Hkv, D, Lmax, num_splits, &ns);
   if (st != LG_OK) return st;
   if (bytes == nullptr) return LG_ERR_INVALID_ARG;
-  if (ns == 1) {
-    *bytes = 0;
-    return LG_OK;
-  }
-  *bytes = round256((size_t)B * H * ns * D * 4) + round256((size_t)B * H * ns * 4) + round256((size_t)B * Hkv * 4);
+  *bytes = lg::decode_scratch_bytes(B, H, Hkv, D, ns);
   return LG_OK;
 }
 
-static lg_status_t decode_common(const void* q, const void* k_cache, const void* v_cache, const int32_t* cache_lens,
-                                 const int32_t* block_table, int32_t max_blocks, int64_t num_pages, void* o,
-                                 float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax,
-                                 int32_t num_splits, float scale, void* workspace, size_t workspace_bytes,
-                                 lg_stream_t stream) {
+}  // extern "C"
+
+namespace lg {
+
+// Bytes of split partials and tickets for ns pieces (0 for one piece): the
+// workspace layout of every decode entry point.
+size_t decode_scratch_bytes(int B, int H, int Hkv, int D, int ns) {
+  if (ns <= 1) return 0;
+  return round256((size_t)B * H * ns * D * 4) + round256((size_t)B * H * ns * 4) + round256((size_t)B * Hkv * 4);
+}
+
+lg_status_t decode_call(const void* q, const void* k_cache, const void* v_cache, const int32_t* cache_lens,
+                        const int32_t* block_table, int32_t max_blocks, int64_t num_pages, void* o, int32_t o_dtype,
+                        float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax, int32_t num_splits,
+                        float scale, void* workspace, size_t workspace_bytes, bool shrink_to_fit,
+                        cudaStream_t stream) {
   if (!q || !k_cache || !v_cache || !cache_lens || !o) return LG_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || Hkv <= 0 || D <= 0 || Lmax <= 0 || num_splits < 0) return LG_ERR_INVALID_ARG;
   if (H % Hkv != 0) return LG_ERR_INVALID_ARG;
+  if (o_dtype != LG_BF16 && o_dtype != LG_F32) return LG_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return LG_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return LG_ERR_UNSUPPORTED;
   const int G = H / Hkv;
@@ -640,15 +653,19 @@ static lg_status_t decode_common(const void* q, const void* k_cache, const void*
     return LG_ERR_UNSUPPORTED;
   int ns, rps;
   decode_split_rule(B, H, Hkv, D, Lmax, num_splits, &ns, &rps);
-  size_t need = 0;
-  lg_sparse_decode_workspace(B, H, Hkv, D, Lmax, num_splits, &need);
+  if (shrink_to_fit && num_splits == 0) {
+    // Automatic count and a fixed scratch size: fewer, longer pieces until the partials fit.
+    while (ns > 1 && decode_scratch_bytes(B, H, Hkv, D, ns) > workspace_bytes) --ns;
+    rps = (Lmax + ns - 1) / ns;
+    ns = (Lmax + rps - 1) / rps;
+  }
+  const size_t need = decode_scratch_bytes(B, H, Hkv, D, ns);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LG_ERR_WORKSPACE;
   if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return LG_ERR_UNSUPPORTED;
   lg_status_t st;
   unsigned int* err = error_word(&st);
   if (st != LG_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  lg::DecodeParams prm;
+  DecodeParams prm;
   prm.q = q;
   prm.k_cache = k_cache;
   prm.v_cache = v_cache;
@@ -657,6 +674,7 @@ static lg_status_t decode_common(const void* q, const void* k_cache, const void*
   prm.max_blocks = max_blocks;
   prm.num_pages = num_pages;
   prm.o = o;
+  prm.o_f32 = o_dtype == LG_F32 ? 1 : 0;
   prm.lse = lse;
   prm.part_o = nullptr;
   prm.part_lse = nullptr;
@@ -668,7 +686,8 @@ static lg_status_t decode_common(const void* q, const void* k_cache, const void*
     prm.part_lse = reinterpret_cast<float*>(w);
     w += round256((size_t)B * H * ns * 4);
     prm.tickets = reinterpret_cast<unsigned int*>(w);
-    st = cuda_status(cudaMemsetAsync(prm.tickets, 0, (size_t)B * Hkv * 4, s));
+    // The tickets must start at zero whatever the workspace holds.
+    st = cuda_status(cudaMemsetAsync(prm.tickets, 0, (size_t)B * Hkv * 4, stream));
     if (st != LG_OK) return st;
   }
   prm.B = B;
@@ -679,25 +698,31 @@ static lg_status_t decode_common(const void* q, const void* k_cache, const void*
   prm.rows_per_split = rps;
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.err = err;
-  return cuda_status(lg::launch_decode(D, G, prm, s));
+  return cuda_status(launch_decode(D, G, prm, stream));
 }
 
+}  // namespace lg
+
+extern "C" {
+
 lg_status_t lg_sparse_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* cache_lens,
-                             void* o, float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax,
-                             int32_t num_splits, float scale, void* workspace, size_t workspace_bytes,
+                             void* o, int32_t o_dtype, float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D,
+                             int32_t Lmax, int32_t num_splits, float scale, void* workspace, size_t workspace_bytes,
                              lg_stream_t stream) {
-  return decode_common(q, k_cache, v_cache, cache_lens, nullptr, 0, 0, o, lse, B, H, Hkv, D, Lmax, num_splits, scale,
-                       workspace, workspace_bytes, stream);
+  return lg::decode_call(q, k_cache, v_cache, cache_lens, nullptr, 0, 0, o, o_dtype, lse, B, H, Hkv, D, Lmax,
+                         num_splits, scale, workspace, workspace_bytes, false, static_cast<cudaStream_t>(stream));
 }
 
 lg_status_t lg_sparse_decode_paged(const void* q, const void* k_pool, const void* v_pool, int64_t num_pages,
                                    const int32_t* block_table, int32_t max_blocks, const int32_t* cache_lens, void* o,
-                                   float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t num_splits,
-                                   float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream) {
+                                   int32_t o_dtype, float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D,
+                                   int32_t num_splits, float scale, void* workspace, size_t workspace_bytes,
+                                   lg_stream_t stream) {
   lg_status_t st = check_paged(k_pool, v_pool, num_pages, block_table, max_blocks, cache_lens, B, Hkv, D);
   if (st != LG_OK) return st;
-  return decode_common(q, k_pool, v_pool, cache_lens, block_table, max_blocks, num_pages, o, lse, B, H, Hkv, D,
-                       64 * max_blocks, num_splits, scale, workspace, workspace_bytes, stream);
+  return lg::decode_call(q, k_pool, v_pool, cache_lens, block_table, max_blocks, num_pages, o, o_dtype, lse, B, H,
+                         Hkv, D, 64 * max_blocks, num_splits, scale, workspace, workspace_bytes, false,
+                         static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------- numerics

@@ -70,6 +70,25 @@ __device__ __forceinline__ void merge_state(float& m, float& l, float (&a)[E], f
   m = mn;
 }
 
+// Eight consecutive output elements a[e] * inv at element offset idx of o:
+// bf16 (round to nearest even, one 16-byte store) or, in the fp32 output
+// mode, the fp32 values themselves (two 16-byte stores).
+template <int D>
+__device__ __forceinline__ void store_o8(const DecodeParams& prm, size_t idx, const float (&a)[8], float inv) {
+  if (prm.o_f32) {
+    float4* d = reinterpret_cast<float4*>(static_cast<float*>(prm.o) + idx);
+    d[0] = make_float4(a[0] * inv, a[1] * inv, a[2] * inv, a[3] * inv);
+    d[1] = make_float4(a[4] * inv, a[5] * inv, a[6] * inv, a[7] * inv);
+  } else {
+    uint4 out;
+    out.x = pack_bf16x2(a[0] * inv, a[1] * inv);
+    out.y = pack_bf16x2(a[2] * inv, a[3] * inv);
+    out.z = pack_bf16x2(a[4] * inv, a[5] * inv);
+    out.w = pack_bf16x2(a[6] * inv, a[7] * inv);
+    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(prm.o) + idx) = out;
+  }
+}
+
 // The end of every decode kernel: merge the NW warp states (m, l in log2 units,
 // unnormalised o) of each query head in shared memory, then write o / lse
 // (one split) or the split's partial, and let the last CTA of each (b, kv
@@ -101,16 +120,10 @@ __device__ __forceinline__ void decode_finish(const DecodeParams& prm, const flo
       merge_state<8>(M, Lsum, A, sm_m[w][g], sm_l[w][g], a2);
     }
   }
-  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(prm.o);
   if (ns == 1) {
     if (owner) {
       const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-      uint4 out;
-      out.x = pack_bf16x2(A[0] * inv, A[1] * inv);
-      out.y = pack_bf16x2(A[2] * inv, A[3] * inv);
-      out.z = pack_bf16x2(A[4] * inv, A[5] * inv);
-      out.w = pack_bf16x2(A[6] * inv, A[7] * inv);
-      *reinterpret_cast<uint4*>(o + ((size_t)b * H + h) * D + 8 * c) = out;
+      store_o8<D>(prm, ((size_t)b * H + h) * D + 8 * c, A, inv);
       if (c == 0 && prm.lse != nullptr)
         prm.lse[(size_t)b * H + h] = Lsum > 0.f ? (M + __log2f(Lsum)) * 0.69314718055994531f : -INFINITY;
     }
@@ -159,12 +172,7 @@ __device__ __forceinline__ void decode_finish(const DecodeParams& prm, const flo
       Af[7] = fmaf(w, x1.w, Af[7]);
     }
     const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-    uint4 out;
-    out.x = pack_bf16x2(Af[0] * inv, Af[1] * inv);
-    out.y = pack_bf16x2(Af[2] * inv, Af[3] * inv);
-    out.z = pack_bf16x2(Af[4] * inv, Af[5] * inv);
-    out.w = pack_bf16x2(Af[6] * inv, Af[7] * inv);
-    *reinterpret_cast<uint4*>(o + ((size_t)b * H + h) * D + 8 * c) = out;
+    store_o8<D>(prm, ((size_t)b * H + h) * D + 8 * c, Af, inv);
     if (c == 0 && prm.lse != nullptr)
       prm.lse[(size_t)b * H + h] = Ls > 0.f ? (Mx + __log2f(Ls)) * 0.69314718055994531f : -INFINITY;
   }

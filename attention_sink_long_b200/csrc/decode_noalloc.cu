@@ -5,19 +5,23 @@
 // allocations, a latency-critical decode loop where cudaMalloc / cudaFree
 // would synchronise the device and stall every other stream, or a thin C / FFI
 // caller with no device allocator of its own. This entry point runs the same
-// decode kernel as lg_sparse_decode, but keeps the split partials and tickets
-// in a fixed array compiled into the library, so the caller passes only its
-// inputs and outputs. The paper has no counterpart; this is a deployment
-// convenience.
+// validation, split rule and decode kernel as lg_sparse_decode (decode_call in
+// api.cu), but keeps the split partials and tickets in a fixed array compiled
+// into the library, so the caller passes only its inputs and outputs. The
+// paper has no counterpart; this is a deployment convenience.
 //
 // The array is LG_DECODE_NOALLOC_SCRATCH_BYTES (16 MiB) per device, held from
 // the moment the library is loaded on a device until the process exits. Its
 // name is a host-side stand-in in host code, not a device address, so the
-// device address is looked up with cudaGetSymbolAddress once per device (with
-// that device current) on the first call, and cached. Every call shares the
-// array and it keeps the last call's contents: the tickets are cleared on the
-// stream at every call, and calls that overlap on the GPU (other streams, other
-// host threads) race on it -- serialise them.
+// device address is looked up with cudaGetSymbolAddress (with the device
+// current) on the first call on a device and cached together with the
+// device's current context; a new context (after cudaDeviceReset) triggers a
+// fresh look-up. Every call shares the array and it keeps the last call's
+// contents: the tickets are cleared on the stream at every call, and calls
+// that overlap on the GPU (other streams, other host threads) race on it --
+// serialise them.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "lg_kernels.h"
@@ -28,31 +32,39 @@ namespace {
 
 constexpr int kMaxNoallocDevices = 64;
 
-size_t r256(size_t x) { return (x + 255) & ~size_t(255); }
-
-size_t scratch_need(int B, int H, int Hkv, int D, int ns) {
-  if (ns <= 1) return 0;
-  return r256((size_t)B * H * ns * D * 4) + r256((size_t)B * H * ns * 4) + r256((size_t)B * Hkv * 4);
+// The driver's cuCtxGetCurrent, reached through the runtime (nothing links libcuda).
+PFN_cuCtxGetCurrent_v4000 ctx_get_current() {
+  static std::once_flag once;
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+  });
+  return fn;
 }
 
-// Device address of the scratch array on the current device; resolved on the
-// first call per device, with that device current.
-unsigned char* scratch_address(lg_status_t* st) {
+// Device address of the scratch array on device dev, which is current.
+unsigned char* scratch_address(int dev, lg_status_t* st) {
   static std::mutex mu;
   static unsigned char* addr[kMaxNoallocDevices] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxNoallocDevices) {
-    *st = LG_ERR_CUDA;
-    return nullptr;
-  }
+  static CUcontext ctx_of[kMaxNoallocDevices] = {};
+  *st = LG_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxNoallocDevices) return nullptr;
+  PFN_cuCtxGetCurrent_v4000 get_ctx = ctx_get_current();
+  if (get_ctx == nullptr) return nullptr;
+  // cudaSetDevice makes the device's primary context current (and creates it if needed).
+  if (cudaSetDevice(dev) != cudaSuccess) return nullptr;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  if (addr[dev] == nullptr || ctx_of[dev] != ctx) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_noalloc_scratch) != cudaSuccess || p == nullptr) {
-      *st = LG_ERR_CUDA;
-      return nullptr;
-    }
+    if (cudaGetSymbolAddress(&p, g_decode_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
     addr[dev] = static_cast<unsigned char*>(p);
+    ctx_of[dev] = ctx;
   }
   *st = LG_OK;
   return addr[dev];
@@ -61,65 +73,29 @@ unsigned char* scratch_address(lg_status_t* st) {
 }  // namespace
 
 extern "C" lg_status_t lg_sparse_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
-                                                const int32_t* cache_lens, void* o, float* lse, int32_t B, int32_t H,
-                                                int32_t Hkv, int32_t D, int32_t Lmax, int32_t num_splits,
-                                                float scale, lg_stream_t stream) {
-  if (!q || !k_cache || !v_cache || !cache_lens || !o) return LG_ERR_INVALID_ARG;
-  if (B <= 0 || H <= 0 || Hkv <= 0 || D <= 0 || Lmax <= 0 || num_splits < 0) return LG_ERR_INVALID_ARG;
-  if (H % Hkv != 0) return LG_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || !isfinite(scale)) return LG_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return LG_ERR_UNSUPPORTED;
-  const int G = H / Hkv;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return LG_ERR_UNSUPPORTED;
-  if (B > 65535 || Hkv > 65535) return LG_ERR_UNSUPPORTED;
-  const auto mis16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
-  if (mis16(q) || mis16(k_cache) || mis16(v_cache) || mis16(o) || (reinterpret_cast<uintptr_t>(cache_lens) & 3u) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u))
-    return LG_ERR_UNSUPPORTED;
-
-  // Same split rule as lg_sparse_decode; in automatic mode the split count is
-  // lowered until the partials fit the fixed array, an explicit count that does
-  // not fit is rejected.
-  int32_t ns = 1;
-  lg_status_t st = lg_sparse_decode_splits(B, H, Hkv, D, Lmax, num_splits, &ns);
-  if (st != LG_OK) return st;
-  if (scratch_need(B, H, Hkv, D, ns) > (size_t)LG_DECODE_NOALLOC_SCRATCH_BYTES) {
-    if (num_splits > 0) return LG_ERR_WORKSPACE;
-    while (ns > 1 && scratch_need(B, H, Hkv, D, ns) > (size_t)LG_DECODE_NOALLOC_SCRATCH_BYTES) --ns;
-  }
-  int rps = (Lmax + ns - 1) / ns;
-  ns = (Lmax + rps - 1) / rps;
-
-  unsigned char* scratch = scratch_address(&st);
-  if (st != LG_OK) return st;
+                                                const int32_t* cache_lens, void* o, int32_t o_dtype, float* lse,
+                                                int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax,
+                                                int32_t num_splits, float scale, lg_stream_t stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  lg::DecodeParams prm;
-  prm.q = q;
-  prm.k_cache = k_cache;
-  prm.v_cache = v_cache;
-  prm.lens = cache_lens;
-  prm.o = o;
-  prm.lse = lse;
-  prm.part_o = nullptr;
-  prm.part_lse = nullptr;
-  prm.tickets = nullptr;
-  if (ns > 1) {
-    unsigned char* w = scratch;
-    prm.part_o = reinterpret_cast<float*>(w);
-    w += r256((size_t)B * H * ns * D * 4);
-    prm.part_lse = reinterpret_cast<float*>(w);
-    w += r256((size_t)B * H * ns * 4);
-    prm.tickets = reinterpret_cast<unsigned int*>(w);
-    // Tickets must start at zero; the array keeps whatever the last call left.
-    if (cudaMemsetAsync(prm.tickets, 0, (size_t)B * Hkv * 4, s) != cudaSuccess) return LG_ERR_CUDA;
+  // The scratch address belongs to the current device, so the stream and the
+  // query must be on it too: a kernel given another device's array would read
+  // and write memory that is not its own.
+  int dev = -1, sdev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LG_ERR_CUDA;
+  if (cudaStreamGetDevice(s, &sdev) != cudaSuccess) return LG_ERR_INVALID_ARG;
+  if (sdev != dev) return LG_ERR_INVALID_ARG;
+  if (q != nullptr) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, q) != cudaSuccess) return LG_ERR_INVALID_ARG;
+    if ((a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) || a.device != dev)
+      return LG_ERR_INVALID_ARG;
   }
-  prm.B = B;
-  prm.H = H;
-  prm.Hkv = Hkv;
-  prm.Lmax = Lmax;
-  prm.ns = ns;
-  prm.rows_per_split = rps;
-  prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.err = nullptr;  // the decode kernel has no device-side waits
-  return lg::launch_decode(D, G, prm, s) == cudaSuccess ? LG_OK : LG_ERR_CUDA;
+  lg_status_t st = LG_OK;
+  unsigned char* scratch = scratch_address(dev, &st);
+  if (st != LG_OK) return st;
+  // Same validation, split rule and launch as lg_sparse_decode. An automatic
+  // split count is lowered until the partials fit the array; an explicit one
+  // that does not fit returns LG_ERR_WORKSPACE before anything is launched.
+  return lg::decode_call(q, k_cache, v_cache, cache_lens, nullptr, 0, 0, o, o_dtype, lse, B, H, Hkv, D, Lmax,
+                         num_splits, scale, scratch, LG_DECODE_NOALLOC_SCRATCH_BYTES, true, s);
 }

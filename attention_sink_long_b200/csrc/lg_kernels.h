@@ -102,7 +102,8 @@ struct DecodeParams {
   const int32_t* block_table = nullptr;  // [B, max_blocks] page of each 64-row cache block, or nullptr (contiguous)
   int max_blocks = 0;
   long long num_pages = 0;  // pages in the pool (paged cache)
-  void* o;              // [B, H, D] bf16
+  void* o;              // [B, H, D] bf16, or fp32 when o_f32
+  int o_f32 = 0;        // 1: o is written as fp32 (the unrounded result)
   float* lse;           // [B, H] or nullptr
   float* part_o;        // [B, H, ns, D] fp32 (ns > 1)
   float* part_lse;      // [B, H, ns] (log2 units)
@@ -114,10 +115,21 @@ struct DecodeParams {
 
 cudaError_t launch_decode(int D, int G, const DecodeParams& prm, cudaStream_t stream);
 
+// Every decode entry point (api.cu): validation, the split rule, the scratch
+// layout (decode_scratch_bytes) and the launch. With shrink_to_fit and an
+// automatic split count, the count is lowered until the partials fit
+// workspace_bytes (the fixed scratch of lg_sparse_decode_noalloc).
+size_t decode_scratch_bytes(int B, int H, int Hkv, int D, int ns);
+lg_status_t decode_call(const void* q, const void* k_cache, const void* v_cache, const int32_t* cache_lens,
+                        const int32_t* block_table, int32_t max_blocks, int64_t num_pages, void* o, int32_t o_dtype,
+                        float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax, int32_t num_splits,
+                        float scale, void* workspace, size_t workspace_bytes, bool shrink_to_fit,
+                        cudaStream_t stream);
+
 cudaError_t launch_wait_selftest(long long limit, unsigned int* err, cudaStream_t stream);
 cudaError_t launch_exp2(const float* x, float* y, long long n, int method, cudaStream_t stream);
 
-cudaError_t launch_pattern_iterate(const lg_pattern_t& p, int seqlen, int tile_blocks, int transpose, int32_t* out,
+cudaError_t launch_pattern_iterate(const lg_pattern_t& p, int seqlen, int tile_blocks, int mode, int32_t* out,
                                    int cap, cudaStream_t stream);
 
 }  // namespace lg

@@ -51,10 +51,12 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
-    ap.add_argument("--workload", choices=["step32k", "fwd128k", "bwd128k", "decode", "handoff", "blocksparse128k", "varlen", "decode_paged",
-                                               "gqa32k", "fp8qk32k", "decode_gqa"],
+    ap.add_argument("--workload", choices=["step32k", "fwd128k", "bwd128k", "decode", "handoff", "blocksparse128k",
+                                           "varlen", "decode_paged", "gqa32k", "fp8qk32k", "decode_gqa", "d64_32k"],
                     default="step32k")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the 128K / 32-layer / head-dim-64 rows the default step32k run adds")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
     return ap.parse_args(argv)
@@ -71,15 +73,18 @@ def max_over_ranks(value: float, dist, device) -> float:
     return float(t.item())
 
 
-def pick_peak(peaks, clocks, bound):
-    """Roofline denominator: the measured burst figure, or the sustained one
-    when the power cap throttled the SM clock during the timed region."""
+SUSTAINED_REGION_S = 2.0  # a timed region this long runs at the power-capped sustained rate
+
+
+def pick_peak(peaks, region_s, bound):
+    """Roofline denominator: the measured burst figure for a kernel timed in a
+    short region (the cuBLAS burst it is compared with is timed the same way),
+    the sustained figure once the timed region lasts seconds."""
     if bound == "hbm":
         return peaks["hbm_gbs"], "copy bandwidth"
-    capped = bool(clocks) and "sw_power_cap" in clocks.get("reasons", [])
-    if capped:
-        return peaks["bf16_tflops_sustained"], "sustained (sw_power_cap active)"
-    return peaks["bf16_tflops"], "burst"
+    if region_s >= SUSTAINED_REGION_S:
+        return peaks["bf16_tflops_sustained"], f"sustained (timed region {region_s:.2f} s)"
+    return peaks["bf16_tflops"], f"burst (timed region {region_s:.2f} s)"
 
 
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "kernel_traffic.json")
@@ -155,6 +160,11 @@ def workload(name):
         return {"workload": "grouped-query 32K: fwd + training bwd sink+window {64,1,64,0}, H32 Hkv8 D128",
                 "prefill": {"B": 1, "S": 32768, "H": 32, "Hkv": 8, "D": D},
                 "fwd": [("sink+window", SINK_WINDOW)], "bwd": [("sink+window", SINK_WINDOW)], "decode": None}
+    if name == "d64_32k":
+        return {"workload": "head dim 64 sink+window 32K: fwd + training bwd {64,1,64,0}, B1 H32 D64",
+                "prefill": {"B": 1, "S": 32768, "H": 32, "Hkv": 32, "D": 64},
+                "fwd": [("sink+window d64", SINK_WINDOW)], "bwd": [("sink+window d64", SINK_WINDOW)],
+                "decode": None}
     if name == "bwd128k":
         return {"workload": "128K sink+window training backward {64,1,64,0}",
                 "prefill": {"B": 1, "S": 131072, "H": 32, "Hkv": 32, "D": D},
@@ -289,9 +299,6 @@ class CudaStep:
             for n, p in wl["fwd"]:
                 self.parts.append((f"fwd {n}", "fwd_fp8qk" if wl.get("fp8qk") else "fwd",
                                    4 * D * pairs_of(p, S) * B * H, None, 1))
-            if wl["bwd"] and not self._bwd_available(pf, wl["bwd"][0][1]):
-                wl = dict(wl, bwd=[], workload=wl["workload"] + " (backward not available in this build)")
-                self.wl = wl
             if wl["bwd"]:
                 self.dq, self.dk, self.dv = torch.empty_like(self.q), torch.empty_like(self.k), torch.empty_like(self.v)
                 self.bwd_ws = torch.empty(max(lg.lg_sparse_attn_bwd_workspace(wl["bwd"][0][1], B, S, H, Hkv, D), 1),
@@ -391,23 +398,6 @@ class CudaStep:
         L = pg["L"]
         nbytes = 2 * B * L * Hkv * D * 2 + 2 * B * H * D * 2
         self.parts.append(("decode paged sink+window", "decode", 4 * D * L * B * H, nbytes, 1))
-
-    def _bwd_available(self, pf, pattern):
-        """One tiny backward call: False when the library reports it unsupported."""
-        lg, torch = self.lg, self.torch
-        D = pf["D"]
-        t = torch.zeros(1, 128, 1, D, dtype=torch.bfloat16, device=self.dev)
-        lse = torch.zeros(1, 1, 128, dtype=torch.float32, device=self.dev)
-        ws = torch.empty(lg.lg_sparse_attn_bwd_workspace(pattern, 1, 128, 1, 1, D), dtype=torch.uint8,
-                         device=self.dev)
-        try:
-            lg.lg_sparse_attn_bwd(pattern, t, t, t, t, t, lse, torch.empty_like(t), torch.empty_like(t),
-                                  torch.empty_like(t), 0.1, ws)
-        except lg.LgError as e:
-            if e.status == 4:
-                return False
-            raise
-        return True
 
     def run(self, events=None):
         """Launch one step; if events is given, record one event after each part."""
@@ -621,21 +611,12 @@ def cuda_arm(args, rank, world, dist):
                      step_flops / (ms_per_step * 1e-3) / 1e12)
 
     peaks, peak_src = load_peaks()
-    tensor_peak, tensor_kind = pick_peak(peaks, clk, "tensor")
+    tensor_peak, tensor_kind = pick_peak(peaks, total_ms * 1e-3, "tensor")
     rows = {}
     dominant = None
     for i, (name, kind, flops, nbytes, nl) in enumerate(step.parts):
         ms = statistics.mean(per_part_ms[i])
-        r = {"ms": round(ms, 4), "useful_tflops": round(flops / (ms * 1e-3) / 1e12, 2)}
-        if kind.startswith("decode") or kind == "copy":
-            r["gbs"] = round(nbytes / (ms * 1e-3) / 1e9, 1)
-            r["frac_hbm"] = round(r["gbs"] / peaks["hbm_gbs"], 4)
-        elif kind == "fwd_fp8qk":
-            # half of the FLOPs (S) at the fp8 rate, twice bf16: the mixed peak is 4/3 of bf16's
-            r["frac_mixed_fp8_bf16_peak"] = round(r["useful_tflops"] / (tensor_peak * 4 / 3), 4)
-        else:
-            r["frac_bf16"] = round(r["useful_tflops"] / tensor_peak, 4)
-        rows[name] = r
+        rows[name] = part_row(kind, flops, nbytes, ms, peaks, tensor_peak)
         if dominant is None or ms * weights[i] > dominant[1]:
             dominant = (i, ms * weights[i])
     di = dominant[0]
@@ -654,6 +635,9 @@ def cuda_arm(args, rank, world, dist):
         roof["peak_source"] = f"{peak_src} bf16 dense, {tensor_kind}" + (
             "; x 4/3: S (half the FLOPs) on the fp8 path at twice the bf16 rate (nominal ratio)"
             if dkind == "fwd_fp8qk" else "")
+        # The same kernel against the other measured figure, for context.
+        other = peaks["bf16_tflops_sustained"] if pk == peaks["bf16_tflops"] else peaks["bf16_tflops"]
+        roof["frac_" + ("sustained" if pk == peaks["bf16_tflops"] else "burst")] = round(achieved / other, 4)
     roof["traffic"] = recorded_traffic(dname, args.workload)
     roof["kernel"] = dname
 
@@ -682,6 +666,12 @@ def cuda_arm(args, rank, world, dist):
             e2e["scope"] = "the sparse-layer decode call end to end (cache, query up; output, LSE down); the " \
                            "full-layer caches stay on the device"
 
+    # The metric's other configurations (128K forward and backward, the 32-layer
+    # decode step, head dim 64), each timed alone after the step: one GPU only.
+    others = None
+    if world == 1 and args.workload == "step32k" and not args.no_other_workloads:
+        others = other_workload_rows(device, steps=10, warmup=3)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, args.cpu_seconds)
@@ -707,8 +697,81 @@ def cuda_arm(args, rank, world, dist):
         "config": config, "roofline": roof, "rows": rows, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches, "clocks": clk,
     }
+    if others is not None:
+        line["rows_other_workloads"] = others
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def part_row(kind, flops, nbytes, ms, peaks, tensor_peak):
+    """Per-part figures: useful TFLOP/s (and GB/s for HBM-bound parts) with their roofline fractions."""
+    r = {"ms": round(ms, 4), "useful_tflops": round(flops / (ms * 1e-3) / 1e12, 2)}
+    if kind.startswith("decode") or kind == "copy":
+        r["gbs"] = round(nbytes / (ms * 1e-3) / 1e9, 1)
+        r["frac_hbm"] = round(r["gbs"] / peaks["hbm_gbs"], 4)
+    elif kind == "fwd_fp8qk":
+        # half of the FLOPs (S) at the fp8 rate, twice bf16: the mixed peak is 4/3 of bf16's
+        r["frac_mixed_fp8_bf16_peak"] = round(r["useful_tflops"] / (tensor_peak * 4 / 3), 4)
+    else:
+        r["frac_bf16"] = round(r["useful_tflops"] / tensor_peak, 4)
+        r["frac_bf16_sustained"] = round(r["useful_tflops"] / peaks["bf16_tflops_sustained"], 4)
+        if kind == "bwd":
+            # 10 D FLOP per pair counts the five GEMMs (S recomputed); 8 D leaves the recompute out.
+            r["useful_tflops_8d"] = round(0.8 * r["useful_tflops"], 2)
+            r["frac_bf16_8d"] = round(0.8 * r["useful_tflops"] / tensor_peak, 4)
+    return r
+
+
+# The other configurations of the metric, timed in the default run beside the
+# 32K step (each alone, CUDA events, after warm-up): the 128K block-sparse
+# forward, the 128K sink+window backward, the full-layer decode and the
+# 32-layer decode step it makes with the sparse layer, and the head-dim-64
+# sink+window forward + backward at 32K.
+OTHER_WORKLOADS = ["fwd128k", "bwd128k", "decode", "d64_32k"]
+
+
+def other_workload_rows(device, steps, warmup):
+    import torch
+
+    peaks, _ = load_peaks()
+    out = {}
+    for name in OTHER_WORKLOADS:
+        wl = workload(name)
+        step = CudaStep(wl, device)
+        for _ in range(warmup):
+            step.run()
+        torch.cuda.synchronize()
+        nparts = len(step.parts)
+        t0 = torch.cuda.Event(enable_timing=True)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nparts)] for _ in range(steps)]
+        t0.record(step.stream)
+        for k in range(steps):
+            step.run(evs[k])
+        torch.cuda.synchronize()
+        per = [[] for _ in range(nparts)]
+        for k in range(steps):
+            prev = t0 if k == 0 else evs[k - 1][-1]
+            for i in range(nparts):
+                per[i].append(prev.elapsed_time(evs[k][i]))
+                prev = evs[k][i]
+        region_s = t0.elapsed_time(evs[-1][-1]) * 1e-3
+        tensor_peak, kind_s = pick_peak(peaks, region_s, "tensor")
+        rows = {}
+        for i, (pname, kind, flops, nbytes, _) in enumerate(step.parts):
+            rows[pname] = part_row(kind, flops, nbytes, statistics.mean(per[i]), peaks, tensor_peak)
+        entry = {"workload": wl["workload"], "steps": steps, "tensor_peak": kind_s, "rows": rows}
+        if name == "decode":
+            w = step.step_weights()
+            ms = sum(wi * statistics.mean(per[i]) for i, wi in enumerate(w))
+            gb = sum(wi * p[3] for wi, p in zip(w, step.parts)) / 1e9
+            entry["step_32_layers"] = {"ms": round(ms, 3), "gbs": round(gb / (ms * 1e-3), 1),
+                                       "frac_hbm": round(gb / (ms * 1e-3) / peaks["hbm_gbs"], 4),
+                                       "composition": "21 sparse-layer + 11 full-layer calls, from per-call times"}
+        assert step.lg.lg_device_status(device.index or 0) == 0, f"a bounded device wait ran out in {name}"
+        out[name] = entry
+        del step
+        torch.cuda.empty_cache()
+    return out
 
 
 # ----------------------------------------------------------------------------
@@ -777,8 +840,16 @@ def oracle_sample(wl, budget_s, seed=11):
                     oracle.attention_rows(qh, kh, vh, rows, op, scale)
                     job_flops += 4 * D * pairs
                 else:
+                    # dQ rows of a query block (S, dP, dQ: 6 D per pair), then dK / dV
+                    # rows of a KV block (the dV and dK products: 4 D per pair), so the
+                    # backward is credited the same 10 D per pair as the GPU arm.
                     oracle.attention_backward_rows(qh, kh, vh, doh, rows, op, scale)
-                    job_flops += 6 * D * pairs  # S, dP and dQ for these rows
+                    job_flops += 6 * D * pairs
+                    kblk = int(rng.integers(0, nqb))
+                    krows = np.arange(kblk * 64, kblk * 64 + 64)
+                    kpairs = int(oracle.allowed(np.arange(S)[:, None], krows[None, :], op).sum())
+                    oracle.attention_backward_kv_rows(qh, kh, vh, doh, krows, op, scale)
+                    job_flops += 4 * D * kpairs
             elif kind == "handoff":
                 kc, vc, rws = oracle.reduced_cache(hk, hv, ho["S"], p)
                 job_flops += 2 * 2 * len(rws) * ho["D"] * 2  # bytes: K and V rows read and written (bf16)
@@ -792,7 +863,8 @@ def oracle_sample(wl, budget_s, seed=11):
         dt = time.perf_counter() - t_start
         flops += job_flops
         t_used += dt
-        what = {"decode": "(b,h) rows", "handoff": "one-head prompt compactions"}.get(kind, "query blocks of one head")
+        what = {"decode": "(b,h) rows", "handoff": "one-head prompt compactions",
+                "bwd": "query blocks (dQ) + KV blocks (dK, dV) of one head"}.get(kind, "query blocks of one head")
         desc.append(f"{name}: {n_done} {what}")
     return flops, t_used, "; ".join(desc)
 
@@ -819,7 +891,8 @@ def cpu_baseline(wl, budget_s):
     unit, sc = work_unit(wl)
     return {"value": round(flops / secs / sc, 6), "unit": unit, "cores": cpu_cores(), "kind": "oracle",
             "sample": f"fp64 numpy oracle, {secs:.1f} s: {desc}; useful FLOPs credited 4D/pair fwd, "
-                      f"6D/pair bwd dQ rows, 4D/row decode; decode-only and hand-off workloads credited their bf16 "
+                      f"10D/pair bwd (6D for the sampled dQ rows + 4D for the sampled dK/dV rows, as the GPU "
+                      f"arm's 10D), 4D/row decode; decode-only and hand-off workloads credited their bf16 "
                       f"bytes"}
 
 

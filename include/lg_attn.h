@@ -114,20 +114,34 @@ lg_status_t lg_pattern_expand_t(const lg_pattern_t* pattern, int32_t seqlen, int
 lg_status_t lg_pattern_pairs(const lg_pattern_t* pattern, int32_t seqlen, int64_t* pairs);
 
 /*
- * Runs, on the device, the block iterator the attention kernels use, and
- * records what it visits, so tests can compare it bit for bit with the CSR.
- * Tiles are tile_blocks (1 or 2) consecutive 64-token blocks. With
- * transpose == 0 a tile is a range of query blocks and the iterator yields
- * KV blocks (forward); with transpose == 1 it is a range of KV blocks and
- * yields query blocks (backward). For tile u, out[u * (cap + 1)] receives the
- * count n and out[u * (cap + 1) + 1 + e] the e-th visited block as
- * (block << 2) | membership, where bit t of membership says whether the
- * visited block is in the list of the tile's t-th block. Device pointer
- * out holds ceil(nqb / tile_blocks) * (cap + 1) int32; entries beyond cap are
- * not written (the count still is).
+ * Runs, on the device, the block iterators the attention kernels use, and
+ * records what they visit, so tests can compare them bit for bit with the
+ * CSR / CSC lists (static, block-wise access: atlas.scime.ai summary,
+ * "Approach"). One record per tile u at out[u * (cap + 1)]: the entry count
+ * n, then the entries (entries beyond cap are not written; the count still
+ * is). A block entry is (block << 8) | membership, bit t of the membership
+ * saying whether the entry is in the list of the tile's t-th block. Modes:
+ *   0  forward union: tiles of tile_blocks (1, 2, 4, 8) query blocks; the
+ *      KV blocks of the union of their lists, ascending (n < 0 flags an
+ *      iterator whose closed-form count disagrees with its walk);
+ *   1  backward union: tiles of tile_blocks (1, 2) KV blocks; the query
+ *      blocks of the union of their transposed lists, ascending;
+ *   2  the forward kernels' chunked walk of a query span of tile_blocks
+ *      (4 or 8) blocks: two entries per chunk of two consecutive listed KV
+ *      blocks, the second -1 when the chunk holds one block;
+ *   3  the backward kernels' KV tiles (tile_blocks == 2): tile u of the
+ *      pairing of KV blocks (sink / strided blocks with each other, then the
+ *      window blocks in order) records its blocks kx, ky (-1 for none), the
+ *      first and last query block it walks, then one entry per query block
+ *      in that range, bit 0 / bit 1 for kx / ky.
+ * Device pointer out holds (number of tiles) * (cap + 1) int32 (mode 3:
+ * ceil(nqb / 2) tiles). Errors: LG_ERR_INVALID_ARG (bad pattern or mode,
+ * NULL out, seqlen not a positive multiple of block_size, cap < 0),
+ * LG_ERR_UNSUPPORTED (block_size != 64, tile_blocks not listed for the
+ * mode, 2^23 or more blocks), LG_ERR_CUDA (launch).
  */
 lg_status_t lg_pattern_iterate_device(const lg_pattern_t* pattern, int32_t seqlen, int32_t tile_blocks,
-                                      int32_t transpose, int32_t* out, int32_t cap, lg_stream_t stream);
+                                      int32_t mode, int32_t* out, int32_t cap, lg_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Prefill forward                                                          */
@@ -345,7 +359,9 @@ lg_status_t lg_sparse_decode_workspace(int32_t B, int32_t H, int32_t Hkv, int32_
  * Device pointers: q [B,H,D] bf16; k_cache, v_cache [B,Lmax,Hkv,D] bf16;
  * cache_lens [B] int32 with 1 <= cache_lens[b] <= Lmax (values are read on
  * the device and clamped to [0, Lmax]; a zero length yields o = 0,
- * lse = -inf); o [B,H,D] bf16 (written); lse [B,H] fp32 (written, may be NULL).
+ * lse = -inf); o [B,H,D] (written) of element type o_dtype: LG_BF16 (round
+ * to nearest even) or LG_F32 (the merged fp32 result before that rounding);
+ * lse [B,H] fp32 (written, may be NULL).
  * The KV range of each (b, kv head) is cut into num_splits pieces (0 = auto,
  * see lg_sparse_decode_splits); partial results are merged by
  * log-sum-exp in the same launch by the last CTA to finish each (b, kv head).
@@ -353,8 +369,8 @@ lg_status_t lg_sparse_decode_workspace(int32_t B, int32_t H, int32_t Hkv, int32_
  * ticket region is cleared on the stream by every call.
  */
 lg_status_t lg_sparse_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* cache_lens,
-                             void* o, float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t Lmax,
-                             int32_t num_splits, float scale, void* workspace, size_t workspace_bytes,
+                             void* o, int32_t o_dtype, float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D,
+                             int32_t Lmax, int32_t num_splits, float scale, void* workspace, size_t workspace_bytes,
                              lg_stream_t stream);
 
 /*
@@ -369,8 +385,9 @@ lg_status_t lg_sparse_decode(const void* q, const void* k_cache, const void* v_c
  */
 lg_status_t lg_sparse_decode_paged(const void* q, const void* k_pool, const void* v_pool, int64_t num_pages,
                                    const int32_t* block_table, int32_t max_blocks, const int32_t* cache_lens, void* o,
-                                   float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D, int32_t num_splits,
-                                   float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream);
+                                   int32_t o_dtype, float* lse, int32_t B, int32_t H, int32_t Hkv, int32_t D,
+                                   int32_t num_splits, float scale, void* workspace, size_t workspace_bytes,
+                                   lg_stream_t stream);
 
 /*
  * Size of the fixed device scratch array behind lg_sparse_decode_noalloc:
@@ -387,11 +404,16 @@ lg_status_t lg_sparse_decode_paged(const void* q, const void* k_pool, const void
  * the device and stall every other stream, and a thin C / FFI caller with no
  * device allocator of its own. Arguments and results are those of
  * lg_sparse_decode minus the workspace; the caller still passes all inputs
- * and outputs. Nothing is allocated or freed.
+ * and outputs (o of element type o_dtype, as lg_sparse_decode). Nothing is
+ * allocated or freed.
  * The split partials and tickets live in one file-scope device array of
  * LG_DECODE_NOALLOC_SCRATCH_BYTES. The first call on a device looks up the
- * array's device address (cudaGetSymbolAddress, with that device current);
- * make that first call before any stream capture. With num_splits == 0 the
+ * array's device address (cudaGetSymbolAddress, with that device current)
+ * and caches it with the device's current context; a call that finds a new
+ * context there (after cudaDeviceReset) looks it up again. Make the first
+ * call on a device before any stream capture. The current device must be the
+ * one the stream and q belong to (LG_ERR_INVALID_ARG otherwise: the array of
+ * one device is not the scratch of another). With num_splits == 0 the
  * automatic split count is lowered until the partials fit the array; an
  * explicit num_splits whose partials need more than the array holds
  * (B * H * num_splits * (D + 1) * 4 bytes, roughly) returns LG_ERR_WORKSPACE
@@ -400,9 +422,9 @@ lg_status_t lg_sparse_decode_paged(const void* q, const void* k_pool, const void
  * streams, other host threads) race on it, so serialise them.
  */
 lg_status_t lg_sparse_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
-                                     const int32_t* cache_lens, void* o, float* lse, int32_t B, int32_t H,
-                                     int32_t Hkv, int32_t D, int32_t Lmax, int32_t num_splits, float scale,
-                                     lg_stream_t stream);
+                                     const int32_t* cache_lens, void* o, int32_t o_dtype, float* lse, int32_t B,
+                                     int32_t H, int32_t Hkv, int32_t D, int32_t Lmax, int32_t num_splits,
+                                     float scale, lg_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Numerics                                                                 */

@@ -27,15 +27,6 @@ def report(name, got, ref):
     }
 
 
-def bf16_round(x):
-    """x rounded to the nearest bf16 (via fp32), as float64: the reference for an
-    output the library writes only in bf16, where the bound applies before the
-    output rounding."""
-    import torch
-
-    return torch.from_numpy(np.asarray(x, dtype=np.float64)).float().to(torch.bfloat16).double().numpy()
-
-
 def assert_close(name, got, ref, max_tol=MAX_TOL, mean_tol=MEAN_TOL):
     r = report(name, got, ref)
     assert r["nonfinite"] == 0, r

@@ -136,11 +136,18 @@ def test_bwd_and_decode_argument_errors():
     assert bwd([None] + P[1:]) == 1
     assert bwd(P, gdt=2) == 1                           # gradient dtype
     assert bwd(P, odt=5) == 1                           # O dtype
-    args = [0x10000, 0x20000, 0x30000, 0x40000, 0x50000, 0x60000]
-    assert L.lg_sparse_decode(*args, 32, 32, 32, 96, 4160, 0, 0.1, None, 0, None) == 2   # D
-    assert L.lg_sparse_decode(*args, 32, 24, 8, 128, 4160, 0, 0.1, None, 0, None) == 2   # G = 3
-    assert L.lg_sparse_decode(*args, 32, 32, 32, 128, 4160, 0, 0.1, None, 0, None) == 3  # workspace needed
-    assert L.lg_sparse_decode(*args, 32, 32, 32, 128, 0, 0, 0.1, None, 0, None) == 1
+    args = [0x10000, 0x20000, 0x30000, 0x40000, 0x50000]  # q, k_cache, v_cache, cache_lens, o
+
+    def dec(B=32, H=32, Hkv=32, D=128, L=4160, odt=0, lse=0x60000):
+        return L_.lg_sparse_decode(*args, odt, lse, B, H, Hkv, D, L, 0, 0.1, None, 0, None)
+
+    L_ = L
+    assert dec(D=96) == 2                 # D
+    assert dec(H=24, Hkv=8) == 2          # G = 3
+    assert dec() == 3                     # workspace needed
+    assert dec(L=0) == 1
+    assert dec(odt=2) == 1                # o dtype
+    assert dec(lse=0x60002) == 2          # misaligned lse
 
 
 def test_workspace_queries():
@@ -266,9 +273,9 @@ def test_paged_cache_argument_errors():
     assert append(MB=(1 << 24) + 1) == 2
 
     def decode(q=0x10000, kp=0x30000, tbl=0x50000, lens=0x70000, B=2, H=8, Hkv=8, D=128, P=256, MB=65, ns=1,
-               scale=0.088, ws=None, wsb=0):
-        return L.lg_sparse_decode_paged(q, kp, 0x40000, P, tbl, MB, lens, 0x90000, None, B, H, Hkv, D, ns, scale, ws,
-                                        wsb, None)
+               scale=0.088, ws=None, wsb=0, odt=0):
+        return L.lg_sparse_decode_paged(q, kp, 0x40000, P, tbl, MB, lens, 0x90000, odt, None, B, H, Hkv, D, ns, scale,
+                                        ws, wsb, None)
 
     assert decode(q=None) == 1
     assert decode(lens=None) == 1
@@ -280,6 +287,7 @@ def test_paged_cache_argument_errors():
     assert decode(kp=0x30008) == 2
     assert decode(MB=(1 << 24) + 1) == 2
     assert decode(ns=4) == 3            # four splits need a workspace
+    assert decode(odt=3) == 1           # o dtype
 
 
 def test_bwd_varlen_argument_errors():

@@ -43,10 +43,14 @@ def test_max_over_ranks_two_gloo_ranks():
 
 def test_peak_choice():
     peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1650.0, "bf16_tflops_sustained": 1400.0}
-    assert bench.pick_peak(peaks, {"reasons": []}, "tensor") == (1650.0, "burst")
-    assert bench.pick_peak(peaks, {"reasons": ["sw_power_cap"]}, "tensor")[0] == 1400.0
-    assert bench.pick_peak(peaks, None, "tensor")[0] == 1650.0
-    assert bench.pick_peak(peaks, {"reasons": ["sw_power_cap"]}, "hbm")[0] == 6500.0
+    # A kernel timed in a sub-second region is compared with the burst figure (timed the same
+    # way), one timed over seconds with the power-capped sustained figure.
+    assert bench.pick_peak(peaks, 0.7, "tensor")[0] == 1650.0
+    assert bench.pick_peak(peaks, 0.7, "tensor")[1].startswith("burst")
+    assert bench.pick_peak(peaks, 1.99, "tensor")[0] == 1650.0
+    assert bench.pick_peak(peaks, 2.0, "tensor")[0] == 1400.0
+    assert bench.pick_peak(peaks, 30.0, "tensor")[1].startswith("sustained")
+    assert bench.pick_peak(peaks, 30.0, "hbm")[0] == 6500.0
 
 
 def test_recorded_traffic_is_tied_to_kernel_sources(tmp_path, monkeypatch):

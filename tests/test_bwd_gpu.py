@@ -90,6 +90,48 @@ def test_bwd_matches_oracle_small(B, S, H, Hkv, D, pat, odt):
     assert_bf16_rounding_of("dV", bv, dv)
 
 
+GQA_TRAINING = [
+    # B, S, H, Hkv, D, pattern -- query-head groups with the forward's bf16 O (the training format)
+    (2, 384, 4, 2, 128, lg.Pattern(64, 0, 2, 3)),
+    (1, 640, 4, 1, 128, lg.Pattern(64, 2, 3, 0)),
+    (1, 512, 8, 1, 128, lg.Pattern(64, 1, 2, 0)),
+    (1, 1024, 4, 1, 64, lg.Pattern(64, 1, 4, 0)),
+    (2, 512, 4, 2, 64, lg.Pattern(64, 1, 2, 4)),
+]
+
+
+@pytest.mark.parametrize("B,S,H,Hkv,D,pat", GQA_TRAINING)
+def test_bwd_gqa_training_format_small(B, S, H, Hkv, D, pat):
+    """Query-head groups with the bf16 O the forward writes for training,
+    compared in full. The backward forms Delta = rowsum(dO * O) from the O it
+    is handed, so the reference is the oracle's gradient with Delta taken from
+    that same bf16 O: the comparison then measures the kernel, not the bf16
+    rounding of its O input (which alone moves dK by up to ~1e-2 on these
+    shapes)."""
+    q, k, v, do = si.prefill_inputs(B, S, H, Hkv, D, with_dout=True)
+    scale = 1.0 / math.sqrt(D)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, H, S, dtype=torch.float32, device="cuda")
+    lg.lg_sparse_attn_fwd(pat, qd, kd, vd, o, lse, scale)
+    ws = torch.empty(lg.lg_sparse_attn_bwd_workspace(pat, B, S, H, Hkv, D), dtype=torch.uint8, device="cuda")
+    grads = {}
+    for dt in (torch.float32, torch.bfloat16):
+        g = tuple(torch.empty(t.shape, dtype=dt, device="cuda") for t in (qd, kd, vd))
+        ws.fill_(0xFF)
+        lg.lg_sparse_attn_bwd(pat, qd, kd, vd, o, dod, lse, *g, scale, ws)
+        grads[dt] = g
+    torch.cuda.synchronize()
+    assert lg.lg_device_status(0) == 0
+    rdq, rdk, rdv, _ = oracle.attention_backward(q, k, v, do, oracle.Pattern(*pat), scale, o=o.cpu())
+    dq, dk, dv = grads[torch.float32]
+    assert_close("dQ", dq.cpu().numpy(), rdq)
+    assert_close("dK", dk.cpu().numpy(), rdk)
+    assert_close("dV", dv.cpu().numpy(), rdv)
+    for name, b16, f32 in zip(("dQ", "dK", "dV"), grads[torch.bfloat16], grads[torch.float32]):
+        assert_bf16_rounding_of(name, b16, f32)
+
+
 @pytest.mark.parametrize("pat", [lg.Pattern(64, 1, 64, 0), lg.Pattern(64, 1, 16, 32)],
                          ids=["sink_window", "block_sparse"])
 def test_bwd_128k_sampled(pat):
