@@ -26,7 +26,7 @@ __all__ = [
     "LgError", "Pattern", "lib", "lg_strerror", "lg_version",
     "lg_pattern_expand", "lg_pattern_expand_t", "lg_pattern_pairs", "lg_pattern_iterate_device",
     "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd", "lg_sparse_attn_fwd_varlen", "lg_sparse_attn_fwd_fp8qk",
-    "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd", "lg_sparse_attn_bwd_varlen",
+    "lg_sparse_attn_fwd_pair", "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd", "lg_sparse_attn_bwd_varlen",
     "lg_sparse_decode_splits", "lg_sparse_decode_workspace", "lg_sparse_decode",
     "lg_sparse_decode_noalloc", "lg_kv_compact_rows", "lg_kv_compact", "lg_kv_compact_paged", "lg_kv_append_paged",
     "lg_sparse_decode_paged", "lg_exp2_device", "lg_wait_selftest", "lg_device_status", "EXPORTED_SYMBOLS",
@@ -35,7 +35,7 @@ __all__ = [
 EXPORTED_SYMBOLS = (
     "lg_strerror", "lg_version", "lg_pattern_expand", "lg_pattern_expand_t", "lg_pattern_pairs",
     "lg_pattern_iterate_device", "lg_sparse_attn_fwd_workspace", "lg_sparse_attn_fwd", "lg_sparse_attn_fwd_varlen",
-    "lg_sparse_attn_fwd_fp8qk",
+    "lg_sparse_attn_fwd_fp8qk", "lg_sparse_attn_fwd_pair",
     "lg_sparse_attn_bwd_workspace", "lg_sparse_attn_bwd", "lg_sparse_attn_bwd_varlen", "lg_sparse_decode_splits",
     "lg_sparse_decode_workspace", "lg_sparse_decode", "lg_sparse_decode_noalloc", "lg_kv_compact_rows",
     "lg_kv_compact", "lg_kv_compact_paged", "lg_kv_append_paged", "lg_sparse_decode_paged", "lg_exp2_device",
@@ -83,6 +83,8 @@ _SIGS = {
                                   + [_c_i32] * 6 + [_c_f, _c_vp]),
     "lg_sparse_attn_fwd_fp8qk": (_c_i32, [_P(_lg_pattern_t), _c_vp, _c_vp, _c_vp, _c_f, _c_f, _c_vp, _c_i32, _c_vp]
                                  + [_c_i32] * 5 + [_c_f, _c_vp]),
+    "lg_sparse_attn_fwd_pair": (_c_i32, [_P(_lg_pattern_t), _c_vp, _c_vp, _c_vp, _c_vp, _c_i32, _c_vp] + [_c_i32] * 5
+                                + [_c_f, _c_vp]),
     "lg_sparse_attn_bwd_workspace": (_c_i32, [_P(_lg_pattern_t)] + [_c_i32] * 5 + [_P(_c_sz)]),
     "lg_sparse_attn_bwd": (_c_i32, [_P(_lg_pattern_t)] + [_c_vp] * 4 + [_c_i32] + [_c_vp] * 5 + [_c_i32] * 6
                            + [_c_f, _c_vp, _c_sz, _c_vp]),
@@ -253,6 +255,25 @@ def lg_sparse_attn_fwd(pattern, q, k, v, o, lse, scale: float, workspace=None, s
     _check(lib().lg_sparse_attn_fwd(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), odt,
                                     _ptr(lse), B, S, H, Hkv, D, float(scale), _ptr(workspace), ws, _stream(stream)),
            "lg_sparse_attn_fwd")
+
+
+def lg_sparse_attn_fwd_pair(pattern, q, k, v, o, lse, scale: float, stream=None):
+    """lg_sparse_attn_fwd computed by CTA pairs sharing 256-row MMAs (head dim 128):
+    q [B,S,H,128], k/v [B,S,Hkv,128] bf16; o bf16 or fp32 (written); lse [B,H,S] fp32 or None."""
+    import torch
+
+    B, S, H, D = q.shape
+    Hkv = k.shape[2]
+    _expect(q, "q", torch.bfloat16, (B, S, H, D))
+    _expect(k, "k", torch.bfloat16, (B, S, Hkv, D), q.device)
+    _expect(v, "v", torch.bfloat16, (B, S, Hkv, D), q.device)
+    odt = _dtype_code(o, "o")
+    _expect(o, "o", o.dtype, (B, S, H, D), q.device)
+    if lse is not None:
+        _expect(lse, "lse", torch.float32, (B, H, S), q.device)
+    _check(lib().lg_sparse_attn_fwd_pair(ctypes.byref(_pat(pattern)), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                         o.data_ptr(), odt, _ptr(lse), B, S, H, Hkv, D, float(scale),
+                                         _stream(stream)), "lg_sparse_attn_fwd_pair")
 
 
 def lg_sparse_attn_fwd_varlen(pattern, q, k, v, o, lse, cu_seqlens, max_seqlen: int, scale: float, stream=None):

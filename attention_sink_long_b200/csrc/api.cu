@@ -288,6 +288,39 @@ lg_status_t lg_sparse_attn_fwd(const lg_pattern_t* p, const void* q, const void*
   return cuda_status(lg::launch_fwd(D, tq, tk, tv, to, prm, B, static_cast<cudaStream_t>(stream)));
 }
 
+lg_status_t lg_sparse_attn_fwd_pair(const lg_pattern_t* p, const void* q, const void* k, const void* v, void* o,
+                                    int32_t o_dtype, float* lse, int32_t B, int32_t S, int32_t H, int32_t Hkv,
+                                    int32_t D, float scale, lg_stream_t stream) {
+  lg_status_t st = check_prefill_shape(p, B, S, H, Hkv, D);
+  if (st != LG_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return LG_ERR_INVALID_ARG;
+  if (o_dtype != LG_BF16 && o_dtype != LG_F32) return LG_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return LG_ERR_INVALID_ARG;
+  if (D != 128) return LG_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return LG_ERR_UNSUPPORTED;
+  unsigned int* err = error_word(&st);
+  if (st != LG_OK) return st;
+  CUtensorMap tq, tk, tv, to;
+  if ((st = make_map(&tq, q, B, S, H, D, 128)) != LG_OK) return st;
+  if ((st = make_map(&tk, k, B, S, Hkv, D, 64)) != LG_OK) return st;
+  if ((st = make_map(&tv, v, B, S, Hkv, D, 64)) != LG_OK) return st;
+  if ((st = make_map(&to, o_dtype == LG_F32 ? q : o, B, S, H, D, 64)) != LG_OK) return st;
+  lg::FwdParams prm;
+  prm.pat = *p;
+  prm.lse = lse;
+  prm.o_f32 = o_dtype == LG_F32 ? static_cast<float*>(o) : nullptr;
+  prm.S = S;
+  prm.H = H;
+  prm.Hkv = Hkv;
+  prm.nqb = S / 64;
+  prm.nqt = (S + 511) / 512;  // 512-row spans, one per CTA pair
+  prm.cu_seqlens = nullptr;
+  prm.max_len = S;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.err = err;
+  return cuda_status(lg::launch_fwd2(tq, tk, tv, to, prm, B, static_cast<cudaStream_t>(stream)));
+}
+
 lg_status_t lg_sparse_attn_fwd_fp8qk(const lg_pattern_t* p, const void* q8, const void* k8, const void* v,
                                      float q_descale, float k_descale, void* o, int32_t o_dtype, float* lse, int32_t B,
                                      int32_t S, int32_t H, int32_t Hkv, int32_t D, float scale, lg_stream_t stream) {

@@ -24,6 +24,9 @@ struct FwdParams {
 
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const FwdParams& prm, int B, cudaStream_t stream);
+// Head dim 128, bf16: the CTA-pair kernel (cta_group::2 MMAs over 512-row query spans).
+cudaError_t launch_fwd2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const CUtensorMap& to, const FwdParams& prm, int B, cudaStream_t stream);
 // Head dim 128, Q and K in fp8 e4m3 (tensor maps over bytes, one 128-byte panel per row).
 cudaError_t launch_fwd_fp8qk(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& to, const FwdParams& prm, int B, cudaStream_t stream);

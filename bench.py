@@ -52,7 +52,8 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--workload", choices=["step32k", "fwd128k", "bwd128k", "decode", "handoff", "blocksparse128k",
-                                           "varlen", "decode_paged", "gqa32k", "fp8qk32k", "decode_gqa", "d64_32k"],
+                                           "varlen", "decode_paged", "gqa32k", "fp8qk32k", "decode_gqa", "d64_32k",
+                                           "pair32k"],
                     default="step32k")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end loop")
     ap.add_argument("--no-other-workloads", action="store_true",
@@ -160,6 +161,13 @@ def workload(name):
         return {"workload": "grouped-query 32K: fwd + training bwd sink+window {64,1,64,0}, H32 Hkv8 D128",
                 "prefill": {"B": 1, "S": 32768, "H": 32, "Hkv": 8, "D": D},
                 "fwd": [("sink+window", SINK_WINDOW)], "bwd": [("sink+window", SINK_WINDOW)], "decode": None}
+    if name == "pair32k":
+        # The CTA-pair forward (lg_sparse_attn_fwd_pair: 256-row cta_group::2 MMAs) beside the default one.
+        return {"workload": "CTA-pair forward vs the default forward, 32K dense and sink+window, B1 H32 D128",
+                "prefill": {"B": 1, "S": 32768, "H": 32, "Hkv": 32, "D": D},
+                "fwd": [("dense pair", FULL), ("dense", FULL), ("sink+window pair", SINK_WINDOW),
+                        ("sink+window", SINK_WINDOW)], "bwd": [], "decode": None, "pair_parts": ["dense pair",
+                                                                                                 "sink+window pair"]}
     if name == "d64_32k":
         return {"workload": "head dim 64 sink+window 32K: fwd + training bwd {64,1,64,0}, B1 H32 D64",
                 "prefill": {"B": 1, "S": 32768, "H": 32, "Hkv": 32, "D": 64},
@@ -407,6 +415,8 @@ class CudaStep:
             if wl.get("fp8qk"):
                 lg.lg_sparse_attn_fwd_fp8qk(p, self.q8, self.k8, self.v, 0.25, 0.5, self.o[n], self.lse[n],
                                             self.scale)
+            elif n in wl.get("pair_parts", ()):
+                lg.lg_sparse_attn_fwd_pair(p, self.q, self.k, self.v, self.o[n], self.lse[n], self.scale)
             else:
                 lg.lg_sparse_attn_fwd(p, self.q, self.k, self.v, self.o[n], self.lse[n], self.scale)
             if events is not None:
@@ -725,9 +735,10 @@ def part_row(kind, flops, nbytes, ms, peaks, tensor_peak):
 # The other configurations of the metric, timed in the default run beside the
 # 32K step (each alone, CUDA events, after warm-up): the 128K block-sparse
 # forward, the 128K sink+window backward, the full-layer decode and the
-# 32-layer decode step it makes with the sparse layer, and the head-dim-64
-# sink+window forward + backward at 32K.
-OTHER_WORKLOADS = ["fwd128k", "bwd128k", "decode", "d64_32k"]
+# 32-layer decode step it makes with the sparse layer, the head-dim-64
+# sink+window forward + backward at 32K, and the CTA-pair forward beside the
+# default one.
+OTHER_WORKLOADS = ["fwd128k", "bwd128k", "decode", "d64_32k", "pair32k"]
 
 
 def other_workload_rows(device, steps, warmup):

@@ -165,6 +165,23 @@ lg_status_t lg_sparse_attn_fwd(const lg_pattern_t* pattern, const void* q, const
                                int32_t D, float scale, void* workspace, size_t workspace_bytes, lg_stream_t stream);
 
 /*
+ * The forward above (head dim 128) computed by pairs of CTAs that share
+ * 256-row tcgen05 MMAs (cta_group::2; no TMA multicast): each pair owns a
+ * 512-row query span of one head, each CTA loads half of every K/V chunk,
+ * and P goes through shared memory so the next chunk's S = Q K^T runs while
+ * the softmax of this one is still exponentiating. Same arithmetic and
+ * results as lg_sparse_attn_fwd (bit-equal on the dense pattern; within one
+ * bf16 ulp of O and 2e-6 of LSE where the wider span changes which
+ * partially-masked chunks a row meets). A throughput variant: on the
+ * workloads measured it runs at 0.9-1.0x of lg_sparse_attn_fwd's speed.
+ * Arguments, layouts and errors as lg_sparse_attn_fwd (no workspace);
+ * LG_ERR_UNSUPPORTED for D != 128.
+ */
+lg_status_t lg_sparse_attn_fwd_pair(const lg_pattern_t* pattern, const void* q, const void* k, const void* v,
+                                    void* o, int32_t o_dtype, float* lse, int32_t B, int32_t S, int32_t H,
+                                    int32_t Hkv, int32_t D, float scale, lg_stream_t stream);
+
+/*
  * The forward above with Q and K in fp8 e4m3 (one byte each, head dim 128):
  * S = (q8 k8^T) * q_descale * k_descale, computed on the fp8 tensor-core path
  * at twice the bf16 rate; the softmax, P V (bf16) and the outputs are those of

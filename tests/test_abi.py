@@ -334,3 +334,21 @@ def test_fwd_fp8qk_argument_errors():
     assert call(D=64) == 2            # fp8 Q/K: head dim 128 only
     assert call(S=1000) == 2
     assert call(q=0x10008) == 2
+
+
+def test_fwd_pair_argument_errors():
+    L = lg.lib()
+    p = lg._lg_pattern_t(64, 1, 64, 0)
+
+    def call(q=0x10000, B=1, S=1024, H=4, Hkv=4, D=128, odt=0, scale=0.088, lse=0x50000):
+        return L.lg_sparse_attn_fwd_pair(ctypes.byref(p), q, 0x20000, 0x30000, 0x40000, odt, lse, B, S, H, Hkv, D,
+                                         scale, None)
+
+    assert call(q=None) == 1
+    assert call(odt=5) == 1
+    assert call(scale=0.0) == 1
+    assert call(H=4, Hkv=3) == 1
+    assert call(D=64) == 2            # the pair kernel: head dim 128 only
+    assert call(S=1000) == 2
+    assert call(q=0x10008) == 2
+    assert call(lse=0x50004) == 2

@@ -1,7 +1,9 @@
 """Forward parity: the tcgen05 prefill kernel through the C-ABI vs the fp64 oracle.
 
 Small shapes are compared element by element (several 128-row tiles, a ragged
-64-row tail, GQA, every pattern term, D = 64 and 128). The full-size workloads
+64-row tail, GQA, every pattern term, D = 64 and 128). The CTA-pair forward
+(lg_sparse_attn_fwd_pair, head dim 128) runs the same cases, including
+512-row spans the sequence end cuts short, and two full-size workloads. The full-size workloads
 (32K sink+window and dense, 128K block-sparse) are compared on sampled query
 blocks of the first and last head, whose rows the oracle computes one by one.
 """
@@ -41,6 +43,12 @@ SMALL = [
     (1, 2048, 2, 2, 128, lg.Pattern(64, 1, 16, 4)),
     (1, 1280, 2, 2, 128, lg.Pattern(64, 0, 1, 0)),     # diagonal only: first block half-masked per tile
     (1, 1024, 2, 2, 128, lg.Pattern(64, 1, 2, 5)),
+    # For the CTA-pair forward (512-row spans): spans cut short by the sequence end (one block
+    # left: the odd CTA has no rows; 384 rows left: the odd CTA's second tile has none), and
+    # unions of odd length (a lone last block in the chunk walk).
+    (1, 576, 2, 2, 128, lg.Pattern(64, 1, 2, 0)),
+    (2, 896, 4, 4, 128, lg.Pattern(64, 0, 3, 0)),
+    (1, 1536, 4, 1, 128, lg.Pattern(64, 3, 2, 5)),
 ]
 
 
@@ -95,3 +103,56 @@ def test_fwd_full_size_sampled(name, S, pat):
         ro, rl = oracle.attention_rows(qh, kh, vh, rows, op, scale)
         assert_close(f"{name} O h{h}", o[0, rows, h].float().cpu().numpy(), ro)
         assert_lse(f"{name} LSE h{h}", lse[0, h, rows].cpu().numpy(), rl)
+
+
+def run_fwd_pair(pattern, q, k, v, scale, o_dtype=torch.bfloat16):
+    B, S, H, D = q.shape
+    o = torch.empty(q.shape, dtype=o_dtype, device=q.device)
+    lse = torch.empty(B, H, S, dtype=torch.float32, device=q.device)
+    lg.lg_sparse_attn_fwd_pair(pattern, q, k, v, o, lse, scale)
+    torch.cuda.synchronize()
+    assert lg.lg_device_status(q.device.index or 0) == 0
+    return o, lse
+
+
+@pytest.mark.parametrize("B,S,H,Hkv,D,pat", [c for c in SMALL if c[4] == 128])
+def test_fwd_pair_matches_oracle_small(B, S, H, Hkv, D, pat):
+    q, k, v = si.prefill_inputs(B, S, H, Hkv, D)
+    scale = 1.0 / math.sqrt(D)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o32, lse = run_fwd_pair(pat, qd, kd, vd, scale, torch.float32)
+    ro, rlse = oracle.attention_forward(q, k, v, oracle.Pattern(*pat), scale)
+    assert_close("O fp32", o32.cpu().numpy(), ro)
+    assert_lse("LSE", lse.cpu().numpy(), rlse)
+    o16, lse16 = run_fwd_pair(pat, qd, kd, vd, scale)
+    assert torch.equal(lse16, lse)
+    assert torch.equal(o32.to(torch.bfloat16), o16)
+    # the single-CTA forward computes the same rows: within one bf16 ulp (same arithmetic,
+    # chunks of a wider span may pair other blocks together)
+    o1, l1 = run_fwd(pat, qd, kd, vd, scale, torch.float32)
+    assert torch.allclose(o1, o32, rtol=2**-7, atol=1e-6)
+    assert float((l1 - lse).abs().max()) <= 1e-5
+
+
+def test_fwd_pair_rejects_head_dim_64():
+    q, k, v = si.prefill_inputs(1, 256, 2, 2, 64)
+    o = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(lg.LgError) as e:
+        lg.lg_sparse_attn_fwd_pair(lg.Pattern(64, 1, 2, 0), q.cuda(), k.cuda(), v.cuda(), o, None, 0.125)
+    assert e.value.status == 2
+
+
+@pytest.mark.parametrize("name,S,pat", [LARGE[1], LARGE[2]])
+def test_fwd_pair_full_size_sampled(name, S, pat):
+    B, H, D = 1, 32, 128
+    dev = torch.device("cuda")
+    q, k, v = si.prefill_inputs_device(B, S, H, H, D, dev)
+    scale = 1.0 / math.sqrt(D)
+    o, lse = run_fwd_pair(pat, q, k, v, scale)
+    rows = np.concatenate([np.arange(b * 64, (b + 1) * 64) for b in sampled_blocks(S // 64)])
+    op = oracle.Pattern(*pat)
+    for h in (0, H - 1):
+        qh, kh, vh = (t[0, :, h].float().cpu().numpy() for t in (q, k, v))
+        ro, rl = oracle.attention_rows(qh, kh, vh, rows, op, scale)
+        assert_close(f"{name} pair O h{h}", o[0, rows, h].float().cpu().numpy(), ro)
+        assert_lse(f"{name} pair LSE h{h}", lse[0, h, rows].cpu().numpy(), rl)
