@@ -127,10 +127,11 @@ def test_fwd_pair_matches_oracle_small(B, S, H, Hkv, D, pat):
     o16, lse16 = run_fwd_pair(pat, qd, kd, vd, scale)
     assert torch.equal(lse16, lse)
     assert torch.equal(o32.to(torch.bfloat16), o16)
-    # the single-CTA forward computes the same rows: within one bf16 ulp (same arithmetic,
-    # chunks of a wider span may pair other blocks together)
+    # The single-CTA forward computes the same rows. A 512-row span pairs other KV blocks into
+    # chunks than a 256-row span does, so the bf16 rounding of P and the lazy-rescale points
+    # differ: the two outputs agree to the parity bound, not bit for bit.
     o1, l1 = run_fwd(pat, qd, kd, vd, scale, torch.float32)
-    assert torch.allclose(o1, o32, rtol=2**-7, atol=1e-6)
+    assert_close("O pair vs single", o32.cpu().numpy(), o1.cpu().numpy())
     assert float((l1 - lse).abs().max()) <= 1e-5
 
 
