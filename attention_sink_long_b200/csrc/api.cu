@@ -436,10 +436,8 @@ static lg_status_t bwd_common(const lg_pattern_t* p, const void* q, const void* 
   float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) + round256((size_t)Bm * H * S * D * 4));
   float* lse2 = reinterpret_cast<float*>(reinterpret_cast<char*>(delta) + round256((size_t)Bm * H * S * 4));
 
-  // Head dim 128 runs the 128-row-step kernel, whose KV tiles are two
-  // separately placed 64-row blocks (BlockPairing); the head-dim-64 kernel's
-  // tiles are 128 consecutive rows, also moved as two 64-row boxes.
-  const bool paired = (D == 128);
+  // The 128-row-step kernel's KV tiles are two separately placed 64-row
+  // blocks (BlockPairing), each moved as its own 64-row box.
   CUtensorMap tq, tk, tv, tdo, tdk, tdv;
   if ((st = make_map(&tq, q, Bm, S, H, D, 64)) != LG_OK) return st;
   if ((st = make_map(&tk, k, Bm, S, Hkv, D, 64)) != LG_OK) return st;
@@ -474,15 +472,11 @@ static lg_status_t bwd_common(const lg_pattern_t* p, const void* q, const void* 
     std::vector<int> counts(prm.nkt);
     const lg::BlockPairing bp(*p, prm.nqb);
     for (int t = 0; t < prm.nkt; ++t) {
-      if (paired) {
-        int x, y;
-        bp.pair(t, &x, &y);
-        const int first = y >= 0 ? imin(x, y) : x;
-        const int last = y >= 0 ? imax(bp.reach(x), bp.reach(y)) : bp.reach(x);
-        counts[t] = last - first + 1;
-      } else {
-        counts[t] = lg::QIter(*p, 2 * t, imin(2 * t + 1, prm.nqb - 1), prm.nqb).count();
-      }
+      int x, y;
+      bp.pair(t, &x, &y);
+      const int first = y >= 0 ? imin(x, y) : x;
+      const int last = y >= 0 ? imax(bp.reach(x), bp.reach(y)) : bp.reach(x);
+      counts[t] = last - first + 1;
     }
     std::vector<int> sorted_counts(counts);
     std::nth_element(sorted_counts.begin(), sorted_counts.begin() + prm.nkt / 2, sorted_counts.end());

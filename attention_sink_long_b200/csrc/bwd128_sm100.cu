@@ -1,5 +1,5 @@
-// bwd128_sm100.cu -- LongGen sparse causal attention, training backward for
-// head dim 128, on sm_100a.
+// bwd128_sm100.cu -- LongGen sparse causal attention, training backward with
+// 128-row KV tiles and 128-row query steps, for head dims 64 and 128, on sm_100a.
 //
 // "A Little Goes a Long Way" (LongGen), Abstract insights 1-2 and the
 // atlas.scime.ai summary, "Approach": the sparse layers are trained, so the
@@ -16,16 +16,20 @@
 // the same query blocks -- and walks those query blocks two at a time: a
 // 128-row query step (with query-head groups, the steps of every query head
 // of the group in turn, dK and dV accumulating over all of them).
-// Every GEMM of a step is then an M = 128, N = 128 tcgen05 MMA -- the shape
-// the tensor core runs at full rate (an N = 64 instruction takes about as
-// long as an N = 128 one):
+// At head dim 128 every GEMM of a step is then an M = 128, N = 128 tcgen05
+// MMA -- the shape the tensor core runs at full rate (an N = 64 instruction
+// takes about as long as an N = 128 one):
 //   S^T  = K Q^T       SS, both K-major               -> TMEM region R_s
 //   dP^T = V dO^T      SS, both K-major               -> TMEM region R_d
 //   dV  += P^T dO      TS: P^T (bf16) from TMEM, dO MN-major
 //   dK  += dS^T Q      SS: dS^T (bf16) from shared memory, Q MN-major
 //   dQ^T = K^T dS^T    SS, both MN-major              -> R_d, drained with
 //                      coalesced fp32 reductions into the dQ accumulator.
-// TMEM columns: dV [0,128), dK [128,256), R_s [256,384), R_d [384,512).
+// TMEM columns: dV [0,D), dK [D,2D), R_s [2D,2D+128), R_d [2D+128,2D+256).
+// At head dim 64 S^T and dP^T keep M = N = 128 (K = 64), dV and dK run with
+// N = 64, and dQ^T keeps M = 128: its A operand's second 64-row half reads
+// whatever lies one panel further on and lands in TMEM lanes 64-127, which
+// nothing reads (an M = 64 instruction would take as long).
 // The P/dS warps read S^T and write P^T (bf16, two per column) over the first
 // half of the columns they read, so no warp overwrites columns another warp
 // still reads. R_d holds dP^T until the warps have read it, then dQ^T.
@@ -46,49 +50,57 @@
 // Warps: 0-7 P / dS + epilogue (two per TMEM lane quarter: KV rows
 // 32 (w % 4) .. +31, query columns [64 (w / 4), +64) of the step), 8 TMA
 // producer, 9 TMEM owner + MMA issuer, 10-13 dQ drain (one per lane quarter).
-// Shared memory: K, V, two Q / dO stages, dS^T -- seven 32 KB tiles (224 KB)
-// -- plus barriers and the LSE / Delta stages after them.
+// Shared memory: K, V, two Q / dO stages (128 x D bf16 each) and dS^T
+// (128 x 128 bf16) -- 224 KB at head dim 128, 128 KB at 64 -- plus barriers
+// and the LSE / Delta stages after them.
 #include "lg_common.cuh"
 #include "lg_kernels.h"
 #include "lg_pattern.cuh"
 
 namespace lg {
 
+template <int D_>
 struct Bwd128Layout {
-  static constexpr int D = 128;
+  static constexpr int D = D_;
+  static constexpr int DP = D / 64;             // 64-column (128-byte) panels per row
   static constexpr int QS = 2;                  // Q / dO / LSE / Delta stages
-  static constexpr int TILE = 128 * 128 * 2;    // a 128 x 128 bf16 tile, two 64-column panels
+  static constexpr int TILE = 128 * D * 2;      // a 128 x D bf16 tile (K, V, Q, dO)
   static constexpr int PANEL = 128 * 128;       // one 64-column panel of 128 rows (bytes)
+  static constexpr int DS_TILE = 128 * 128 * 2; // dS^T: 128 KV rows x 128 query columns, two panels
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
   static constexpr int OFF_Q = OFF_V + TILE;          // QS stages
   static constexpr int OFF_DO = OFF_Q + QS * TILE;    // QS stages
   static constexpr int OFF_DS = OFF_DO + QS * TILE;   // dS^T, rows = KV, columns = query
-  static constexpr int TILES = OFF_DS + TILE;         // 229376
+  static constexpr int TILES = OFF_DS + DS_TILE;      // 229376 at head dim 128
   static constexpr int NBAR = 1 + 4 * QS + 8;
   static constexpr int OFF_BAR = TILES;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_LSE = (OFF_MISC + 16 + 15) / 16 * 16;  // QS x 128 fp32
   static constexpr int OFF_DEL = OFF_LSE + QS * 512;   // QS x 128 fp32
   static constexpr int BYTES = OFF_DEL + QS * 512;
-  static constexpr int ALLOC = 232448;                 // the per-block maximum
+  // Head dim 128 needs nearly the whole per-block maximum; the smaller layout
+  // asks for its size plus the 1024-byte alignment slack.
+  static constexpr int ALLOC = D == 128 ? 232448 : BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t T_DV = 0, T_DK = 128, T_RS = 256, T_RD = 384;
+  static constexpr uint32_t T_DV = 0, T_DK = D, T_RS = 2 * D, T_RD = 2 * D + 128;
   static_assert(OFF_LSE % 16 == 0, "bulk copies need 16-byte aligned destinations");
+  static_assert(BYTES <= ALLOC && ALLOC <= 232448, "shared memory budget");
+  static_assert(T_RD + 128 <= TMEM_COLS, "TMEM budget");
 };
 
-template <bool GQA>
+template <int D, bool GQA>
 __global__ void __launch_bounds__(448, 1)
     lg_bwd128_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                      const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
                      const BwdParams prm) {
-  using L = Bwd128Layout;
+  using L = Bwd128Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // The tiles need a 1024-byte aligned base (128-byte swizzle) and the layout
-  // uses nearly the whole per-block allocation, so it only fits when the
-  // dynamic shared memory starts close enough to such a boundary. Checked
+  // The tiles need a 1024-byte aligned base (128-byte swizzle); at head dim
+  // 128 the layout uses nearly the whole per-block allocation, so it only fits
+  // when the dynamic shared memory starts close enough to such a boundary. Checked
   // uniformly before anything else; a misfit is reported, never run.
   if ((size_t)(smem - smem_raw) + (size_t)L::BYTES > (size_t)L::ALLOC) {
     if (threadIdx.x == 0) atomicOr(prm.err, kErrSmemFit);
@@ -211,7 +223,7 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(p_full, 256);
     mbar_init(ds_full, 256);
     mbar_init(dq_full, 1);
-    mbar_init(dq_free, 128);
+    mbar_init(dq_free, D);  // the drain threads of the D real dQ^T rows
     mbar_init(dss_free, 1);
     mbar_init(acc_done, 1);
     *abort_flag = 0;
@@ -231,7 +243,7 @@ __global__ void __launch_bounds__(448, 1)
     if (lane == 0) {
       mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
       for (int hb = 0; hb < 2; ++hb)
-        for (int p = 0; p < 2; ++p) {
+        for (int p = 0; p < L::DP; ++p) {
           tma_load_4d(smem + L::OFF_K + p * L::PANEL + hb * 8192, &tmK, kv_full, 64 * p, h, base + 64 * kload[hb], bc);
           tma_load_4d(smem + L::OFF_V + p * L::PANEL + hb * 8192, &tmV, kv_full, 64 * p, h, base + 64 * kload[hb], bc);
         }
@@ -249,7 +261,7 @@ __global__ void __launch_bounds__(448, 1)
         mbar_arrive_expect_tx(&qo_full[st], L::TILE + nl * 256);
         issued_o = m + 1;
         for (int hb = 0; hb < 2; ++hb)
-          for (int p = 0; p < 2; ++p)
+          for (int p = 0; p < L::DP; ++p)
             tma_load_4d(smem + L::OFF_DO + st * L::TILE + p * L::PANEL + hb * 8192, &tmdO, &qo_full[st], 64 * p, hq,
                         base + 64 * (i0 + hb), bc);
         for (int hb = 0; hb < nl; ++hb) {
@@ -260,7 +272,7 @@ __global__ void __launch_bounds__(448, 1)
         mbar_arrive_expect_tx(&qq_full[st], L::TILE + nl * 256);
         issued_q = m + 1;
         for (int hb = 0; hb < 2; ++hb)
-          for (int p = 0; p < 2; ++p)
+          for (int p = 0; p < L::DP; ++p)
             tma_load_4d(smem + L::OFF_Q + st * L::TILE + p * L::PANEL + hb * 8192, &tmQ, &qq_full[st], 64 * p, hq,
                         base + 64 * (i0 + hb), bc);
         for (int hb = 0; hb < nl; ++hb) {
@@ -292,12 +304,13 @@ __global__ void __launch_bounds__(448, 1)
     {
       const uint32_t leader = elect_one();
       constexpr uint32_t idesc_kk = idesc_bf16(128, 128, false, false);   // S^T, dP^T
-      constexpr uint32_t idesc_kmn = idesc_bf16(128, 128, false, true);   // dV (A in TMEM), dK
+      constexpr uint32_t idesc_kmn = idesc_bf16(128, D, false, true);     // dV (A in TMEM), dK
       constexpr uint32_t idesc_mnmn = idesc_bf16(128, 128, true, true);   // dQ^T
       // Descriptor bases (the start field moves by 16-byte units per k-step).
       // K-major operands advance 32 bytes per k-step inside a 64-column panel
       // and jump a panel every four; MN-major ones advance 16 rows (2048 bytes)
-      // and reach their second 64-element half through the leading offset.
+      // and reach their second 64-element half through the leading offset (at
+      // head dim 64, K^T's second half is the unread upper half of dQ^T).
       const uint64_t dK_k = sdesc_sw128(sbase + L::OFF_K, 16, 1024);
       const uint64_t dV_k = sdesc_sw128(sbase + L::OFF_V, 16, 1024);
       const uint64_t dK_mn = sdesc_sw128(sbase + L::OFF_K, L::PANEL, 1024);
@@ -317,14 +330,14 @@ __global__ void __launch_bounds__(448, 1)
       auto issue_s = [&](int n) {
         const uint64_t q = q_k(n);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
+        for (int kk = 0; kk < D / 16; ++kk)
           tc_mma_ss_if(leader, tmem + L::T_RS, dK_k + kofs(kk), q + kofs(kk), idesc_kk, kk > 0 ? 1u : 0u);
       };
       // dP^T(n) = V dO(n)^T into R_d.
       auto issue_dp = [&](int n) {
         const uint64_t o = o_k(n);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
+        for (int kk = 0; kk < D / 16; ++kk)
           tc_mma_ss_if(leader, tmem + L::T_RD, dV_k + kofs(kk), o + kofs(kk), idesc_kk, kk > 0 ? 1u : 0u);
       };
       // dV += P^T(n) dO(n); P^T of query columns [64 hf, +64) sits in R_s
@@ -556,7 +569,7 @@ __global__ void __launch_bounds__(448, 1)
     }
 
     // ------------------------------------------------------------ dK, dV epilogue
-    // Warp (quarter, half) writes rows of its quarter, columns [64 half, +64).
+    // Warp (quarter, half) writes rows of its quarter, columns [D/2 half, +D/2).
     bool ok = (n == NT) && !*abort_flag;
     if (ok) ok = mbar_wait(acc_done, 0, abort_flag, err, kErrBwdWait);
     ok = __all_sync(0xffffffffu, ok);
@@ -570,8 +583,8 @@ __global__ void __launch_bounds__(448, 1)
         const float mul = which == 0 ? 1.f : prm.scale;
         float* dst = (which == 0 ? prm.dv_f32 : prm.dk_f32) + (((size_t)lin0 + krow) * prm.Hkv + h) * L::D;
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int col = c0 + 32 * q;
+        for (int q = 0; q < D / 64; ++q) {
+          const int col = (D / 2) * hf + 32 * q;
           uint32_t o[32];
           tmem_ld32(t_lane + tcol + col, o);
           if (kvb >= 0) {
@@ -591,15 +604,16 @@ __global__ void __launch_bounds__(448, 1)
       for (int which = 0; which < 2; ++which) {
         const uint32_t tcol = which == 0 ? L::T_DV : L::T_DK;
         const float mul = which == 0 ? 1.f : prm.scale;
-        const uint32_t panel = sbase + (which == 0 ? L::OFF_V : L::OFF_K) + (uint32_t)hf * L::PANEL;
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
+        for (int q = 0; q < D / 64; ++q) {
+          const int col = (D / 2) * hf + 32 * q;  // 32 columns: four 16-byte chunks of a panel row
+          const uint32_t panel = sbase + (which == 0 ? L::OFF_V : L::OFF_K) + (uint32_t)(col >> 6) * L::PANEL;
           uint32_t o[32];
-          tmem_ld32(t_lane + tcol + c0 + 32 * q, o);
+          tmem_ld32(t_lane + tcol + col, o);
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             const float* f = reinterpret_cast<const float*>(&o[8 * q4]);
-            st_shared_v4(panel + sw128_offset(r, 4 * q + q4), pack_bf16x2(f[0] * mul, f[1] * mul),
+            st_shared_v4(panel + sw128_offset(r, ((col & 63) >> 3) + q4), pack_bf16x2(f[0] * mul, f[1] * mul),
                          pack_bf16x2(f[2] * mul, f[3] * mul), pack_bf16x2(f[4] * mul, f[5] * mul),
                          pack_bf16x2(f[6] * mul, f[7] * mul));
           }
@@ -610,7 +624,7 @@ __global__ void __launch_bounds__(448, 1)
     named_bar_sync(1, 256);
     if (threadIdx.x == 0 && ok && !prm.grad_f32) {
       for (int hb = 0; hb < (ky >= 0 ? 2 : 1); ++hb)
-        for (int p = 0; p < 2; ++p) {
+        for (int p = 0; p < L::DP; ++p) {
           tma_store_4d(&tmdV, smem + L::OFF_V + p * L::PANEL + hb * 8192, 64 * p, h, base + 64 * kload[hb], bc);
           tma_store_4d(&tmdK, smem + L::OFF_K + p * L::PANEL + hb * 8192, 64 * p, h, base + 64 * kload[hb], bc);
         }
@@ -621,11 +635,12 @@ __global__ void __launch_bounds__(448, 1)
     // ------------------------------------------------------------ dQ drain warps 10-13
     // Thread = dQ^T row d (TMEM lane); a warp's 32 lanes hit 32 consecutive dQ
     // elements of one query row, so every reduction below is one coalesced
-    // 128-byte request.
+    // 128-byte request. At head dim 64 the warps of lane quarters 0 and 1
+    // drain; the other two hold no dQ^T rows and stop here.
     const int quarter = warp & 3;
     const int d = quarter * 32 + lane;
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
-    for (int n = 0; n < NT; ++n) {  // n: global step
+    for (int n = 0; n < NT && 32 * quarter < D; ++n) {  // n: global step
       const int hq = GQA ? h * G + n / N : h;  // query head
       const int i0 = step_block(n);
       const bool second = i0 + 1 <= last;  // the step's second query block is in the list range
@@ -674,21 +689,28 @@ __global__ void __launch_bounds__(448, 1)
   }
 }
 
+template <int D, bool GQA>
+static cudaError_t launch_bwd128_impl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                      const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv,
+                                      const BwdParams& prm, int B, cudaStream_t stream) {
+  using L = Bwd128Layout<D>;
+  cudaError_t e = cudaFuncSetAttribute(lg_bwd128_kernel<D, GQA>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+  if (e != cudaSuccess) return e;
+  dim3 grid(prm.nkt * prm.Hkv, B);
+  lg_bwd128_kernel<D, GQA><<<grid, 448, L::ALLOC, stream>>>(tq, tk, tv, tdo, tdk, tdv, prm);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_bwd128(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                           const CUtensorMap& tdk, const CUtensorMap& tdv, const BwdParams& prm, int B,
                           cudaStream_t stream) {
-  using L = Bwd128Layout;
-  static_assert(L::BYTES <= L::ALLOC, "shared memory budget");
   const bool gqa = prm.H != prm.Hkv;
-  cudaError_t e = cudaFuncSetAttribute(gqa ? lg_bwd128_kernel<true> : lg_bwd128_kernel<false>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
-  if (e != cudaSuccess) return e;
-  dim3 grid(prm.nkt * prm.Hkv, B);
-  if (gqa)
-    lg_bwd128_kernel<true><<<grid, 448, L::ALLOC, stream>>>(tq, tk, tv, tdo, tdk, tdv, prm);
-  else
-    lg_bwd128_kernel<false><<<grid, 448, L::ALLOC, stream>>>(tq, tk, tv, tdo, tdk, tdv, prm);
-  return cudaGetLastError();
+  if (prm.D == 64)
+    return gqa ? launch_bwd128_impl<64, true>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream)
+               : launch_bwd128_impl<64, false>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
+  if (prm.D != 128) return cudaErrorInvalidValue;
+  return gqa ? launch_bwd128_impl<128, true>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream)
+             : launch_bwd128_impl<128, false>(tq, tk, tv, tdo, tdk, tdv, prm, B, stream);
 }
 
 }  // namespace lg

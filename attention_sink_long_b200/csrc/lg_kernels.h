@@ -43,7 +43,7 @@ struct BwdParams {
   float scale;       // softmax scale
   float scale_log2;  // scale * log2(e)
   int n_heavy;       // KV tiles scheduled first (for every head), ascending
-  int heavy[128];    // their tile indices; see lg_bwd_kernel's launch order
+  int heavy[128];    // their tile indices; see lg_bwd128_kernel's launch order
   int split_lo;      // 1: P and dS also enter dV / dK as bf16 residuals (GQA groups)
   int grad_f32;      // 1: dK / dV written as fp32 straight from the accumulators
   float* dk_f32;     // [B, S, Hkv, D] when grad_f32
@@ -59,7 +59,8 @@ cudaError_t launch_bwd_pre(const void* o, int o_f32, const void* dout, float* de
 cudaError_t launch_bwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& tdo, const CUtensorMap& tdk, const CUtensorMap& tdv, const BwdParams& prm,
                        int B, cudaStream_t stream);
-// Head dim 128, H == Hkv: 128-row query steps, every MMA M = N = 128.
+// Head dims 64 and 128, with or without query-head groups: 128-row KV tiles
+// (two 64-row blocks) and 128-row query steps.
 cudaError_t launch_bwd128(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                           const CUtensorMap& tdk, const CUtensorMap& tdv, const BwdParams& prm, int B,
                           cudaStream_t stream);

@@ -71,6 +71,13 @@ SMALL = [
     (2, 640, 2, 2, 128, lg.Pattern.full(64), torch.float32),        # dense causal, odd 128-row step count
     (1, 1024, 2, 2, 128, lg.Pattern(64, 1, 4, 0), torch.bfloat16),  # attention sink at head dim 128, bf16 O
     (1, 512, 8, 1, 128, lg.Pattern(64, 1, 2, 0), torch.float32),    # 8 query heads per KV head
+    # head dim 64 on the same 128-row-step kernel
+    (1, 192, 2, 2, 64, lg.Pattern(64, 1, 1, 0), torch.float32),     # ragged 64-row tail KV tile
+    (1, 64, 1, 1, 64, lg.Pattern(64, 1, 1, 0), torch.float32),      # a single block
+    (1, 2048, 2, 2, 64, lg.Pattern(64, 1, 16, 4), torch.float32),   # sink + window + strided blocks
+    (1, 1280, 2, 2, 64, lg.Pattern(64, 0, 1, 0), torch.float32),    # diagonal only
+    (2, 640, 2, 2, 64, lg.Pattern.full(64), torch.bfloat16),        # dense causal, odd 128-row step count
+    (1, 512, 8, 1, 64, lg.Pattern(64, 1, 2, 0), torch.float32),     # 8 query heads per KV head
 ]
 
 
@@ -155,11 +162,11 @@ def test_bwd_128k_sampled(pat):
         assert_close(f"dV h{h}", dv[0, krows, h].cpu().numpy(), rdv)
 
 
-def _gqa_sampled(S, H, Hkv, pat, qblocks, kvblocks):
+def _gqa_sampled(S, H, Hkv, pat, qblocks, kvblocks, D=128):
     """O and dQ rows of sampled query blocks and dK / dV rows of sampled KV
     blocks against the oracle, which sums dK / dV over the query heads of the
     KV head (bf16 O as in training)."""
-    B, D = 1, 128
+    B = 1
     op = oracle.Pattern(*pat)
     G = H // Hkv
     dev = torch.device("cuda")
@@ -208,3 +215,9 @@ def test_gqa_64k_block_sparse_sampled():
     nqb = 65536 // 64
     _gqa_sampled(65536, 8, 2, lg.Pattern(64, 1, 16, 32), (0, 33, nqb // 2 + 5, nqb - 1),
                  (0, 32, nqb // 2, nqb // 2 + 7, nqb - 1))
+
+
+def test_d64_32k_sampled():
+    """The head-dim-64 workload bench.py times: 32K sink+window, H32, D64."""
+    nqb = 32768 // 64
+    _gqa_sampled(32768, 32, 32, lg.Pattern(64, 1, 64, 0), (0, 5, nqb // 2, nqb - 1), (0, 1, nqb // 3, nqb - 1), D=64)

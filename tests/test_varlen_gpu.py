@@ -134,11 +134,12 @@ def run_varlen_fwd_bwd(pat, q, k, v, do, cu, max_len, scale, odt=torch.float32, 
 
 
 BWD_CASES = [
-    # lens, H, Hkv, D, pattern, O dtype: both backward kernels (head dim 128 with H == Hkv; GQA / head dim 64)
+    # lens, H, Hkv, D, pattern, O dtype: head dims 128 and 64, with and without query-head groups
     ([192, 64, 512, 1024, 320], 2, 2, 128, (64, 1, 4, 0), torch.float32),
     ([256, 640, 128], 2, 2, 128, (64, 1, 2, 4), torch.float32),
     ([384, 64, 448], 4, 2, 128, (64, 0, 2, 3), torch.float32),
     ([320, 192, 576], 2, 1, 64, (64, 0, 2**31 - 1, 0), torch.float32),
+    ([192, 64, 512, 1024, 320], 2, 2, 64, (64, 1, 4, 0), torch.float32),
     ([1024, 512], 2, 2, 128, (64, 1, 4, 0), torch.bfloat16),
 ]
 
