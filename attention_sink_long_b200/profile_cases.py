@@ -12,6 +12,8 @@ heads for the prefill kernels and with the batch for decode and hand-off):
   fwd_pair     B1 H16 S16384 D128 full causal, on the CTA-pair forward (lg_sparse_attn_fwd_pair)
   bwd_sw       B1 H8 S32768 D128 sink+window backward  (1/4 of the 32K H32 backward)
   bwd_gqa      B1 H8 Hkv2 S32768 D128 sink+window      (1/4 of the 32K H32 Hkv8 backward)
+  fwd_d64      B1 H16 S16384 D64 sink+window           (1/4 of the 32K H32 head-dim-64 forward)
+  bwd_d64      B1 H8 S32768 D64 sink+window backward   (1/4 of the 32K H32 head-dim-64 backward)
   decode       B32 H32 D128, 4160 cached rows          (the sparse-layer decode itself)
   decode_full  B1 H32 D128, 131072 cached rows         (1/32 of the full-layer decode)
   decode_gqa   B32 H32 Hkv8 D128, 4160 cached rows     (the grouped-query decode itself)
@@ -27,29 +29,31 @@ import attention_sink_long_b200 as lg
 import synthetic_inputs as si
 
 SW, FULL, BS = (64, 1, 64, 0), (64, 0, 2**31 - 1, 0), (64, 1, 16, 32)
-CASES = ("fwd_dense", "fwd_sw", "fwd_bs", "fwd_pair", "bwd_sw", "bwd_gqa", "decode", "decode_full", "decode_gqa", "handoff")
+CASES = ("fwd_dense", "fwd_sw", "fwd_bs", "fwd_pair", "fwd_d64", "bwd_sw", "bwd_gqa", "bwd_d64", "decode", "decode_full",
+         "decode_gqa", "handoff")
 
 
 def run(case: str) -> None:
     d = torch.device("cuda")
-    sc = 1 / math.sqrt(128)
+    D = 64 if case.endswith("_d64") else 128
+    sc = 1 / math.sqrt(D)
     if case.startswith("fwd"):
-        pat = {"fwd_dense": FULL, "fwd_sw": SW, "fwd_bs": BS, "fwd_pair": FULL}[case]
+        pat = {"fwd_dense": FULL, "fwd_sw": SW, "fwd_bs": BS, "fwd_pair": FULL, "fwd_d64": SW}[case]
         S, H = (131072, 8) if case == "fwd_bs" else (16384, 16)
-        q, k, v = si.prefill_inputs_device(1, S, H, H, 128, d)
+        q, k, v = si.prefill_inputs_device(1, S, H, H, D, d)
         o = torch.empty_like(q)
         lse = torch.empty(1, H, S, device=d)
         fwd = lg.lg_sparse_attn_fwd_pair if case == "fwd_pair" else lg.lg_sparse_attn_fwd
         for _ in range(3):
             fwd(pat, q, k, v, o, lse, sc)
-    elif case in ("bwd_sw", "bwd_gqa"):
-        H, Hkv = (8, 8) if case == "bwd_sw" else (8, 2)
-        q, k, v, do = si.prefill_inputs_device(1, 32768, H, Hkv, 128, d, with_dout=True)
+    elif case in ("bwd_sw", "bwd_gqa", "bwd_d64"):
+        H, Hkv = (8, 2) if case == "bwd_gqa" else (8, 8)
+        q, k, v, do = si.prefill_inputs_device(1, 32768, H, Hkv, D, d, with_dout=True)
         o = torch.empty_like(q)
         lse = torch.empty(1, H, 32768, device=d)
         lg.lg_sparse_attn_fwd(SW, q, k, v, o, lse, sc)
         g = [torch.empty_like(t) for t in (q, k, v)]
-        w = torch.empty(lg.lg_sparse_attn_bwd_workspace(SW, 1, 32768, H, Hkv, 128), dtype=torch.uint8, device=d)
+        w = torch.empty(lg.lg_sparse_attn_bwd_workspace(SW, 1, 32768, H, Hkv, D), dtype=torch.uint8, device=d)
         for _ in range(3):
             lg.lg_sparse_attn_bwd(SW, q, k, v, o, do, lse, *g, sc, w)
     elif case.startswith("decode"):
