@@ -49,6 +49,14 @@ SMALL = [
     (1, 576, 2, 2, 128, lg.Pattern(64, 1, 2, 0)),
     (2, 896, 4, 4, 128, lg.Pattern(64, 0, 3, 0)),
     (1, 1536, 4, 1, 128, lg.Pattern(64, 3, 2, 5)),
+    # Head dim 64: ragged tail, a single block, strided blocks, diagonal only, query-head
+    # groups, odd unions.
+    (1, 192, 2, 2, 64, lg.Pattern(64, 1, 1, 0)),
+    (1, 64, 1, 1, 64, lg.Pattern(64, 1, 1, 0)),
+    (1, 2048, 2, 2, 64, lg.Pattern(64, 1, 16, 4)),
+    (1, 1280, 2, 2, 64, lg.Pattern(64, 0, 1, 0)),
+    (1, 640, 2, 1, 64, lg.Pattern(64, 2, 3, 0)),
+    (2, 896, 4, 4, 64, lg.Pattern(64, 0, 3, 0)),
 ]
 
 
@@ -66,6 +74,25 @@ def test_fwd_matches_oracle_small(B, S, H, Hkv, D, pat):
     assert_close("O fp32", o32.cpu().numpy(), ro)
     assert torch.equal(lse32, lse)
     assert torch.equal(o32.to(torch.bfloat16), o)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_fwd_lazy_rescale_with_growing_scores(D):
+    """Keys whose scale grows along the sequence push each row's running max up
+    by more than 2^8 from one KV chunk to the next, so O is rescaled at nearly
+    every chunk, at both head dims. Such rows are carried by
+    a few keys, so the bf16 rounding of their P (2^-9 relative) no longer
+    averages out; V is scaled by 1/4 to keep that rounding well inside the
+    bound -- the growth of the scores, set by K alone, is unchanged."""
+    B, S, H = 1, 1024, 2
+    q, k, v = si.prefill_inputs(B, S, H, H, D)
+    k = (k.float() * torch.linspace(1.0, 60.0, S).view(1, S, 1, 1)).to(torch.bfloat16)
+    v = (v.float() * 0.25).to(torch.bfloat16)
+    scale = 1.0 / math.sqrt(D)
+    o, lse = run_fwd(lg.Pattern.full(64), q.cuda(), k.cuda(), v.cuda(), scale, torch.float32)
+    ro, rlse = oracle.attention_forward(q, k, v, oracle.Pattern(*lg.Pattern.full(64)), scale)
+    assert_close("O fp32", o.cpu().numpy(), ro)
+    assert_lse("LSE", lse.cpu().numpy(), rlse)
 
 
 def test_fwd_repeatable():
@@ -157,3 +184,20 @@ def test_fwd_pair_full_size_sampled(name, S, pat):
         ro, rl = oracle.attention_rows(qh, kh, vh, rows, op, scale)
         assert_close(f"{name} pair O h{h}", o[0, rows, h].float().cpu().numpy(), ro)
         assert_lse(f"{name} pair LSE h{h}", lse[0, h, rows].cpu().numpy(), rl)
+
+
+def test_fwd_head_dim_64_full_size_sampled():
+    """The head-dim-64 workload bench.py times: 32K sink+window, B1 H32 D64."""
+    B, S, H, D = 1, 32768, 32, 64
+    pat = lg.Pattern(64, 1, 64, 0)
+    dev = torch.device("cuda")
+    q, k, v = si.prefill_inputs_device(B, S, H, H, D, dev)
+    scale = 1.0 / math.sqrt(D)
+    o, lse = run_fwd(pat, q, k, v, scale)
+    rows = np.concatenate([np.arange(b * 64, (b + 1) * 64) for b in sampled_blocks(S // 64)])
+    op = oracle.Pattern(*pat)
+    for h in (0, H - 1):
+        qh, kh, vh = (t[0, :, h].float().cpu().numpy() for t in (q, k, v))
+        ro, rl = oracle.attention_rows(qh, kh, vh, rows, op, scale)
+        assert_close(f"D64 O h{h}", o[0, rows, h].float().cpu().numpy(), ro)
+        assert_lse(f"D64 LSE h{h}", lse[0, h, rows].cpu().numpy(), rl)
