@@ -398,12 +398,62 @@ lg_status_t lg_sparse_attn_fwd_varlen(const lg_pattern_t* p, const void* q, cons
 }
 
 // ---------------------------------------------------------------- backward
+namespace {
+
+// Heavy KV tiles of the backward (query-list length above twice the median,
+// e.g. the sink tile, seen by every query; at most 128), and, when a head has
+// exactly one, how its walk splits into chunks about as long as a median tile.
+struct HeavyPlan {
+  int n_heavy = 0;
+  int heavy[128];
+  int n_chunks = 0;     // 0: not split
+  int chunk_steps = 0;  // 128-row query steps per chunk
+};
+
+HeavyPlan heavy_plan(const lg_pattern_t& p, int nqb, int nkt) {
+  HeavyPlan hp;
+  std::vector<int> counts(nkt);
+  const lg::BlockPairing bp(p, nqb);
+  for (int t = 0; t < nkt; ++t) {
+    int x, y;
+    bp.pair(t, &x, &y);
+    const int first = y >= 0 ? imin(x, y) : x;
+    const int last = y >= 0 ? imax(bp.reach(x), bp.reach(y)) : bp.reach(x);
+    counts[t] = last - first + 1;
+  }
+  std::vector<int> sorted_counts(counts);
+  std::nth_element(sorted_counts.begin(), sorted_counts.begin() + nkt / 2, sorted_counts.end());
+  const int median = sorted_counts[nkt / 2];
+  for (int t = 0; t < nkt && hp.n_heavy < 128; ++t)
+    if (counts[t] > 2 * median) hp.heavy[hp.n_heavy++] = t;
+  if (hp.n_heavy == 1) {
+    const int steps = (counts[hp.heavy[0]] + 1) / 2;
+    const int ch = imax((median + 1) / 2, 16);
+    if (steps > ch) {
+      hp.chunk_steps = ch;
+      hp.n_chunks = (steps + ch - 1) / ch;
+    }
+  }
+  return hp;
+}
+
+// Bytes of the split heavy tile's partials and tickets for a (B, S) call.
+size_t heavy_part_bytes(const lg_pattern_t& p, int B, int S, int Hkv, int D) {
+  const HeavyPlan hp = heavy_plan(p, S / 64, (S + 127) / 128);
+  if (hp.n_chunks == 0) return 0;
+  return round256((size_t)B * Hkv * hp.n_chunks * 2 * 128 * D * sizeof(float)) +
+         round256((size_t)B * Hkv * sizeof(unsigned int));
+}
+
+}  // namespace
+
 lg_status_t lg_sparse_attn_bwd_workspace(const lg_pattern_t* p, int32_t B, int32_t S, int32_t H, int32_t Hkv,
                                          int32_t D, size_t* bytes) {
   lg_status_t st = check_prefill_shape(p, B, S, H, Hkv, D);
   if (st != LG_OK) return st;
   if (bytes == nullptr) return LG_ERR_INVALID_ARG;
-  *bytes = round256((size_t)B * H * S * D * sizeof(float)) + 2 * round256((size_t)B * H * S * sizeof(float));
+  *bytes = round256((size_t)B * H * S * D * sizeof(float)) + 2 * round256((size_t)B * H * S * sizeof(float)) +
+           heavy_part_bytes(*p, B, S, Hkv, D);
   return LG_OK;
 }
 
@@ -466,24 +516,23 @@ static lg_status_t bwd_common(const lg_pattern_t* p, const void* q, const void* 
   prm.max_len = max_len;
   prm.scale = scale;
   prm.scale_log2 = scale * 1.4426950408889634f;
-  // Heavy KV tiles: query-list length above twice the median (e.g. the sink
-  // tile, seen by every query). Scheduled first; at most 128 of them.
+  // Heavy KV tiles (see heavy_plan); with one per head, in a fixed-length
+  // batch, its walk is split into chunks (the packed-sequence call, whose
+  // workspace query cannot size per-sequence partials, keeps one CTA).
   {
-    std::vector<int> counts(prm.nkt);
-    const lg::BlockPairing bp(*p, prm.nqb);
-    for (int t = 0; t < prm.nkt; ++t) {
-      int x, y;
-      bp.pair(t, &x, &y);
-      const int first = y >= 0 ? imin(x, y) : x;
-      const int last = y >= 0 ? imax(bp.reach(x), bp.reach(y)) : bp.reach(x);
-      counts[t] = last - first + 1;
+    const HeavyPlan hp = heavy_plan(*p, prm.nqb, prm.nkt);
+    prm.n_heavy = hp.n_heavy;
+    for (int t = 0; t < hp.n_heavy; ++t) prm.heavy[t] = hp.heavy[t];
+    if (!varlen && hp.n_chunks > 0) {
+      prm.n_chunks = hp.n_chunks;
+      prm.chunk_steps = hp.chunk_steps;
+      char* w = reinterpret_cast<char*>(lse2) + round256((size_t)Bm * H * S * 4);
+      prm.hk_part = reinterpret_cast<float*>(w);
+      w += round256((size_t)Bm * Hkv * hp.n_chunks * 2 * 128 * D * sizeof(float));
+      prm.hk_ticket = reinterpret_cast<unsigned int*>(w);
+      st = cuda_status(cudaMemsetAsync(prm.hk_ticket, 0, (size_t)Bm * Hkv * sizeof(unsigned int), s));
+      if (st != LG_OK) return st;
     }
-    std::vector<int> sorted_counts(counts);
-    std::nth_element(sorted_counts.begin(), sorted_counts.begin() + prm.nkt / 2, sorted_counts.end());
-    const int median = sorted_counts[prm.nkt / 2];
-    prm.n_heavy = 0;
-    for (int t = 0; t < prm.nkt && prm.n_heavy < 128; ++t)
-      if (counts[t] > 2 * median) prm.heavy[prm.n_heavy++] = t;
   }
   // dK and dV of a KV head sum over its H / Hkv query heads, so their size
   // grows with the group; the bf16 residuals of P and dS then keep the bf16

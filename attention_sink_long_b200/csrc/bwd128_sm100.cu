@@ -126,6 +126,7 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t* acc_done = s_full + 7;         // every MMA complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 8);  // this chunk sums the partials
   const float* s_lse = reinterpret_cast<const float*>(smem + L::OFF_LSE);
   const float* s_del = reinterpret_cast<const float*>(smem + L::OFF_DEL);
 
@@ -162,9 +163,30 @@ __global__ void __launch_bounds__(448, 1)
   // the 128K block-sparse {64,1,16,32} backward: 22.0 ms against 24.3-26.5;
   // at 32K, where each tile's own order hits L2 anyway, the change was within
   // +-4 %). Otherwise the heavy tiles run interleaved across heads, ascending.
+  // When each head has a single heavy tile (the sink tile of a sink + window
+  // pattern) in a fixed-length batch, its walk is split instead into
+  // n_chunks ranges of query steps, one CTA each, placed evenly among the
+  // head's other tiles in launch order: each chunk then sweeps the query rows
+  // that the tiles running beside it read and reduce into, so Q, dO and the
+  // dQ accumulator come from L2 once rather than in a second sweep of their own.
   int u, h;
+  int chunk = -1;     // this CTA's chunk of the split heavy tile, or -1
   bool down = false;  // walk the query steps from the last to the first
-  {
+  if (prm.n_chunks > 0) {
+    const int nch = prm.n_chunks;
+    const int R = prm.nkt - 1 + nch;  // slots per head: the other tiles and the chunks
+    h = blockIdx.x / R;
+    const int sl = blockIdx.x % R;
+    // Chunk c takes slot floor(c R / nch); cnt = chunk slots at or before sl.
+    const int cnt = ((sl + 1) * nch + R - 1) / R;
+    if (cnt > 0 && ((cnt - 1) * R) / nch == sl) {
+      chunk = cnt - 1;
+      u = prm.heavy[0];
+    } else {
+      u = sl - cnt;
+      u += (u >= prm.heavy[0]) ? 1 : 0;  // skip the heavy tile
+    }
+  } else {
     const int Lx = blockIdx.x;
     const int nh = prm.n_heavy;
     if (Lx < nh * prm.Hkv) {
@@ -198,16 +220,21 @@ __global__ void __launch_bounds__(448, 1)
   const int q_first = ky >= 0 ? imin(kx, ky) : kx;
   const int last = ky >= 0 ? imax(bp.reach(kx), bp.reach(ky)) : bp.reach(kx);
   const int N = (last - q_first + 2) / 2;  // 128-row query steps (the last one may hold one block)
+  // The query steps this CTA walks: [t0, t0 + NQ) (all N, or one chunk).
+  const int t0 = chunk >= 0 ? chunk * prm.chunk_steps : 0;
+  const int NQ = chunk >= 0 ? imin(prm.chunk_steps, N - t0) : N;
+  if (NQ <= 0) return;  // (a chunk past the tile's last step: none with a fixed-length batch)
   // With query-head groups the CTA walks every query head of its KV head:
-  // step m is query step m % N of query head h * G + m / N, and dK / dV
+  // step m is query step t0 + m % NQ of query head h * G + m / NQ, and dK / dV
   // accumulate over the whole group.
   const int G = GQA ? prm.H / prm.Hkv : 1;
-  const int NT = G * N;
+  const int NT = G * NQ;
   // First query block of step m (of its query head), in the tile's walk order.
   auto step_block = [&](int m) -> int {
-    const int t = GQA ? m % N : m;
+    const int t = t0 + (GQA ? m % NQ : m);
     return q_first + 2 * (down ? N - 1 - t : t);
   };
+  auto step_head = [&](int m) -> int { return GQA ? h * G + m / NQ : h; };
   unsigned int* err = prm.err;
 
   if (threadIdx.x == 0) {
@@ -251,7 +278,7 @@ __global__ void __launch_bounds__(448, 1)
       for (int m = 0; m < NT; ++m) {
         const int st = m & 1;
         const uint32_t use = (uint32_t)(m >> 1);
-        const int hq = GQA ? h * G + m / N : h;  // query head
+        const int hq = step_head(m);  // query head
         const int i0 = step_block(m);
         // Both 64-row halves always load (rows past the sequence arrive as
         // zeros), so a stage never holds stale operands; LSE / Delta only
@@ -451,7 +478,7 @@ __global__ void __launch_bounds__(448, 1)
     const uint32_t t_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const float sl2 = prm.scale_log2;
     int n = 0;
-    for (; n < NT; ++n) {  // n: global step (query head h * G + n / N)
+    for (; n < NT; ++n) {  // n: step of this CTA (query head step_head(n))
       const int st = n & 1;
       const uint32_t par = (uint32_t)n & 1;
       const int i = step_block(n) + hf;  // this warp's query block
@@ -573,20 +600,82 @@ __global__ void __launch_bounds__(448, 1)
     bool ok = (n == NT) && !*abort_flag;
     if (ok) ok = mbar_wait(acc_done, 0, abort_flag, err, kErrBwdWait);
     ok = __all_sync(0xffffffffu, ok);
+    // A chunk of a split heavy tile hands its fp32 dV / dK partial to the
+    // workspace; the chunk that finishes last sums all of them, in chunk order
+    // (so the result does not depend on which one that is), and writes the
+    // gradients below; the others stop here.
+    const size_t per_chunk = (size_t)2 * 128 * L::D;
+    const int nch_live = chunk >= 0 ? (N + prm.chunk_steps - 1) / prm.chunk_steps : 0;
+    const float* part = nullptr;
+    if (chunk >= 0) {
+      float* mine = prm.hk_part + (((size_t)b * prm.Hkv + h) * prm.n_chunks + chunk) * per_chunk;
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int which = 0; which < 2; ++which)
+#pragma unroll
+          for (int q = 0; q < D / 64; ++q) {
+            const int col = (D / 2) * hf + 32 * q;
+            uint32_t o[32];
+            tmem_ld32(t_lane + (which == 0 ? L::T_DV : L::T_DK) + col, o);
+            float4* d4 = reinterpret_cast<float4*>(mine + ((size_t)which * 128 + r) * L::D + col);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              d4[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                  __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+          }
+      }
+      __threadfence();
+      named_bar_sync(1, 256);
+      if (threadIdx.x == 0) {
+        const unsigned int prev = ok ? atomicAdd(&prm.hk_ticket[b * prm.Hkv + h], 1u) : 0u;
+        *last_flag = (ok && prev == (unsigned int)(nch_live - 1)) ? 1 : 0;
+      }
+      named_bar_sync(1, 256);
+      ok = *last_flag != 0;
+      if (ok) {
+        __threadfence();
+        part = prm.hk_part + ((size_t)b * prm.Hkv + h) * prm.n_chunks * per_chunk;
+      }
+    }
+    // 32 columns of this thread's dV (which = 0) or dK row: from TMEM, or the
+    // sum of the chunks' partials.
+    auto acc_cols = [&](int which, int col, uint32_t (&o)[32]) {
+      if (part == nullptr) {
+        tmem_ld32(t_lane + (which == 0 ? L::T_DV : L::T_DK) + col, o);
+        return;
+      }
+      float a[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) a[e] = 0.f;
+      for (int c2 = 0; c2 < nch_live; ++c2) {
+        const float4* src =
+            reinterpret_cast<const float4*>(part + (size_t)c2 * per_chunk + ((size_t)which * 128 + r) * L::D + col);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float4 v = __ldcg(src + e);
+          a[4 * e] += v.x;
+          a[4 * e + 1] += v.y;
+          a[4 * e + 2] += v.z;
+          a[4 * e + 3] += v.w;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(a[e]);
+    };
     if (ok && prm.grad_f32) {
       // fp32 gradients: each thread stores its part of a KV row straight from TMEM.
       tc_fence_after();
       const int krow = kvb >= 0 ? 64 * kvb + (r & 63) : 0;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
-        const uint32_t tcol = which == 0 ? L::T_DV : L::T_DK;
         const float mul = which == 0 ? 1.f : prm.scale;
         float* dst = (which == 0 ? prm.dv_f32 : prm.dk_f32) + (((size_t)lin0 + krow) * prm.Hkv + h) * L::D;
 #pragma unroll
         for (int q = 0; q < D / 64; ++q) {
           const int col = (D / 2) * hf + 32 * q;
           uint32_t o[32];
-          tmem_ld32(t_lane + tcol + col, o);
+          acc_cols(which, col, o);
           if (kvb >= 0) {
             float4* d4 = reinterpret_cast<float4*>(dst + col);
 #pragma unroll
@@ -602,14 +691,13 @@ __global__ void __launch_bounds__(448, 1)
       tc_fence_after();
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
-        const uint32_t tcol = which == 0 ? L::T_DV : L::T_DK;
         const float mul = which == 0 ? 1.f : prm.scale;
 #pragma unroll
         for (int q = 0; q < D / 64; ++q) {
           const int col = (D / 2) * hf + 32 * q;  // 32 columns: four 16-byte chunks of a panel row
           const uint32_t panel = sbase + (which == 0 ? L::OFF_V : L::OFF_K) + (uint32_t)(col >> 6) * L::PANEL;
           uint32_t o[32];
-          tmem_ld32(t_lane + tcol + col, o);
+          acc_cols(which, col, o);
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             const float* f = reinterpret_cast<const float*>(&o[8 * q4]);
@@ -641,7 +729,7 @@ __global__ void __launch_bounds__(448, 1)
     const int d = quarter * 32 + lane;
     const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
     for (int n = 0; n < NT && 32 * quarter < D; ++n) {  // n: global step
-      const int hq = GQA ? h * G + n / N : h;  // query head
+      const int hq = step_head(n);  // query head
       const int i0 = step_block(n);
       const bool second = i0 + 1 <= last;  // the step's second query block is in the list range
       if (!__all_sync(0xffffffffu, mbar_wait(dq_full, (uint32_t)n & 1, abort_flag, err, kErrBwdWait))) break;
@@ -696,7 +784,8 @@ static cudaError_t launch_bwd128_impl(const CUtensorMap& tq, const CUtensorMap& 
   using L = Bwd128Layout<D>;
   cudaError_t e = cudaFuncSetAttribute(lg_bwd128_kernel<D, GQA>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
   if (e != cudaSuccess) return e;
-  dim3 grid(prm.nkt * prm.Hkv, B);
+  // With the heavy tile split, each head has its other nkt - 1 tiles and n_chunks chunks.
+  dim3 grid((prm.n_chunks > 0 ? prm.nkt - 1 + prm.n_chunks : prm.nkt) * prm.Hkv, B);
   lg_bwd128_kernel<D, GQA><<<grid, 448, L::ALLOC, stream>>>(tq, tk, tv, tdo, tdk, tdv, prm);
   return cudaGetLastError();
 }

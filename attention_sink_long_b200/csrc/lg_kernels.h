@@ -50,6 +50,15 @@ struct BwdParams {
   float* dv_f32;
   const int32_t* cu_seqlens = nullptr;  // device [B + 1] offsets of packed sequences (S = total rows), or nullptr
   int max_len = 0;                      // with cu_seqlens: the longest sequence (nkt covers it)
+  // The single heavy tile of each head split into n_chunks query ranges of
+  // chunk_steps 128-row steps, one CTA each (0: not split). Each chunk writes
+  // its fp32 dV / dK partial to hk_part [B, Hkv, n_chunks, 2, 128, D]; the
+  // last to finish (hk_ticket [B, Hkv], zero on entry) sums them in chunk
+  // order and writes the gradients.
+  int n_chunks = 0;
+  int chunk_steps = 0;
+  float* hk_part = nullptr;
+  unsigned int* hk_ticket = nullptr;
   unsigned int* err;
 };
 

@@ -220,7 +220,13 @@ lg_status_t lg_sparse_attn_fwd_varlen(const lg_pattern_t* pattern, const void* q
 /* Training backward                                                        */
 /* ------------------------------------------------------------------------ */
 
-/* Workspace bytes for lg_sparse_attn_bwd: fp32 dQ accumulator [B,H,S,D] plus Delta and LSE * log2(e) [B,H,S]. */
+/*
+ * Workspace bytes for lg_sparse_attn_bwd: fp32 dQ accumulator [B,H,S,D] plus
+ * Delta and LSE * log2(e) [B,H,S]; and, when each head has a single KV tile
+ * that far more queries see than the rest (the sink tile of a sink + window
+ * pattern), fp32 dV / dK partials of that tile's walk split into chunks
+ * [B,Hkv,chunks,2,128,D] and B*Hkv counters.
+ */
 lg_status_t lg_sparse_attn_bwd_workspace(const lg_pattern_t* pattern, int32_t B, int32_t S, int32_t H,
                                          int32_t Hkv, int32_t D, size_t* bytes);
 
@@ -235,6 +241,9 @@ lg_status_t lg_sparse_attn_bwd_workspace(const lg_pattern_t* pattern, int32_t B,
  * element type grad_dtype. P and dS enter the tensor-core products as bf16;
  * with query-head groups (H > Hkv) they also enter dV / dK as a bf16 hi + lo
  * pair (exact to fp32 accumulation), since those sums grow with the group.
+ * A single heavy KV tile per head (the sink tile) is walked by several CTAs,
+ * each over a range of query rows; its dV / dK are the sum of their fp32
+ * partials taken in a fixed order, so results do not vary from run to run.
  * workspace (device, 256-byte aligned) of at least the queried size; its
  * contents on entry do not matter.
  */

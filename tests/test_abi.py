@@ -162,6 +162,27 @@ def test_workspace_queries():
     assert lg.lg_sparse_decode_splits(2, 8, 8, 128, 100, 7) == 7
 
 
+def _r256(n):
+    return (n + 255) // 256 * 256
+
+
+def test_bwd_workspace_holds_split_sink_tile_partials():
+    """32K sink+window: the other KV tiles walk ~33 query steps (66 blocks), the
+    sink tile all 256, so its walk is split into ceil(256 / 33) = 8 chunks
+    whose fp32 dV / dK partials (2 x 128 x D each, per KV head) and one counter
+    per KV head join the workspace. Dense causal (no tile stands out) and the
+    block-sparse pattern (several heavy tiles per head) keep the base size."""
+    B, S, H, Hkv, D = 1, 32768, 32, 32, 128
+    base = _r256(B * H * S * D * 4) + 2 * _r256(B * H * S * 4)
+    ws = lg.lg_sparse_attn_bwd_workspace(lg.Pattern(64, 1, 64, 0), B, S, H, Hkv, D)
+    assert ws == base + _r256(B * Hkv * 8 * 2 * 128 * D * 4) + _r256(B * Hkv * 4)
+    assert lg.lg_sparse_attn_bwd_workspace(lg.Pattern.full(64), B, S, H, Hkv, D) == base
+    assert lg.lg_sparse_attn_bwd_workspace(lg.Pattern(64, 1, 16, 32), B, S, H, Hkv, D) == base
+    # short sequences: the sink tile's walk is no longer than one chunk, nothing is split
+    assert lg.lg_sparse_attn_bwd_workspace(lg.Pattern(64, 1, 4, 0), 1, 1024, 4, 4, 64) == \
+        _r256(1024 * 4 * 64 * 4) + 2 * _r256(4 * 1024 * 4)
+
+
 @pytest.mark.parametrize("shape,splits", [
     # one query head per KV head: 512-row pieces, halved while B * Hkv * splits < 1184
     ((32, 32, 32, 128, 4160), 9), ((1, 32, 32, 128, 4160), 65), ((32, 32, 32, 64, 4160), 5),

@@ -48,12 +48,16 @@ def run_fwd_bwd(pattern, q, k, v, do, scale, grad_dtype=torch.float32, o_dtype=t
     return dq, dk, dv
 
 
-def assert_bf16_rounding_of(name, got_bf16, ref_f32):
-    """got_bf16 equals ref_f32 rounded to bf16, within one bf16 ulp."""
+def assert_bf16_rounding_of(name, got_bf16, ref_f32, atol=0.0):
+    """got_bf16 equals ref_f32 rounded to bf16, within one bf16 ulp (plus atol,
+    for dQ: its terms arrive through fp32 atomic adds in an order that varies
+    between runs, so two runs' fp32 dQ differ by that rounding -- a few units
+    of 2^-24 of the terms' size -- which near a cancellation to zero is more
+    than a relative bf16 ulp; dK and dV are summed in a fixed order)."""
     r = ref_f32.to(torch.bfloat16).float()
     g = got_bf16.float()
     ulp = torch.where(r == 0, torch.full_like(r, 2.0 ** -133), torch.abs(r) * 2.0 ** -7)
-    bad = (torch.abs(g - r) > ulp * 1.0001).sum().item()
+    bad = (torch.abs(g - r) > ulp * 1.0001 + atol).sum().item()
     assert bad == 0, (name, bad)
 
 
@@ -78,6 +82,10 @@ SMALL = [
     (1, 1280, 2, 2, 64, lg.Pattern(64, 0, 1, 0), torch.float32),    # diagonal only
     (2, 640, 2, 2, 64, lg.Pattern.full(64), torch.bfloat16),        # dense causal, odd 128-row step count
     (1, 512, 8, 1, 64, lg.Pattern(64, 1, 2, 0), torch.float32),     # 8 query heads per KV head
+    # The sink tile's walk split into chunks (32 and 48 query steps against a chunk of 16):
+    # its dV / dK are summed from the chunks' partials.
+    (1, 4096, 2, 2, 128, lg.Pattern(64, 1, 4, 0), torch.float32),
+    (1, 6144, 4, 2, 64, lg.Pattern(64, 1, 2, 0), torch.float32),
 ]
 
 
@@ -92,7 +100,7 @@ def test_bwd_matches_oracle_small(B, S, H, Hkv, D, pat, odt):
     assert_close("dK", dk.cpu().numpy(), rdk)
     assert_close("dV", dv.cpu().numpy(), rdv)
     bq, bk, bv = run_fwd_bwd(pat, qd, kd, vd, dod, scale, torch.bfloat16, o_dtype=odt)
-    assert_bf16_rounding_of("dQ", bq, dq)
+    assert_bf16_rounding_of("dQ", bq, dq, atol=float(dq.abs().max()) * 2.0 ** -16)
     assert_bf16_rounding_of("dK", bk, dk)
     assert_bf16_rounding_of("dV", bv, dv)
 
@@ -136,7 +144,7 @@ def test_bwd_gqa_training_format_small(B, S, H, Hkv, D, pat):
     assert_close("dK", dk.cpu().numpy(), rdk)
     assert_close("dV", dv.cpu().numpy(), rdv)
     for name, b16, f32 in zip(("dQ", "dK", "dV"), grads[torch.bfloat16], grads[torch.float32]):
-        assert_bf16_rounding_of(name, b16, f32)
+        assert_bf16_rounding_of(name, b16, f32, atol=float(f32.abs().max()) * 2.0 ** -16 if name == "dQ" else 0.0)
 
 
 @pytest.mark.parametrize("pat", [lg.Pattern(64, 1, 64, 0), lg.Pattern(64, 1, 16, 32)],
@@ -221,3 +229,15 @@ def test_d64_32k_sampled():
     """The head-dim-64 workload bench.py times: 32K sink+window, H32, D64."""
     nqb = 32768 // 64
     _gqa_sampled(32768, 32, 32, lg.Pattern(64, 1, 64, 0), (0, 5, nqb // 2, nqb - 1), (0, 1, nqb // 3, nqb - 1), D=64)
+
+
+def test_bwd_split_sink_tile_is_deterministic():
+    """The sink tile's dV / dK are summed from its chunks' partials in chunk
+    order, whichever chunk finishes last: two runs give the same bits."""
+    B, S, H, D = 1, 8192, 4, 128
+    pat = lg.Pattern(64, 1, 16, 0)
+    q, k, v, do = si.prefill_inputs(B, S, H, H, D, with_dout=True)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    a = run_fwd_bwd(pat, qd, kd, vd, dod, 1.0 / math.sqrt(D))
+    b = run_fwd_bwd(pat, qd, kd, vd, dod, 1.0 / math.sqrt(D))
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
