@@ -40,6 +40,9 @@ if ROOT not in sys.path:
 
 METRIC = "sparse-attn fwd/bwd useful TFLOP/s & decode GB/s; % of B200 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# The B200 data-sheet figures (dense bf16, HBM3e), reported beside the measured
+# peaks for context; the measured fractions are the headline.
+NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 SINK_WINDOW = (64, 1, 64, 0)
 FULL = (64, 0, 2**31 - 1, 0)
 BLOCK_SPARSE = (64, 1, 16, 32)
@@ -637,6 +640,7 @@ def cuda_arm(args, rank, world, dist):
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4)}
         roof["peak_source"] = f"{peak_src} (copy bandwidth)"
+        roof["frac_nominal"] = round(achieved / NOMINAL_PEAKS["hbm_gbs"], 4)
     else:
         achieved = dflops / (dms * 1e-3) / 1e12
         pk = tensor_peak * 4 / 3 if dkind == "fwd_fp8qk" else tensor_peak
@@ -648,6 +652,8 @@ def cuda_arm(args, rank, world, dist):
         # The same kernel against the other measured figure, for context.
         other = peaks["bf16_tflops_sustained"] if pk == peaks["bf16_tflops"] else peaks["bf16_tflops"]
         roof["frac_" + ("sustained" if pk == peaks["bf16_tflops"] else "burst")] = round(achieved / other, 4)
+        nom = NOMINAL_PEAKS["bf16_tflops"] * (4 / 3 if dkind == "fwd_fp8qk" else 1)
+        roof["frac_nominal"] = round(achieved / nom, 4)
     roof["traffic"] = recorded_traffic(dname, args.workload)
     roof["kernel"] = dname
 
@@ -722,12 +728,14 @@ def part_row(kind, flops, nbytes, ms, peaks, tensor_peak):
     if kind.startswith("decode") or kind == "copy":
         r["gbs"] = round(nbytes / (ms * 1e-3) / 1e9, 1)
         r["frac_hbm"] = round(r["gbs"] / peaks["hbm_gbs"], 4)
+        r["frac_hbm_nominal"] = round(r["gbs"] / NOMINAL_PEAKS["hbm_gbs"], 4)
     elif kind == "fwd_fp8qk":
         # half of the FLOPs (S) at the fp8 rate, twice bf16: the mixed peak is 4/3 of bf16's
         r["frac_mixed_fp8_bf16_peak"] = round(r["useful_tflops"] / (tensor_peak * 4 / 3), 4)
     else:
         r["frac_bf16"] = round(r["useful_tflops"] / tensor_peak, 4)
         r["frac_bf16_sustained"] = round(r["useful_tflops"] / peaks["bf16_tflops_sustained"], 4)
+        r["frac_bf16_nominal"] = round(r["useful_tflops"] / NOMINAL_PEAKS["bf16_tflops"], 4)
         if kind == "bwd":
             # 10 D FLOP per pair counts the five GEMMs (S recomputed); 8 D leaves the recompute out.
             r["useful_tflops_8d"] = round(0.8 * r["useful_tflops"], 2)

@@ -53,6 +53,16 @@ def test_peak_choice():
     assert bench.pick_peak(peaks, 30.0, "hbm")[0] == 6500.0
 
 
+def test_rows_report_measured_and_nominal_fractions():
+    peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1650.0, "bf16_tflops_sustained": 1400.0}
+    r = bench.part_row("fwd", 8.25e12, 0, 10.0, peaks, 1650.0)  # 825 TFLOP/s
+    assert r["frac_bf16"] == 0.5 and r["frac_bf16_nominal"] == round(825 / 2250, 4)
+    b = bench.part_row("bwd", 8.25e12, 0, 10.0, peaks, 1650.0)
+    assert b["frac_bf16_8d"] == 0.4
+    d = bench.part_row("decode", 0, 4e9, 1.0, peaks, 1650.0)  # 4000 GB/s
+    assert d["frac_hbm"] == round(4000 / 6500, 4) and d["frac_hbm_nominal"] == 0.5
+
+
 def test_recorded_traffic_is_tied_to_kernel_sources(tmp_path, monkeypatch):
     assert bench.recorded_traffic("no such part", "step32k") is None
     with open(bench.TRAFFIC_FILE) as f:
