@@ -40,10 +40,11 @@
 //
 // MMA order (one thread; tcgen05 MMAs of one thread execute in order):
 //   S^T(0), dP^T(0), dV(0), S^T(1), then per step n:
-//   [dS(n) ready]  dK(n), dQ^T(n)    (dK first: Q(n)'s stage refills sooner;
-//                  with query-head groups dK's residual half -- which reads R_d
-//                  -- then dQ^T, then dK's shared-memory half, so the drain
-//                  starts 8 MMAs earlier: +3 % at four query heads per KV head)
+//   [dS(n) ready]  dQ^T(n), dK(n)    (dQ^T first: the drain, on the step's
+//                  critical chain, starts a GEMM earlier -- +2 % -- while Q(n)'s
+//                  stage refills a GEMM later; with query-head groups dK's
+//                  residual half, which reads R_d, must come before dQ^T and its
+//                  shared-memory half follows: +3 % at four query heads per KV head)
 //   [dQ^T(n) drained]  dP^T(n+1)
 //   [P(n+1) ready]  dV(n+1)          (dO(n+1)'s stage refills after it)
 //   [Q(n+2) loaded]  S^T(n+2)        (after dV(n+1), which reads P^T(n+1))
@@ -442,11 +443,12 @@ __global__ void __launch_bounds__(448, 1)
         const uint32_t par = (uint32_t)n & 1;
         if (!mbar_wait(ds_full, par, abort_flag, err, kErrBwdWait)) break;
         tc_fence_after();
-        // dK first: it is Q(n)'s last use, so the refill of that stage with
-        // Q(n+2) -- which S^T(n+2) waits for -- starts one GEMM earlier. With
-        // query-head groups dK's residual half must precede dQ^T (both use
-        // R_d) and its shared-memory half follows dQ^T, so the drain, on the
-        // step's critical chain, gets dQ^T 8 MMAs sooner.
+        // dQ^T first: the drain that reads it is on the step's critical chain
+        // (dQ^T(n) -> drain -> dP^T(n+1) -> dS(n+1)); dK, the last use of Q(n),
+        // follows, so that stage's refill with Q(n+2) starts a GEMM later --
+        // measured +2 % overall (interleaved A/B, 32K and 128K). With query-head
+        // groups dK's residual half must precede dQ^T (both use R_d) and its
+        // shared-memory half follows.
         if (GQA) {
           issue_dk_lo(n);
           issue_dq(n);
@@ -454,10 +456,10 @@ __global__ void __launch_bounds__(448, 1)
           issue_dk(n);
           tc_commit_if(leader, &qq_empty[n & 1]);
         } else {
-          issue_dk(n);
-          tc_commit_if(leader, &qq_empty[n & 1]);
           issue_dq(n);
           tc_commit_if(leader, dq_full);
+          issue_dk(n);
+          tc_commit_if(leader, &qq_empty[n & 1]);
         }
         tc_commit_if(leader, dss_free);
         if (n + 1 < NT) {
