@@ -86,6 +86,7 @@ SMALL = [
     # its dV / dK are summed from the chunks' partials.
     (1, 4096, 2, 2, 128, lg.Pattern(64, 1, 4, 0), torch.float32),
     (1, 6144, 4, 2, 64, lg.Pattern(64, 1, 2, 0), torch.float32),
+    (2, 4096, 2, 2, 64, lg.Pattern(64, 1, 4, 0), torch.float32),    # two batch rows, each split
 ]
 
 
