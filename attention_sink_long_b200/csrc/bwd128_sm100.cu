@@ -15,7 +15,10 @@
 // the window-only blocks pair in order), so both halves of the tile see nearly
 // the same query blocks -- and walks those query blocks two at a time: a
 // 128-row query step (with query-head groups, the steps of every query head
-// of the group in turn, dK and dV accumulating over all of them).
+// of the group in turn, dK and dV accumulating over all of them). The one KV
+// tile per head that far more queries see (the sink tile) is instead walked by
+// several CTAs, each over a range of query steps, whose fp32 dK / dV partials
+// the last of them sums (see the launch order below).
 // At head dim 128 every GEMM of a step is then an M = 128, N = 128 tcgen05
 // MMA -- the shape the tensor core runs at full rate (an N = 64 instruction
 // takes about as long as an N = 128 one):
