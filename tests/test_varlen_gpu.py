@@ -165,8 +165,9 @@ def test_varlen_bwd_matches_oracle_per_sequence(lens, H, Hkv, D, pat, odt):
 
 @pytest.mark.parametrize("H,Hkv,D", [(4, 4, 128), (4, 2, 64)])
 def test_varlen_bwd_equal_lengths_match_the_fixed_length_call(H, Hkv, D):
-    """dK / dV bit for bit (each written by one CTA); dQ to within the order of
-    its reduce-adds."""
+    """dK / dV bit for bit (each written by one CTA: at 768 rows the
+    fixed-length call does not split the sink tile's walk either); dQ to
+    within the order of its reduce-adds."""
     B, S = 3, 768
     pat = (64, 1, 4, 0)
     scale = 1.0 / math.sqrt(D)
