@@ -166,7 +166,7 @@ const char* lg_strerror(lg_status_t s) {
   return "unknown status";
 }
 
-int32_t lg_version(void) { return (2 << 16) | 0; }
+int32_t lg_version(void) { return (2 << 16) | 1; }
 
 // ---------------------------------------------------------------- pattern (host)
 lg_status_t lg_pattern_expand(const lg_pattern_t* p, int32_t seqlen, int32_t* row_ptr, int32_t* col, int64_t cap,
